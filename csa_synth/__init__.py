@@ -1,0 +1,190 @@
+"""Seeded synthetic inputs and layer shapes for the DeepSeek-V4 hybrid attention layer.
+
+This module is shared by the CUDA path's tests/bench and by the CPU oracle's tests.
+It holds sizes and random-number recipes only: no step of the method's arithmetic
+(pooling, scoring, selection, RoPE, softmax) lives here.
+
+Workload shapes follow the V4-Flash layer described on the pages:
+  * window 128, CSA ratio m=4 (overlapping windows), HCA ratio m'=128
+    (optimum-intel issue #1748, "What V4-Flash adds vs V3");
+  * head_dim 512 (HF transformers PR #45616, "Config inherits DeepseekV3Config");
+  * a single shared K=V head and a per-head sink (HF docs model_doc/deepseek_v4,
+    "Hybrid attention (section 2.3)").
+
+Value recipe (the same for every workload): q, kv, gate logits, q_I, k_I ~ N(0,1);
+indexer head weights w ~ N(0,1)/sqrt(H_I); sink logits ~ N(0,1) in fp32; every kv row
+(and every directly generated pool row) RMS-normalised, x / sqrt(mean(x^2) + 1e-6),
+in fp64 before rounding to the storage dtype.
+
+Seeds: tensor seed = 1000*workload + 100*layer + tensor_id, tensor ids in the order
+q, kv, gate, q_I, k_I, w, sink, pool.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Dict, List, Optional
+
+import torch
+
+TENSOR_IDS = {"q": 0, "kv": 1, "gate": 2, "q_I": 3, "k_I": 4, "w": 5, "sink": 6, "pool": 7}
+RMS_EPS = 1e-6
+
+
+@dataclasses.dataclass(frozen=True)
+class LayerSpec:
+    """Shape of one attention layer call.
+
+    kind: "csa" (compressed sparse: indexer + top-k), "hca" (heavily compressed: every
+    visible entry) or "sliding" (window only, no pool).
+    Query i sits at absolute position q_pos0 + i; raw kv row r at kv_pos0 + r.
+    decode=True means the pool and k_I are a resident cache (no compressor run).
+    """
+
+    name: str
+    dtype: str  # "f32" or "bf16"
+    B: int
+    S_q: int
+    S_kv: int
+    q_pos0: int
+    kv_pos0: int
+    H: int
+    D: int
+    R: int
+    base: float
+    W: int
+    m: int
+    P: int
+    kind: str
+    H_I: int = 0
+    d_I: int = 0
+    topk: int = 0
+    decode: bool = False
+    workload: int = 0
+    layer: int = 0
+
+    @property
+    def overlap(self) -> int:
+        return 1 if self.kind == "csa" else 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.D)
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    def seed(self, tensor: str) -> int:
+        return 1000 * self.workload + 100 * self.layer + TENSOR_IDS[tensor]
+
+
+def prefill(name, dtype, S, H, D, R, base, W, m, kind, H_I=0, d_I=0, topk=0, B=1,
+            workload=0, layer=0) -> LayerSpec:
+    P = 0 if kind == "sliding" else S // m
+    return LayerSpec(name=name, dtype=dtype, B=B, S_q=S, S_kv=S, q_pos0=0, kv_pos0=0,
+                     H=H, D=D, R=R, base=base, W=W, m=m, P=P, kind=kind, H_I=H_I,
+                     d_I=d_I, topk=topk, workload=workload, layer=layer)
+
+
+# The five workloads.  Bases: one RoPE base per layer, used for q, window keys, entries
+# and the output de-rotation; compressed layers use the slower 160000 base and the
+# sliding-only layer the main 10000 base (HF PR #45616 "compress_rope_parameters ...
+# rope_theta swapped"; mlx-lm PR #1797 "two rotation speeds").
+TINY_CSA = prefill("tiny_csa_f32", "f32", S=256, H=8, D=64, R=16, base=10000.0, W=32,
+                   m=4, kind="csa", H_I=4, d_I=32, topk=16, workload=0)
+CSA_PREFILL = prefill("csa_prefill_s8192", "bf16", S=8192, H=64, D=512, R=64,
+                      base=160000.0, W=128, m=4, kind="csa", H_I=64, d_I=128, topk=512,
+                      workload=1)
+HCA_PREFILL = prefill("hca_prefill_s65536", "bf16", S=65536, H=64, D=512, R=64,
+                      base=160000.0, W=128, m=128, kind="hca", workload=2)
+CSA_DECODE = LayerSpec(name="csa_decode_b64_ctx65536", dtype="bf16", B=64, S_q=1, S_kv=128,
+                       q_pos0=65535, kv_pos0=65408, H=64, D=512, R=64, base=160000.0,
+                       W=128, m=4, P=16384, kind="csa", H_I=64, d_I=128, topk=512,
+                       decode=True, workload=3)
+
+
+def mixed_stack(S: int = 131072) -> List[LayerSpec]:
+    """Four-layer long-context block: CSA, HCA, CSA, sliding-only."""
+    return [
+        prefill("mixed_l0_csa", "bf16", S=S, H=64, D=512, R=64, base=160000.0, W=128, m=4,
+                kind="csa", H_I=64, d_I=128, topk=512, workload=4, layer=0),
+        prefill("mixed_l1_hca", "bf16", S=S, H=64, D=512, R=64, base=160000.0, W=128, m=128,
+                kind="hca", workload=4, layer=1),
+        prefill("mixed_l2_csa", "bf16", S=S, H=64, D=512, R=64, base=160000.0, W=128, m=4,
+                kind="csa", H_I=64, d_I=128, topk=512, workload=4, layer=2),
+        prefill("mixed_l3_sliding", "bf16", S=S, H=64, D=512, R=64, base=10000.0, W=128,
+                m=4, kind="sliding", workload=4, layer=3),
+    ]
+
+
+WORKLOADS: Dict[int, List[LayerSpec]] = {
+    0: [TINY_CSA],
+    1: [CSA_PREFILL],
+    2: [HCA_PREFILL],
+    3: [CSA_DECODE],
+    4: mixed_stack(),
+}
+
+
+def _randn(shape, seed: int, device) -> torch.Tensor:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+
+
+def _rms_rows(x: torch.Tensor) -> torch.Tensor:
+    xd = x.double()
+    return xd / torch.sqrt(xd.pow(2).mean(dim=-1, keepdim=True) + RMS_EPS)
+
+
+def make_inputs(spec: LayerSpec, device="cpu") -> Dict[str, Optional[torch.Tensor]]:
+    """Seeded inputs for one layer, in the layer's storage dtype, on `device`.
+
+    q [B,S_q,H,D]; kv [B,S_kv,D]; gate [B,S_kv,D] (prefill) ; pool [B,P,D] (decode);
+    q_I [B,S_q,H_I,d_I]; w [B,S_q,H_I]; k_I [B,P,d_I] (CSA only); sink [H] fp32.
+    The random stream depends on the device type; callers compare both sides on one copy.
+    """
+    dt = spec.torch_dtype
+    out: Dict[str, Optional[torch.Tensor]] = {}
+    out["q"] = _randn((spec.B, spec.S_q, spec.H, spec.D), spec.seed("q"), device).to(dt)
+    out["kv"] = _rms_rows(_randn((spec.B, spec.S_kv, spec.D), spec.seed("kv"), device)).to(dt)
+    if spec.decode:
+        out["gate"] = None
+        out["pool"] = _rms_rows(_randn((spec.B, spec.P, spec.D), spec.seed("pool"), device)).to(dt)
+    else:
+        out["gate"] = _randn((spec.B, spec.S_kv, spec.D), spec.seed("gate"), device).to(dt)
+        out["pool"] = None
+    if spec.kind == "csa":
+        out["q_I"] = _randn((spec.B, spec.S_q, spec.H_I, spec.d_I), spec.seed("q_I"), device).to(dt)
+        out["k_I"] = _randn((spec.B, spec.P, spec.d_I), spec.seed("k_I"), device).to(dt)
+        out["w"] = (_randn((spec.B, spec.S_q, spec.H_I), spec.seed("w"), device)
+                    / math.sqrt(spec.H_I)).to(dt)
+    else:
+        out["q_I"] = out["k_I"] = out["w"] = None
+    out["sink"] = _randn((spec.H,), spec.seed("sink"), device)
+    return out
+
+
+def sample_rows(spec: LayerSpec, n_random: int = 256, seed: int = 12345) -> List[int]:
+    """Query rows (0-based) to check on large shapes: the early rows, rows around the
+    window edge, the top-k saturation point, every 128-boundary neighbourhood that is
+    cheap, the last 16 rows and a seeded random set."""
+    S = spec.S_q
+    rows = set()
+    m = max(spec.m, 1)
+    rows.update(range(0, min(S, 2 * m + 2)))
+    for c in (spec.W - 1, spec.W, spec.W + 1):
+        if 0 <= c < S:
+            rows.add(c)
+    if spec.topk:
+        for c in (spec.topk * m - 2, spec.topk * m - 1, spec.topk * m):
+            if 0 <= c < S:
+                rows.add(c)
+    for c in range(127, S, max(128, S // 16)):
+        rows.update(x for x in (c, c + 1) if x < S)
+    rows.update(range(max(0, S - 16), S))
+    g = torch.Generator().manual_seed(seed)
+    if S > 0:
+        rows.update(torch.randint(0, S, (n_random,), generator=g).tolist())
+    return sorted(rows)

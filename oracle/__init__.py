@@ -1,0 +1,195 @@
+"""fp64 CPU oracle for the DeepSeek-V4 hybrid compressed attention layer.
+
+TEST INFRASTRUCTURE ONLY: the CPU tests, the smoke check and the benchmark's CPU
+baseline call it; the product path never does.  The arithmetic lives in plain C
+(csa_oracle.c, compiled with gcc into liboracle.so); this module only converts arrays to
+float64 and calls it.  It shares no code with the CUDA library.
+
+Function map (each C function's comment cites the page passage it follows):
+  compress      -> orc_compress       gated pooling, CSA/HCA windows
+  n_visible     -> orc_n_visible      causal visibility of compressed entries
+  index_scores  -> orc_index_scores   Lightning Indexer score
+  topk          -> orc_topk           top-k with -1 marker
+  attend        -> orc_attend         sink MQA over window + entries, RoPE, de-rotation
+  attend_keys   -> orc_attend_keys    the same for one query over explicit keys
+  rope          -> orc_rope_rows      interleaved-pair partial RoPE
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "csa_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_dp = ctypes.POINTER(ctypes.c_double)
+_lp = ctypes.POINTER(ctypes.c_int64)
+_ip = ctypes.POINTER(ctypes.c_int32)
+_i64 = ctypes.c_int64
+
+
+def build(force: bool = False) -> str:
+    """Compile csa_oracle.c with gcc (-O2, OpenMP, IEEE semantics: no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp.%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _bind(path: str):
+    lib = ctypes.CDLL(path)
+    lib.orc_rope_rows.argtypes = [_dp, _dp, _i64, _i64, _i64, ctypes.c_double]
+    lib.orc_compress.argtypes = [_dp, _dp, _dp, _i64, _i64, _i64, _i64, ctypes.c_int]
+    lib.orc_n_visible.argtypes = [_i64, _i64, _i64]
+    lib.orc_n_visible.restype = _i64
+    lib.orc_index_scores.argtypes = [_dp, _dp, _dp, _lp, _i64, _i64, _i64, _i64, _i64, _i64, _dp]
+    lib.orc_topk.argtypes = [_dp, _lp, _i64, _i64, _i64, _i64, _i64, _ip, _dp]
+    lib.orc_attend_keys.argtypes = [_dp, ctypes.c_double, _dp, _dp, _i64, _dp, _i64, _i64, _i64,
+                                    ctypes.c_double, ctypes.c_double, _dp]
+    lib.orc_attend.argtypes = [_dp, _lp, _i64, _dp, _i64, _i64, _dp, _i64, _i64, _ip, _i64,
+                               ctypes.c_int, _dp, _i64, _i64, _i64, _i64, ctypes.c_double, _i64,
+                               ctypes.c_double, _dp]
+    return lib
+
+
+class using:
+    """Run oracle calls against another build of csa_oracle.c (the mutation tests build
+    deliberately broken copies to show that the pins catch them)."""
+
+    def __init__(self, path: str):
+        self.path = path
+
+    def __enter__(self):
+        global _lib
+        _load()
+        self._saved = _lib
+        _lib = _bind(self.path)
+        return self
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self._saved
+        return False
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = _bind(_LIB)
+            _lib = lib
+    return _lib
+
+
+def _f64(x) -> np.ndarray:
+    if hasattr(x, "detach"):  # torch tensor -> numpy without importing torch here
+        x = x.detach().float().cpu().numpy() if str(x.dtype) == "torch.bfloat16" else x.detach().cpu().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray, t):
+    return a.ctypes.data_as(t)
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise ValueError("oracle %s failed with code %d" % (what, rc))
+
+
+def rope(x, pos, R: int, base: float) -> np.ndarray:
+    """Rotate rows x[..., D] at positions pos[...] (one per row)."""
+    a = _f64(x).copy()
+    D = a.shape[-1]
+    rows = a.reshape(-1, D)
+    p = np.ascontiguousarray(np.broadcast_to(np.asarray(pos, dtype=np.float64),
+                                             a.shape[:-1]).reshape(-1))
+    _check(_load().orc_rope_rows(_ptr(rows, _dp), _ptr(p, _dp), rows.shape[0], D, R, base), "rope")
+    return rows.reshape(a.shape)
+
+
+def compress(kv, gate, m: int, overlap: int) -> np.ndarray:
+    """kv, gate [B,S,D] -> pool [B, S//m, D]."""
+    kv, gate = _f64(kv), _f64(gate)
+    B, S, D = kv.shape
+    pool = np.zeros((B, S // m, D), dtype=np.float64)
+    _check(_load().orc_compress(_ptr(kv, _dp), _ptr(gate, _dp), _ptr(pool, _dp), B, S, D, m,
+                                int(overlap)), "compress")
+    return pool
+
+
+def n_visible(t: int, m: int, P: int) -> int:
+    return int(_load().orc_n_visible(t, m, P))
+
+
+def index_scores(q_I, w, k_I, tpos, m: int) -> np.ndarray:
+    """q_I [B,n,H_I,d_I], w [B,n,H_I], k_I [B,P,d_I], tpos [n] -> scores [B,n,P] (NaN = not visible)."""
+    q_I, w, k_I = _f64(q_I), _f64(w), _f64(k_I)
+    B, n, HI, dI = q_I.shape
+    P = k_I.shape[1]
+    tp = np.ascontiguousarray(np.asarray(tpos, dtype=np.int64))
+    out = np.zeros((B, n, P), dtype=np.float64)
+    _check(_load().orc_index_scores(_ptr(q_I, _dp), _ptr(w, _dp), _ptr(k_I, _dp), _ptr(tp, _lp),
+                                    B, n, P, HI, dI, m, _ptr(out, _dp)), "index_scores")
+    return out
+
+
+def topk(scores, tpos, m: int, k: int):
+    """scores [B,n,P] -> (idx int32 [B,n,k] with -1 padding, selected scores [B,n,k])."""
+    sc = _f64(scores)
+    B, n, P = sc.shape
+    tp = np.ascontiguousarray(np.asarray(tpos, dtype=np.int64))
+    idx = np.zeros((B, n, k), dtype=np.int32)
+    sel = np.zeros((B, n, k), dtype=np.float64)
+    _check(_load().orc_topk(_ptr(sc, _dp), _ptr(tp, _lp), B, n, P, m, k, _ptr(idx, _ip),
+                            _ptr(sel, _dp)), "topk")
+    return idx, sel
+
+
+def attend_keys(q, tq: float, keys, kpos, sink, R: int, base: float, scale: float) -> np.ndarray:
+    """One query q [H,D] at tq over explicit un-rotated keys [n,D] at kpos [n]."""
+    q, keys, sink = _f64(q), _f64(keys), _f64(sink)
+    H, D = q.shape
+    kp = np.ascontiguousarray(np.asarray(kpos, dtype=np.float64))
+    out = np.zeros((H, D), dtype=np.float64)
+    _check(_load().orc_attend_keys(_ptr(q, _dp), float(tq), _ptr(keys, _dp), _ptr(kp, _dp),
+                                   keys.shape[0], _ptr(sink, _dp), H, D, R, base, scale,
+                                   _ptr(out, _dp)), "attend_keys")
+    return out
+
+
+def attend(q, tpos, kv, kv_pos0: int, pool, m: int, idx, sink, R: int, base: float, W: int,
+           scale: float, mode: str) -> np.ndarray:
+    """q [B,n,H,D] at positions tpos [n]; kv [B,S_kv,D] from kv_pos0; pool [B,P,D] or None;
+    idx [B,n,k] int32 (mode "csa") or None (mode "hca" / "sliding"); sink [H]."""
+    q, kv, sink = _f64(q), _f64(kv), _f64(sink)
+    B, n, H, D = q.shape
+    S_kv = kv.shape[1]
+    if pool is None:
+        pool = np.zeros((B, 0, D), dtype=np.float64)
+    pool = _f64(pool)
+    P = pool.shape[1]
+    tp = np.ascontiguousarray(np.asarray(tpos, dtype=np.int64))
+    if mode == "csa":
+        idx_a = np.ascontiguousarray(np.asarray(idx, dtype=np.int32))
+        k = idx_a.shape[-1]
+        mode_i = 0
+    else:
+        idx_a = np.zeros((1,), dtype=np.int32)
+        k = 0
+        mode_i = 1
+    out = np.zeros((B, n, H, D), dtype=np.float64)
+    _check(_load().orc_attend(_ptr(q, _dp), _ptr(tp, _lp), n, _ptr(kv, _dp), S_kv, kv_pos0,
+                              _ptr(pool, _dp), P, m, _ptr(idx_a, _ip), k, mode_i,
+                              _ptr(sink, _dp), B, H, D, R, base, W, scale, _ptr(out, _dp)),
+           "attend")
+    return out
