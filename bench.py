@@ -1,0 +1,532 @@
+"""Benchmark: DeepSeek-V4 CSA/HCA attention layer on B200 through the C ABI.
+
+One step = the whole hot path over one batch of seeded synthetic input already resident
+in HBM: KV Compressor -> Lightning Indexer + top-k -> sparse sink attention (for the CSA
+prefill workload: csa_compress, csa_index_topk, csa_attend).  Default workload: the CSA
+prefill layer at V4-Flash head shape (B=1, S=8192, H=64, D=512, rope 64, window 128,
+m=4, 2048 entries, H_I=64, d_I=128, top-k 512).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 1|2|3|4] [--impl reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own independent layer
+instance (its own seeded sequence), no data-path collective; value = all ranks' tokens
+over the max-over-ranks device time (weak scaling).  --impl reference times the fp64 CPU
+oracle on the host cores instead (rank 0 only), on a bounded sample of query rows.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CSA/HCA layer tokens/s (prefill, decode) on 1 B200; % of HBM / bf16 TC roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- work model
+def n_vis(t, m, P):
+    return min(P, (t + 1) // m) if t >= 0 else 0
+
+
+def n_win(spec, t):
+    lo = max(t - spec.W + 1, spec.kv_pos0)
+    hi = min(t, spec.kv_pos0 + spec.S_kv - 1)
+    return max(0, hi - lo + 1)
+
+
+def algorithmic_work(spec):
+    """Per-stage algorithmic work of one layer call (the definitions' counts):
+    compress bytes = kv + gate read + pool written; indexer FLOPs = sum_t 2 H_I d_I n_vis(t);
+    attention FLOPs = sum_t 4 H D |K_t|; attention HBM bytes = q read + out written +
+    each distinct kv/pool row once."""
+    e = 4 if spec.dtype == "f32" else 2
+    w = {}
+    if not spec.decode and spec.kind != "sliding":
+        w["compress_bytes"] = spec.B * (2 * spec.S_kv * spec.D + spec.P * spec.D) * e
+    keys = 0
+    idx_flops = 0
+    for i in range(spec.S_q):
+        t = spec.q_pos0 + i
+        nv = n_vis(t, spec.m, spec.P)
+        ne = min(spec.topk, nv) if spec.kind == "csa" else (nv if spec.kind == "hca" else 0)
+        keys += n_win(spec, t) + ne
+        if spec.kind == "csa":
+            idx_flops += 2 * spec.H_I * spec.d_I * nv
+    w["attend_flops"] = 4 * spec.B * spec.H * spec.D * keys
+    w["index_flops"] = spec.B * idx_flops
+    w["attend_bytes"] = spec.B * (2 * spec.S_q * spec.H * spec.D + (spec.S_kv + spec.P) * spec.D) * e
+    if spec.kind == "csa":
+        w["index_bytes"] = spec.B * (spec.S_q * spec.H_I * (spec.d_I + 1) + spec.P * spec.d_I) * e \
+            + spec.B * spec.S_q * spec.topk * 4
+    return w
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", "csa_clocks_%d_%d.csv" % (os.getpid(), gpu_index))
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu),
+                                          "--query-gpu=" + self.FIELDS, "--format=csv,noheader",
+                                          "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sms, maxs, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) < 9:
+                    continue
+                try:
+                    sms.append(float(p[1].split()[0]))
+                    maxs.append(float(p[2].split()[0]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, p[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sms:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = sorted(sms)[len(sms) // 4:] or sms  # drop idle-edge samples
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(maxs),
+                "samples": len(sms), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def workload_specs(workload: int):
+    import csa_synth as cs
+    return cs.WORKLOADS[workload]
+
+
+def rank_spec(spec, rank):
+    # each rank: its own independent sequence (seeded per rank)
+    return dataclasses.replace(spec, workload=spec.workload + 10 * rank) if rank else spec
+
+
+class LayerRunner:
+    """Holds one layer's device inputs/outputs and runs it through the C ABI."""
+
+    def __init__(self, spec, device):
+        import torch
+        import csa_synth as cs
+        import sparse_attention_14_b200 as csa
+        self.csa, self.torch, self.spec = csa, torch, spec
+        self.inp = cs.make_inputs(spec, device=device)
+        s = spec
+        dt = s.torch_dtype
+        self.pool = self.inp["pool"] if s.decode else (
+            torch.empty((s.B, s.P, s.D), dtype=dt, device=device) if s.kind != "sliding" else None)
+        self.idx = torch.empty((s.B, s.S_q, s.topk), dtype=torch.int32, device=device) \
+            if s.kind == "csa" else None
+        self.out = torch.empty_like(self.inp["q"])
+        wsi = csa.csa_index_topk_workspace_bytes(s.B, s.S_q, s.P, s.H_I, s.d_I, s.topk, dt) \
+            if s.kind == "csa" else 0
+        wsa = csa.csa_attend_workspace_bytes(0 if s.kind == "csa" else 1, s.B, s.S_q, s.S_kv, s.P,
+                                             s.H, s.D, s.topk, dt)
+        self.ws_i = torch.empty(max(wsi, 1), dtype=torch.uint8, device=device) if wsi else None
+        self.ws_a = torch.empty(max(wsa, 1), dtype=torch.uint8, device=device) if wsa else None
+
+    def stages(self):
+        s = self.spec
+        st = []
+        if not s.decode and s.kind != "sliding":
+            st.append("compress")
+        if s.kind == "csa":
+            st.append("index")
+        st.append("attend")
+        return st
+
+    def run_stage(self, name):
+        s, i, csa = self.spec, self.inp, self.csa
+        if name == "compress":
+            csa.csa_compress(i["kv"], i["gate"], s.m, s.overlap, pool=self.pool)
+        elif name == "index":
+            csa.csa_index_topk(i["q_I"], i["w"], i["k_I"], s.q_pos0, s.m, s.topk, idx=self.idx,
+                               workspace=self.ws_i)
+        elif s.kind == "csa":
+            csa.csa_attend(i["q"], i["kv"], s.kv_pos0, self.pool, self.idx, i["sink"], s.q_pos0, s.R,
+                           s.base, s.W, s.m, s.scale, out=self.out, workspace=self.ws_a)
+        else:
+            csa.hca_attend(i["q"], i["kv"], s.kv_pos0, self.pool if s.kind == "hca" else None,
+                           i["sink"], s.q_pos0, s.R, s.base, s.W, s.m, s.scale, out=self.out,
+                           workspace=self.ws_a)
+
+
+def src_hash(names):
+    h = hashlib.sha256()
+    for n in names:
+        p = os.path.join(ROOT, "sparse_attention_14_b200", "csrc", n)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+STAGE_SOURCES = {"compress": ["compress.cu", "common.cuh"],
+                 "index": ["index_topk.cu", "topk.cuh", "index_tc.cu", "umma.cuh", "common.cuh"],
+                 "attend": ["attend.cu", "attend_tc.cu", "umma.cuh", "common.cuh"]}
+
+
+def ncu_traffic(stage, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current
+    source of that kernel (else None)."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get("workload%d" % workload, {}).get(stage)
+    if not e or e.get("src_sha") != src_hash(STAGE_SOURCES[stage]):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def gpu_arm(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import sparse_attention_14_b200 as csa
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    specs = [rank_spec(s, rank) for s in workload_specs(args.workload)]
+    csa.load_library()
+    stream = torch.cuda.current_stream()
+
+    # mixed stack: allocate per layer inside the step would time allocation; instead keep
+    # every layer resident when it fits, else run layers one at a time (generated per layer)
+    runners = [LayerRunner(s, dev) for s in specs]
+    tokens_per_step = sum(s.B * s.S_q for s in specs[:1])  # the block processes S tokens once
+    stage_names = [(li, st) for li, r in enumerate(runners) for st in r.stages()]
+
+    def step(events=None):
+        for li, st in stage_names:
+            if events is not None:
+                events[(li, st)][0].record(stream)
+            runners[li].run_stage(st)
+            if events is not None:
+                events[(li, st)][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+
+    launches0 = csa.launch_count()
+    clk = ClockSampler(local_rank)
+    clk.start()
+    time.sleep(0.3)
+    ev = {k: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)] for k in stage_names}
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t0.record(stream)
+    for k in range(args.steps):
+        step({key: ev[key][k] for key in stage_names})
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = clk.stop()
+    launches = csa.launch_count() - launches0
+    ms_total = t0.elapsed_time(t1)
+    if world > 1:
+        tt = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total = float(tt.item())
+    ms_step = ms_total / args.steps
+    stage_ms = {"%d:%s" % key: sum(a.elapsed_time(b) for a, b in ev[key]) / args.steps
+                for key in stage_names}
+
+    # end to end through the public API with host buffers: pinned inputs copied in, the
+    # layer run, the output copied back, every step
+    e2e = None
+    if not args.no_e2e:
+        e2e = e2e_arm(args, runners, stage_names, stream, world, dev)
+
+    if rank != 0:
+        return None
+    peaks, peak_kind = load_peaks()
+    spec0 = specs[0]
+    work = [algorithmic_work(s) for s in specs]
+    # dominant kernel = the stage with the largest device time
+    (dom_layer, dom_stage), dom_ms = max(((k, stage_ms["%d:%s" % k]) for k in stage_names),
+                                         key=lambda x: x[1])
+    wk = work[dom_layer]
+    dom_spec = specs[dom_layer]
+    if dom_stage == "compress" or (dom_stage == "attend" and (dom_spec.kind == "sliding" or dom_spec.decode)) \
+            or (dom_stage == "index" and dom_spec.decode):
+        key_b = {"compress": "compress_bytes", "attend": "attend_bytes", "index": "index_bytes"}[dom_stage]
+        achieved = wk[key_b] / (dom_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "algorithmic_bytes_per_launch": wk[key_b]}
+    else:
+        key_f = "attend_flops" if dom_stage == "attend" else "index_flops"
+        achieved = wk[key_f] / (dom_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
+                "algorithmic_flops_per_launch": wk[key_f]}
+    roof.update({"kernel": "%s (layer %d)" % (dom_stage, dom_layer),
+                 "kernel_ms": round(dom_ms, 4), "peak_source": peak_kind + " (burst)",
+                 "traffic": ncu_traffic(dom_stage, args.workload)})
+    tokens = tokens_per_step * world
+    value = tokens / (ms_step * 1e-3)
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32" if spec0.dtype == "f32" else "bf16",
+        "data": "synthetic (seeded N(0,1) q/kv/gate/q_I/k_I, w/sqrt(H_I), RMS-normalised kv)",
+        "config": {"workload": workload_name(args.workload, specs), "B": spec0.B, "S": spec0.S_q,
+                   "H": spec0.H, "D": spec0.D, "rope_dim": spec0.R, "window": spec0.W,
+                   "layers": [s.kind for s in specs], "m": [s.m for s in specs],
+                   "P": [s.P for s in specs], "topk": spec0.topk, "H_I": spec0.H_I,
+                   "d_I": spec0.d_I, "parallelism": "independent layer instance per GPU",
+                   "l2": "inputs larger than L2 (q/out/q_I > 126 MB per step); no flush"},
+        "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
+        "roofline": roof,
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    return line
+
+
+def workload_name(w, specs):
+    return {0: "tiny CSA layer fp32 (S=256)", 1: "CSA prefill bf16 S=8192 (V4-Flash layer shape)",
+            2: "HCA prefill bf16 S=65536", 3: "CSA decode bf16 B=64 at 65536 cached tokens",
+            4: "mixed 4-layer stack bf16 S=131072"}[w]
+
+
+def e2e_arm(args, runners, stage_names, stream, world, dev):
+    import torch
+    import torch.distributed as dist
+    host = []
+    h2d = d2h = 0
+    for r in runners:
+        pairs = []
+        for k, v in r.inp.items():
+            if v is None:
+                continue
+            hv = torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+            hv.copy_(v)
+            pairs.append((hv, v))
+            h2d += v.numel() * v.element_size()
+        ho = torch.empty(r.out.shape, dtype=r.out.dtype, pin_memory=True)
+        d2h += r.out.numel() * r.out.element_size()
+        host.append((pairs, ho))
+    steps = max(1, min(args.steps, 5))
+
+    def one():
+        for (pairs, ho), r in zip(host, runners):
+            for hv, dv in pairs:
+                dv.copy_(hv, non_blocking=True)
+        for li, st in stage_names:
+            runners[li].run_stage(st)
+        for (pairs, ho), r in zip(host, runners):
+            ho.copy_(r.out, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    tokens = runners[0].spec.B * runners[0].spec.S_q * world
+    return {"value": round(tokens / (ms * 1e-3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3),
+            "steps": steps}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_sample_run(spec, rows, inp_cpu=None):
+    """The fp64 oracle over the whole hot path for the given query rows (the compressor
+    runs in full: every sampled row may attend to any entry).  Returns seconds."""
+    import numpy as np
+    import csa_synth as cs
+    import oracle
+    inp = cs.make_inputs(spec, device="cpu") if inp_cpu is None else inp_cpu
+    f64 = lambda t: None if t is None else t.double().numpy()
+    t0 = time.perf_counter()
+    pool = None
+    if spec.decode:
+        pool = f64(inp["pool"])
+    elif spec.kind != "sliding":
+        pool = oracle.compress(f64(inp["kv"]), f64(inp["gate"]), spec.m, spec.overlap)
+    tpos = np.asarray(rows, dtype=np.int64) + spec.q_pos0
+    idx = None
+    if spec.kind == "csa":
+        sc = oracle.index_scores(f64(inp["q_I"][:, rows]), f64(inp["w"][:, rows]), f64(inp["k_I"]),
+                                 tpos, spec.m)
+        idx, _ = oracle.topk(sc, tpos, spec.m, spec.topk)
+    oracle.attend(f64(inp["q"][:, rows]), tpos, f64(inp["kv"]), spec.kv_pos0, pool, spec.m, idx,
+                  f64(inp["sink"]), spec.R, spec.base, spec.W, spec.scale,
+                  "csa" if spec.kind == "csa" else "hca")
+    return time.perf_counter() - t0
+
+
+def oracle_rows(spec, n):
+    # evenly spaced query rows: the same causal mix of window/entry counts as the workload
+    S = spec.S_q
+    n = min(n, S)
+    return sorted({int(round(x)) for x in [(k + 0.5) * S / n for k in range(n)]})
+
+
+def oracle_threads():
+    v = os.environ.get("OMP_NUM_THREADS")
+    return int(v) if v else (len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count())
+
+
+def cpu_baseline(args):
+    spec = workload_specs(args.workload)[0]
+    if spec.B * spec.S_q * spec.D * spec.H > 4e9:
+        spec = dataclasses.replace(spec)  # inputs generated per call below, bounded by rows
+    import csa_synth as cs
+    inp = cs.make_inputs(spec, device="cpu")
+    rows = oracle_rows(spec, 16)
+    dt = oracle_sample_run(spec, rows, inp)
+    # size the sample to about 15 s of CPU work
+    n = max(16, min(spec.S_q, int(16 * 15.0 / max(dt, 1e-3))))
+    rows = oracle_rows(spec, n)
+    dt = oracle_sample_run(spec, rows, inp)
+    units = spec.B * len(rows)
+    return {"value": round(units / dt, 3), "unit": "tokens/s", "cores": oracle_threads(),
+            "kind": "oracle",
+            "sample": "%d of %d query rows (evenly spaced) x B=%d of %s; compressor in full; %.1f s"
+                      % (len(rows), spec.S_q, spec.B, spec.name, dt)}
+
+
+def reference_arm(args, rank, world):
+    if rank != 0:
+        return None
+    import csa_synth as cs
+    spec = workload_specs(args.workload)[0]
+    inp = cs.make_inputs(spec, device="cpu")
+    rows = oracle_rows(spec, 16)
+    dt = oracle_sample_run(spec, rows, inp)
+    n = max(8, min(spec.S_q, int(16 * 6.0 / max(dt, 1e-3))))  # ~6 s per step
+    rows = oracle_rows(spec, n)
+    for _ in range(args.warmup):
+        oracle_sample_run(spec, rows, inp)
+    t = [oracle_sample_run(spec, rows, inp) for _ in range(args.steps)]
+    ms = 1e3 * sum(t) / len(t)
+    units = spec.B * len(rows)
+    value = units / (ms * 1e-3)
+    sample = "%d of %d query rows (evenly spaced) x B=%d of %s per step; compressor in full" % (
+        len(rows), spec.S_q, spec.B, spec.name)
+    return {"metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": workload_name(args.workload, None), "B": spec.B, "S": spec.S_q},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s",
+                             "cores": oracle_threads(), "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", type=int, default=1, choices=[0, 1, 2, 3, 4])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = reference_arm(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        line = gpu_arm(args, rank, world, local_rank)
+        if line is not None:
+            if world == 1 and not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline(args)
+            else:
+                line["cpu_baseline"] = None
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

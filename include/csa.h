@@ -1,0 +1,163 @@
+/*
+ * csa.h -- C ABI of libcsa_b200: the DeepSeek-V4 hybrid compressed attention layer on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer (HF docs model_doc/deepseek_v4, section "Hybrid attention (2.3)"):
+ *   1. a KV Compressor pools raw K=V rows into compressed entries by a per-channel
+ *      softmax of gate logits over each window (CSA: ratio m=4, overlapping windows;
+ *      HCA: ratio m'=128, non-overlapping)                         -> csa_compress
+ *   2. the CSA Lightning Indexer scores every query against the causally visible
+ *      entries and keeps the top-k                                  -> csa_index_topk
+ *   3. single-KV-head shared K=V attention over the sliding window plus the selected
+ *      entries (CSA) or every visible entry (HCA), with a per-head sink logit (eq. 27),
+ *      interleaved-pair partial RoPE on the last rope_dim channels and the output's
+ *      rope slice rotated back by -position (eq. 26)        -> csa_attend / hca_attend
+ *
+ * Conventions shared by every call
+ *  - All tensor pointers are DEVICE pointers owned by the caller; all tensors are dense
+ *    row-major (innermost dimension last).  The library never allocates, frees or
+ *    synchronises: every call only enqueues work on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream) and returns.
+ *  - `dtype` gives the element type of every floating tensor argument except `sink`
+ *    (always fp32) and `scores_opt` (always fp32).  Arithmetic is fp32 throughout;
+ *    bf16 tensors are rounded to nearest-even on store.
+ *  - Positions are absolute token positions.  Query row i is at q_pos0 + i; raw K=V
+ *    row r is at kv_pos0 + r; compressed entry j covers tokens ending at (j+1)*ratio-1,
+ *    is visible to the query at t iff (j+1)*ratio - 1 <= t, and is rotated at position
+ *    j*ratio.  All sequences of a batch share the positions.
+ *  - Errors: arguments are checked on the host before anything is enqueued; a bad
+ *    argument returns CSA_ERR_INVALID_ARG (or CSA_ERR_UNSUPPORTED for a valid shape
+ *    this build does not handle, CSA_ERR_WORKSPACE for a short workspace) and
+ *    csa_last_error() describes it.  A failed launch returns CSA_ERR_CUDA.  Kernels
+ *    never trap.  Tensor pointers must be 16-byte aligned (idx and sink: 4-byte).
+ *  - Shape limits of this build: D % 8 == 0 and 8 <= D <= 1024; rope_dim even and
+ *    <= min(D, 256); 1 <= topk <= 2048; d_I % 8 == 0 and d_I <= 256; H, H_I >= 1.
+ */
+#ifndef CSA_B200_H
+#define CSA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { CSA_F32 = 0, CSA_BF16 = 1 } csa_dtype_t;
+
+typedef enum {
+    CSA_OK = 0,
+    CSA_ERR_INVALID_ARG = -1,
+    CSA_ERR_UNSUPPORTED = -2,
+    CSA_ERR_CUDA = -3,
+    CSA_ERR_WORKSPACE = -4
+} csa_status_t;
+
+/*
+ * csa_compress -- KV Compressor (HF docs model_doc/deepseek_v4 section 2.3.1 "low
+ * compression with overlapping windows", 2.3.2 "m'=128, non-overlapping"; HF PR #45616
+ * "Compressor.forward always returns a tensor ... empty when no window has closed").
+ *
+ *   pool[b,j,d] = sum_{s in Win_j} softmax_{s in Win_j}(gate[b,s,d]) * kv[b,s,d]
+ *   Win_j = [max(0,(j-1)*ratio), (j+1)*ratio) if overlap, else [j*ratio, (j+1)*ratio)
+ *   for j in [0, P), P = floor(S / ratio); a trailing partial window is not emitted.
+ *
+ *   kv, gate : [B, S, D]   raw K=V rows (un-rotated) and gate logits, positions 0..S-1
+ *   pool     : [B, P, D]   output, un-rotated; nothing is written when P == 0
+ *   ratio >= 1; overlap in {0, 1}.
+ */
+csa_status_t csa_compress(const void *kv, const void *gate, void *pool, int64_t B, int64_t S,
+                          int32_t D, int32_t ratio, int32_t overlap, csa_dtype_t dtype,
+                          void *stream);
+
+/*
+ * csa_index_topk -- CSA Lightning Indexer and top-k (HF docs model_doc/deepseek_v4
+ * section 2.3.1, eq. 13-17 named there; section "Attention mask layout": queries before
+ * the first closed window get only the -1 marker).
+ *
+ *   score[t,j] = sum_{h < H_I} w[b,i,h] * max(0, <q_I[b,i,h,:], k_I[b,j,:]>)
+ *   for the visible entries j < n_vis(t) = min(P, floor((t+1)/ratio)), t = q_pos0 + i.
+ *   idx[b,i,:] = the min(topk, n_vis) best entries, score descending (ties: lower j
+ *   first), then -1 padding.
+ *
+ *   q_I : [B, S_q, H_I, d_I]   w : [B, S_q, H_I]   k_I : [B, P, d_I]
+ *   idx : [B, S_q, topk] int32 output
+ *   scores_opt : NULL, or [B, S_q, topk] fp32 output holding each kept entry's score
+ *                (NaN in the -1 slots)
+ *   workspace  : device scratch of at least csa_index_topk_workspace_bytes(...) bytes
+ *                (may be NULL when that is 0); contents are not preserved.
+ */
+csa_status_t csa_index_topk(const void *q_I, const void *w, const void *k_I, int64_t B,
+                            int64_t S_q, int64_t q_pos0, int64_t P, int32_t H_I, int32_t d_I,
+                            int32_t ratio, int32_t topk, int32_t *idx, float *scores_opt,
+                            void *workspace, size_t workspace_bytes, csa_dtype_t dtype,
+                            void *stream);
+
+size_t csa_index_topk_workspace_bytes(int64_t B, int64_t S_q, int64_t P, int32_t H_I,
+                                      int32_t d_I, int32_t topk, csa_dtype_t dtype);
+
+/*
+ * csa_attend -- CSA attention: shared K=V single-head MQA over the sliding window plus
+ * the selected entries, with sink, partial RoPE and output de-rotation (HF docs
+ * model_doc/deepseek_v4 section 2.3 "shared K=V Multi-Query Attention", "partial
+ * rotary positional embedding ... position -i (eq. 26)", "learnable attention sink per
+ * head (eq. 27)", "additional branch of sliding window attention"; HF PR #45616 "port
+ * eager_attention_forward from GPT-OSS", un-rotation of the output rope slice).
+ *
+ * For query row i at t = q_pos0 + i, head h:
+ *   keys K_t = { raw rows r : t - window < kv_pos0 + r <= t, 0 <= r < S_kv }
+ *            + { pool entries idx[b,i,c] : idx[b,i,c] in [0, n_vis(t)) }  (other values,
+ *              including -1, are skipped; an entry listed twice counts twice, and so
+ *              does an entry whose tokens are also in the window)
+ *   Rot(x, p): pairs (D-R+2i, D-R+2i+1) of x turned by p * rope_base^(-2i/R), R=rope_dim
+ *   l_x = scale * <Rot(q[b,i,h], t), Rot(key_x, pos_x)>, pos_x = kv_pos0 + r or j*ratio
+ *   M = max(max_x l_x, sink[h]),  Z = exp(sink[h] - M) + sum_x exp(l_x - M)
+ *   out[b,i,h,:] = sum_x exp(l_x - M) / Z * Rot(key_x, pos_x), then its last R channels
+ *                  are rotated by -t.
+ *
+ *   q   : [B, S_q, H, D]        kv : [B, S_kv, D] (un-rotated)   pool : [B, P, D]
+ *   idx : [B, S_q, topk] int32  sink : [H] fp32 (may hold -INFINITY)
+ *   out : [B, S_q, H, D] output
+ *   workspace : device scratch of at least csa_attend_workspace_bytes(...) bytes.
+ *   Requires q_pos0 >= 0 when S_q > 0 and window >= 1.
+ */
+csa_status_t csa_attend(const void *q, const void *kv, int64_t S_kv, int64_t kv_pos0,
+                        const void *pool, int64_t P, const int32_t *idx, int32_t topk,
+                        const float *sink, void *out, int64_t B, int64_t S_q, int64_t q_pos0,
+                        int32_t H, int32_t D, int32_t rope_dim, double rope_base,
+                        int32_t window, int32_t ratio, float scale, void *workspace,
+                        size_t workspace_bytes, csa_dtype_t dtype, void *stream);
+
+/*
+ * hca_attend -- HCA attention (HF docs model_doc/deepseek_v4 section 2.3.2 "no indexer
+ * -- every pool entry participates"; "Attention mask layout": entry w is visible iff
+ * w < (t+1)//m).  Same as csa_attend with K_t's entry part replaced by every visible
+ * entry j < n_vis(t).  P == 0 gives the sliding-window-only layer ("sliding_attention").
+ */
+csa_status_t hca_attend(const void *q, const void *kv, int64_t S_kv, int64_t kv_pos0,
+                        const void *pool, int64_t P, const float *sink, void *out, int64_t B,
+                        int64_t S_q, int64_t q_pos0, int32_t H, int32_t D, int32_t rope_dim,
+                        double rope_base, int32_t window, int32_t ratio, float scale,
+                        void *workspace, size_t workspace_bytes, csa_dtype_t dtype,
+                        void *stream);
+
+/* Scratch bytes csa_attend (mode 0) or hca_attend (mode 1) needs for these sizes. */
+size_t csa_attend_workspace_bytes(int32_t mode, int64_t B, int64_t S_q, int64_t S_kv,
+                                  int64_t P, int32_t H, int32_t D, int32_t topk,
+                                  csa_dtype_t dtype);
+
+/* Message for the last error returned on the calling host thread ("" if none). */
+const char *csa_last_error(void);
+
+/* Number of kernels this library has enqueued in this process (all devices, all
+ * threads); for accounting launches in a timed region. */
+uint64_t csa_launch_count(void);
+
+/* Library version string. */
+const char *csa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA_B200_H */

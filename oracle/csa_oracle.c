@@ -82,6 +82,7 @@ int orc_compress(const double *kv, const double *gate, double *pool,
 {
     if (B < 0 || S < 0 || D <= 0 || m <= 0) return ORC_BAD_ARG;
     int64_t P = S / m;
+#pragma omp parallel for collapse(2) schedule(static)
     for (int64_t b = 0; b < B; ++b) {
         for (int64_t j = 0; j < P; ++j) {
             int64_t lo = overlap ? (j - 1) * m : j * m;

@@ -1,0 +1,186 @@
+"""DeepSeek-V4 hybrid compressed attention (CSA / HCA) on NVIDIA B200.
+
+Thin Python binding over the C ABI of libcsa_b200.so (include/csa.h).  The functions
+below only check tensor metadata and marshal pointers, sizes and the current CUDA
+stream; every step of the layer runs in the library's sm_100a kernels.  If the library
+is missing or cannot be loaded, every call raises: there is no other code path.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+__all__ = ["csa_compress", "csa_index_topk", "csa_attend", "hca_attend",
+           "csa_index_topk_workspace_bytes", "csa_attend_workspace_bytes", "library_path",
+           "load_library", "launch_count", "CsaError", "CSA_F32", "CSA_BF16"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libcsa_b200.so")
+CSA_F32, CSA_BF16 = 0, 1
+_lib = None
+
+
+class CsaError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__("%s returned %d: %s" % (fn, code, msg))
+        self.code = code
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libcsa_b200.so (built by __graft_entry__.build() / build.py)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError("libcsa_b200.so is not built (%s); run `python "
+                          "sparse_attention_14_b200/build.py`" % _LIB_PATH)
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+    lib.csa_compress.argtypes = [vp, vp, vp, i64, i64, i32, i32, i32, ctypes.c_int, vp]
+    lib.csa_index_topk.argtypes = [vp, vp, vp, i64, i64, i64, i64, i32, i32, i32, i32, vp, vp, vp,
+                                   sz, ctypes.c_int, vp]
+    lib.csa_index_topk_workspace_bytes.argtypes = [i64, i64, i64, i32, i32, i32, ctypes.c_int]
+    lib.csa_index_topk_workspace_bytes.restype = sz
+    lib.csa_attend.argtypes = [vp, vp, i64, i64, vp, i64, vp, i32, vp, vp, i64, i64, i64, i32, i32,
+                               i32, ctypes.c_double, i32, i32, ctypes.c_float, vp, sz,
+                               ctypes.c_int, vp]
+    lib.hca_attend.argtypes = [vp, vp, i64, i64, vp, i64, vp, vp, i64, i64, i64, i32, i32, i32,
+                               ctypes.c_double, i32, i32, ctypes.c_float, vp, sz, ctypes.c_int, vp]
+    lib.csa_attend_workspace_bytes.argtypes = [i32, i64, i64, i64, i64, i32, i32, i32,
+                                               ctypes.c_int]
+    lib.csa_attend_workspace_bytes.restype = sz
+    for f in ("csa_compress", "csa_index_topk", "csa_attend", "hca_attend"):
+        getattr(lib, f).restype = ctypes.c_int
+    lib.csa_last_error.restype = ctypes.c_char_p
+    lib.csa_version.restype = ctypes.c_char_p
+    lib.csa_launch_count.restype = ctypes.c_uint64
+    _lib = lib
+    return lib
+
+
+def launch_count() -> int:
+    """Kernels the library has enqueued in this process."""
+    return int(load_library().csa_launch_count())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return CSA_F32
+    if t.dtype == torch.bfloat16:
+        return CSA_BF16
+    raise TypeError("unsupported dtype %s (float32 or bfloat16)" % t.dtype)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _call(fn: str, *args):
+    lib = load_library()
+    rc = getattr(lib, fn)(*args)
+    if rc != 0:
+        raise CsaError(fn, rc, lib.csa_last_error().decode())
+
+
+def _ws(nbytes: int, device, workspace: Optional[torch.Tensor]):
+    if nbytes == 0:
+        return None, 0
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def csa_compress(kv: torch.Tensor, gate: torch.Tensor, ratio: int, overlap: bool,
+                 pool: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """kv, gate [B,S,D] -> pool [B, S//ratio, D] (see include/csa.h)."""
+    B, S, D = kv.shape
+    if gate.shape != kv.shape or gate.dtype != kv.dtype:
+        raise ValueError("gate must match kv in shape and dtype")
+    P = S // ratio
+    if pool is None:
+        pool = torch.empty((B, P, D), dtype=kv.dtype, device=kv.device)
+    _call("csa_compress", _ptr(kv), _ptr(gate), _ptr(pool), B, S, D, ratio, int(bool(overlap)),
+          _dtype_code(kv), _stream(stream))
+    return pool
+
+
+def csa_index_topk_workspace_bytes(B, S_q, P, H_I, d_I, topk, dtype=torch.bfloat16) -> int:
+    code = CSA_F32 if dtype == torch.float32 else CSA_BF16
+    return int(load_library().csa_index_topk_workspace_bytes(B, S_q, P, H_I, d_I, topk, code))
+
+
+def csa_index_topk(q_I: torch.Tensor, w: torch.Tensor, k_I: torch.Tensor, q_pos0: int, ratio: int,
+                   topk: int, idx: Optional[torch.Tensor] = None, want_scores: bool = False,
+                   workspace: Optional[torch.Tensor] = None, stream=None):
+    """q_I [B,S_q,H_I,d_I], w [B,S_q,H_I], k_I [B,P,d_I] -> idx int32 [B,S_q,topk]
+    (and the kept scores fp32 [B,S_q,topk] when want_scores)."""
+    B, S_q, H_I, d_I = q_I.shape
+    P = k_I.shape[1]
+    if idx is None:
+        idx = torch.empty((B, S_q, topk), dtype=torch.int32, device=q_I.device)
+    scores = torch.empty((B, S_q, topk), dtype=torch.float32, device=q_I.device) if want_scores else None
+    ws, wsb = _ws(csa_index_topk_workspace_bytes(B, S_q, P, H_I, d_I, topk, q_I.dtype), q_I.device,
+                  workspace)
+    _call("csa_index_topk", _ptr(q_I), _ptr(w), _ptr(k_I), B, S_q, q_pos0, P, H_I, d_I, ratio, topk,
+          _ptr(idx), _ptr(scores), _ptr(ws), wsb, _dtype_code(q_I), _stream(stream))
+    return (idx, scores) if want_scores else idx
+
+
+def csa_attend_workspace_bytes(mode: int, B, S_q, S_kv, P, H, D, topk, dtype=torch.bfloat16) -> int:
+    code = CSA_F32 if dtype == torch.float32 else CSA_BF16
+    return int(load_library().csa_attend_workspace_bytes(mode, B, S_q, S_kv, P, H, D, topk, code))
+
+
+def csa_attend(q, kv, kv_pos0: int, pool, idx, sink, q_pos0: int, rope_dim: int, rope_base: float,
+               window: int, ratio: int, scale: Optional[float] = None, out=None, workspace=None,
+               stream=None) -> torch.Tensor:
+    """CSA attention; q [B,S_q,H,D], kv [B,S_kv,D], pool [B,P,D], idx int32 [B,S_q,k],
+    sink fp32 [H] -> out [B,S_q,H,D]."""
+    B, S_q, H, D = q.shape
+    S_kv, P, topk = kv.shape[1], pool.shape[1], idx.shape[-1]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    if out is None:
+        out = torch.empty_like(q)
+    ws, wsb = _ws(csa_attend_workspace_bytes(0, B, S_q, S_kv, P, H, D, topk, q.dtype), q.device,
+                  workspace)
+    _call("csa_attend", _ptr(q), _ptr(kv), S_kv, kv_pos0, _ptr(pool), P, _ptr(idx), topk, _ptr(sink),
+          _ptr(out), B, S_q, q_pos0, H, D, rope_dim, rope_base, window, ratio, scale, _ptr(ws), wsb,
+          _dtype_code(q), _stream(stream))
+    return out
+
+
+def hca_attend(q, kv, kv_pos0: int, pool, sink, q_pos0: int, rope_dim: int, rope_base: float,
+               window: int, ratio: int, scale: Optional[float] = None, out=None, workspace=None,
+               stream=None) -> torch.Tensor:
+    """HCA attention over every visible entry (pool None or P == 0: sliding-only layer)."""
+    B, S_q, H, D = q.shape
+    S_kv = kv.shape[1]
+    P = 0 if pool is None else pool.shape[1]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    if out is None:
+        out = torch.empty_like(q)
+    ws, wsb = _ws(csa_attend_workspace_bytes(1, B, S_q, S_kv, P, H, D, 0, q.dtype), q.device,
+                  workspace)
+    _call("hca_attend", _ptr(q), _ptr(kv), S_kv, kv_pos0, _ptr(pool) if P else None, P, _ptr(sink),
+          _ptr(out), B, S_q, q_pos0, H, D, rope_dim, rope_base, window, ratio, scale, _ptr(ws), wsb,
+          _dtype_code(q), _stream(stream))
+    return out

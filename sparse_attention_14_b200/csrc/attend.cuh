@@ -1,0 +1,45 @@
+// attend.cuh -- internal argument block and entry points of the attention kernels.
+#pragma once
+
+#include "common.cuh"
+
+namespace csa {
+
+struct AttendArgs {
+    const void *q;
+    const void *kv;
+    int64_t S_kv;
+    int64_t kv_pos0;
+    const void *pool;
+    int64_t P;
+    const int32_t *idx;
+    int topk;
+    const float *sink;
+    void *out;
+    int64_t B;
+    int64_t S_q;
+    int64_t q_pos0;
+    int H;
+    int D;
+    int rope_dim;
+    double rope_base;
+    int window;
+    int ratio;
+    float scale;
+    void *workspace;
+    size_t workspace_bytes;
+    csa_dtype_t dtype;
+    int mode;        // 0: CSA (idx), 1: HCA (every visible entry; P == 0: sliding only)
+    RopeTable rope;  // filled by the entry point
+};
+
+// General path: any H, D % 8 == 0, either dtype.
+csa_status_t attend_general(const AttendArgs &a, cudaStream_t st);
+
+// Scratch bytes the chosen path needs.
+size_t attend_workspace(const AttendArgs &a);
+
+// Picks the kernel for a validated call.
+csa_status_t attend_dispatch(const AttendArgs &a, cudaStream_t st);
+
+}  // namespace csa

@@ -1,0 +1,54 @@
+// common.cu -- error state, RoPE tables and path selection of libcsa_b200.
+#include <stdarg.h>
+#include <atomic>
+#include <string.h>
+
+#include "attend.cuh"
+#include "common.cuh"
+#include "index_topk.cuh"
+
+namespace csa {
+
+static thread_local char g_error[512];
+static std::atomic<unsigned long long> g_launches{0};
+
+void count_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+
+void set_error(const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_error, sizeof(g_error), fmt, ap);
+    va_end(ap);
+}
+
+void clear_error() { g_error[0] = '\0'; }
+
+void make_rope_table(RopeTable *t, int D, int R, double base) {
+    memset(t, 0, sizeof(*t));
+    t->n_pairs = R / 2;
+    t->first = D - R;
+    for (int i = 0; i < R / 2; ++i) t->inv_freq[i] = pow(base, -2.0 * (double)i / (double)R);
+}
+
+// ------------------------------------------------------------------ path selection
+size_t index_topk_workspace(int64_t, int64_t, int64_t, int, int, int, csa_dtype_t) { return 0; }
+
+csa_status_t index_topk_dispatch(const void *qI, const void *w, const void *kI, int64_t B,
+                                 int64_t S_q, int64_t q_pos0, int64_t P, int H_I, int d_I,
+                                 int ratio, int topk, int32_t *idx, float *scores_opt, void *,
+                                 size_t, csa_dtype_t dtype, cudaStream_t st) {
+    return index_topk_general(qI, w, kI, B, S_q, q_pos0, P, H_I, d_I, ratio, topk, idx,
+                              scores_opt, dtype, st);
+}
+
+size_t attend_workspace(const AttendArgs &) { return 0; }
+
+csa_status_t attend_dispatch(const AttendArgs &a, cudaStream_t st) { return attend_general(a, st); }
+
+}  // namespace csa
+
+extern "C" const char *csa_last_error(void) { return csa::g_error; }
+
+extern "C" uint64_t csa_launch_count(void) { return csa::g_launches.load(); }
+
+extern "C" const char *csa_version(void) { return "csa_b200 0.1 (sm_100a)"; }

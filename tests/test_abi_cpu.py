@@ -1,0 +1,107 @@
+"""The C-ABI library without a GPU: it loads, exports every function include/csa.h
+declares, and rejects bad arguments on the host before touching the device."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+import sparse_attention_14_b200 as csa
+from sparse_attention_14_b200 import build as csa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    csa_build.build()
+    return csa.load_library()
+
+
+def _declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z_0-9]*\s*\*?\s*"
+                                r"([a-z][a-z_0-9]*)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared_functions()
+    assert {"csa_compress", "csa_index_topk", "csa_attend", "hca_attend"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), "missing export %s" % n
+    assert lib.csa_version().decode().startswith("csa_b200")
+
+
+FAKE = ctypes.c_void_p(0x10000)        # never dereferenced: every call below fails validation
+MIS = ctypes.c_void_p(0x10004)         # misaligned
+
+
+def _err(lib):
+    return lib.csa_last_error().decode()
+
+
+def test_compress_rejects(lib):
+    assert lib.csa_compress(FAKE, FAKE, FAKE, 1, 16, 7, 4, 1, 1, None) == -1
+    assert "multiple of 8" in _err(lib)
+    assert lib.csa_compress(FAKE, FAKE, FAKE, 1, 16, 64, 0, 1, 1, None) == -1
+    assert lib.csa_compress(FAKE, FAKE, FAKE, 1, 16, 64, 4, 2, 1, None) == -1
+    assert lib.csa_compress(None, FAKE, FAKE, 1, 16, 64, 4, 1, 1, None) == -1
+    assert lib.csa_compress(MIS, FAKE, FAKE, 1, 16, 64, 4, 1, 1, None) == -1
+    assert "aligned" in _err(lib)
+    assert lib.csa_compress(FAKE, FAKE, FAKE, 1, 16, 64, 4, 1, 7, None) == -1
+    # empty pool (no window closed) and empty batch are valid no-ops
+    assert lib.csa_compress(None, None, None, 1, 3, 64, 4, 1, 1, None) == 0
+    assert lib.csa_compress(None, None, None, 0, 64, 64, 4, 1, 1, None) == 0
+
+
+def test_index_topk_rejects(lib):
+    args = lambda **kw: [kw.get("q", FAKE), kw.get("w", FAKE), kw.get("k", FAKE), kw.get("B", 1),
+                         kw.get("S", 8), kw.get("pos", 0), kw.get("P", 2), kw.get("HI", 4),
+                         kw.get("dI", 32), kw.get("ratio", 4), kw.get("topk", 16),
+                         kw.get("idx", FAKE), None, None, 0, 1, None]
+    assert lib.csa_index_topk(*args(topk=0)) == -1
+    assert lib.csa_index_topk(*args(topk=4096)) == -1
+    assert lib.csa_index_topk(*args(dI=20)) == -1
+    assert lib.csa_index_topk(*args(HI=0)) == -1
+    assert lib.csa_index_topk(*args(pos=-1)) == -1
+    assert lib.csa_index_topk(*args(ratio=0)) == -1
+    assert lib.csa_index_topk(*args(idx=None)) == -1
+    assert lib.csa_index_topk(*args(q=MIS)) == -1
+    assert lib.csa_index_topk(*args(S=0)) == 0
+
+
+def _attend_args(**kw):
+    return [kw.get("q", FAKE), kw.get("kv", FAKE), kw.get("S_kv", 8), kw.get("kv_pos0", 0),
+            kw.get("pool", FAKE), kw.get("P", 2), kw.get("idx", FAKE), kw.get("topk", 4),
+            kw.get("sink", FAKE), kw.get("out", FAKE), kw.get("B", 1), kw.get("S_q", 8),
+            kw.get("q_pos0", 0), kw.get("H", 4), kw.get("D", 64), kw.get("R", 16),
+            kw.get("base", 10000.0), kw.get("W", 8), kw.get("ratio", 4), 0.125, None, 0, 1, None]
+
+
+def test_attend_rejects(lib):
+    assert lib.csa_attend(*_attend_args(R=15)) == -1
+    assert lib.csa_attend(*_attend_args(R=80)) == -1
+    assert lib.csa_attend(*_attend_args(D=60)) == -1
+    assert lib.csa_attend(*_attend_args(W=0)) == -1
+    assert lib.csa_attend(*_attend_args(q_pos0=-3)) == -1
+    assert lib.csa_attend(*_attend_args(base=0.0)) == -1
+    assert lib.csa_attend(*_attend_args(idx=None)) == -1
+    assert lib.csa_attend(*_attend_args(topk=0)) == -1
+    assert lib.csa_attend(*_attend_args(out=MIS)) == -1
+    assert lib.csa_attend(*_attend_args(B=0)) == 0
+    a = _attend_args(R=15)
+    del a[6:8]  # hca_attend has no idx / topk
+    assert lib.hca_attend(*a) == -1
+
+
+def test_binding_raises_without_device_tensors(lib):
+    import torch
+    x = torch.zeros(1, 8, 64)
+    with pytest.raises(ValueError):
+        csa.csa_compress(x, x, 4, True)

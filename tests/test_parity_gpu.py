@@ -1,0 +1,160 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle on the same seeded
+inputs.  Small and mid shapes are checked on every query row (several tiles and a ragged
+tail); the five full workloads are checked end to end on sampled rows, in the launch
+configuration the benchmark times.  Tolerances are in parity_util."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import csa_synth as cs
+from csa_synth import LayerSpec
+from parity_util import (TOL, GpuLayer, check_topk, kk_rows, oracle_attend, oracle_index,
+                         oracle_pool, rel_err, to_np)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+MID = [
+    # fp32, ragged sizes, two sequences
+    LayerSpec(name="mid_csa_f32", dtype="f32", B=2, S_q=301, S_kv=301, q_pos0=0, kv_pos0=0, H=8,
+              D=64, R=16, base=10000.0, W=32, m=4, P=75, kind="csa", H_I=4, d_I=32, topk=16,
+              workload=90),
+    # V4-Flash head shape, several key tiles, ragged tail
+    LayerSpec(name="mid_csa_bf16", dtype="bf16", B=2, S_q=603, S_kv=603, q_pos0=0, kv_pos0=0,
+              H=64, D=512, R=64, base=160000.0, W=128, m=4, P=150, kind="csa", H_I=64, d_I=128,
+              topk=64, workload=91),
+    LayerSpec(name="mid_hca_bf16", dtype="bf16", B=1, S_q=1000, S_kv=1000, q_pos0=0, kv_pos0=0,
+              H=64, D=512, R=64, base=160000.0, W=128, m=128, P=7, kind="hca", workload=92),
+    LayerSpec(name="mid_sliding_bf16", dtype="bf16", B=1, S_q=300, S_kv=300, q_pos0=0, kv_pos0=0,
+              H=16, D=128, R=32, base=10000.0, W=64, m=4, P=0, kind="sliding", workload=93),
+    LayerSpec(name="mid_decode_bf16", dtype="bf16", B=3, S_q=1, S_kv=128, q_pos0=4095,
+              kv_pos0=3968, H=64, D=512, R=64, base=160000.0, W=128, m=4, P=1024, kind="csa",
+              H_I=64, d_I=128, topk=64, decode=True, workload=94),
+    # odd shapes: general path
+    LayerSpec(name="odd_csa_bf16", dtype="bf16", B=1, S_q=77, S_kv=77, q_pos0=0, kv_pos0=0, H=5,
+              D=40, R=8, base=10000.0, W=9, m=3, P=25, kind="csa", H_I=3, d_I=24, topk=7,
+              workload=95),
+    # k > n_vis everywhere, window longer than the sequence
+    LayerSpec(name="sat_csa_f32", dtype="f32", B=1, S_q=50, S_kv=50, q_pos0=0, kv_pos0=0, H=4,
+              D=32, R=8, base=10000.0, W=64, m=4, P=12, kind="csa", H_I=2, d_I=16, topk=32,
+              workload=96),
+]
+
+
+def _inputs(spec):
+    return cs.make_inputs(spec, device=DEV)
+
+
+def _pool_input(spec, inp, ora_pool):
+    """Pool both sides attend over in the stage-wise check: the oracle's pool rounded to
+    the layer dtype (decode: the resident cache itself)."""
+    if spec.decode:
+        return inp["pool"]
+    if ora_pool is None:
+        return None
+    return torch.from_numpy(ora_pool).to(device=DEV, dtype=spec.torch_dtype)
+
+
+@pytest.mark.parametrize("spec", MID, ids=[s.name for s in MID])
+def test_compress_parity(spec):
+    if spec.decode or spec.kind == "sliding":
+        pytest.skip("no compressor in this layer")
+    inp = _inputs(spec)
+    gpu = GpuLayer(spec, inp).compress()
+    torch.cuda.synchronize()
+    ref = oracle_pool(spec, inp)
+    assert gpu.shape == ref.shape
+    assert rel_err(to_np(gpu), ref) <= TOL[spec.dtype]
+
+
+@pytest.mark.parametrize("spec", [s for s in MID if s.kind == "csa"],
+                         ids=[s.name for s in MID if s.kind == "csa"])
+def test_index_topk_parity(spec):
+    inp = _inputs(spec)
+    idx, scores = GpuLayer(spec, inp).index(want_scores=True)
+    torch.cuda.synchronize()
+    rows = list(range(spec.S_q))
+    sc, o_idx, o_sel = oracle_index(spec, inp, rows)
+    g_idx = idx.cpu().numpy()
+    g_sc = scores.cpu().numpy().astype(np.float64)
+    for b in range(spec.B):
+        check_topk(g_idx[b], o_idx[b], sc[b], kk_rows(spec, rows))
+        # scores of the kept entries, where the sets agree slot by slot
+        same = (g_idx[b] == o_idx[b]) & (o_idx[b] >= 0)
+        if same.any():
+            assert rel_err(g_sc[b][same], o_sel[b][same]) <= TOL[spec.dtype] * 0.05
+
+
+@pytest.mark.parametrize("spec", MID, ids=[s.name for s in MID])
+def test_attend_stagewise_parity(spec):
+    """Both sides attend over identical inputs: the oracle's pool (rounded to the layer
+    dtype) and the oracle's top-k."""
+    inp = _inputs(spec)
+    rows = list(range(spec.S_q))
+    ora_pool = oracle_pool(spec, inp)
+    pool_in = _pool_input(spec, inp, ora_pool)
+    idx_in = None
+    o_idx = None
+    if spec.kind == "csa":
+        _, o_idx, _ = oracle_index(spec, inp, rows)
+        idx_in = torch.from_numpy(o_idx).to(DEV)
+    out = GpuLayer(spec, inp).attend(pool_in, idx_in)
+    torch.cuda.synchronize()
+    ref = oracle_attend(spec, inp, rows, None if pool_in is None else to_np(pool_in), o_idx)
+    assert rel_err(to_np(out), ref) <= TOL[spec.dtype]
+
+
+def _end_to_end(spec, rows, inp=None):
+    inp = _inputs(spec) if inp is None else inp
+    layer = GpuLayer(spec, inp)
+    pool = None
+    if spec.decode:
+        pool = inp["pool"]
+    elif spec.kind != "sliding":
+        pool = layer.compress()
+    idx = layer.index(want_scores=False) if spec.kind == "csa" else None
+    out = layer.attend(pool, idx)
+    torch.cuda.synchronize()
+    rows_t = torch.tensor(rows, device=DEV)
+    g_out = to_np(out[:, rows_t])
+    ora_pool = oracle_pool(spec, inp)
+    if pool is not None and not spec.decode:
+        assert rel_err(to_np(pool), ora_pool) <= TOL[spec.dtype]
+    keep = np.ones((spec.B, len(rows)), dtype=bool)
+    o_idx = None
+    if spec.kind == "csa":
+        sc, o_idx, _ = oracle_index(spec, inp, rows)
+        g_idx = idx[:, rows_t].cpu().numpy()
+        for b in range(spec.B):
+            check_topk(g_idx[b], o_idx[b], sc[b], kk_rows(spec, rows))
+            for r in range(len(rows)):
+                keep[b, r] = set(g_idx[b, r].tolist()) == set(o_idx[b, r].tolist())
+    ref = oracle_attend(spec, inp, rows, ora_pool, o_idx)
+    # rows whose top-k legitimately differs inside the tie band attend over other keys
+    assert keep.mean() > 0.9
+    assert rel_err(g_out[keep], ref[keep]) <= TOL[spec.dtype]
+    return inp, out
+
+
+@pytest.mark.parametrize("spec", MID, ids=[s.name for s in MID])
+def test_end_to_end_parity(spec):
+    _end_to_end(spec, list(range(spec.S_q)))
+
+
+@pytest.mark.parametrize("workload", [0, 1, 2, 3])
+def test_workload_end_to_end(workload):
+    for spec in cs.WORKLOADS[workload]:
+        rows = list(range(spec.S_q)) if spec.S_q <= 512 else cs.sample_rows(spec, n_random=96)
+        _end_to_end(spec, rows)
+        torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("layer", [0, 1, 2, 3])
+def test_mixed_stack_layer_end_to_end(layer):
+    spec = cs.WORKLOADS[4][layer]
+    rows = cs.sample_rows(spec, n_random=48)
+    _end_to_end(spec, rows)
+    torch.cuda.empty_cache()
