@@ -149,6 +149,11 @@ size_t csa_attend_workspace_bytes(int32_t mode, int64_t B, int64_t S_q, int64_t 
 /* Message for the last error returned on the calling host thread ("" if none). */
 const char *csa_last_error(void);
 
+/* Nonzero if a kernel of this library gave up on a bounded wait (and skipped the rest
+ * of its work) since the last call; bit 0: attention.  Synchronises the device and
+ * clears the flags.  For tests and diagnostics. */
+uint32_t csa_device_status(void);
+
 /* Number of kernels this library has enqueued in this process (all devices, all
  * threads); for accounting launches in a timed region. */
 uint64_t csa_launch_count(void);

@@ -16,7 +16,7 @@ import torch
 
 __all__ = ["csa_compress", "csa_index_topk", "csa_attend", "hca_attend",
            "csa_index_topk_workspace_bytes", "csa_attend_workspace_bytes", "library_path",
-           "load_library", "launch_count", "CsaError", "CSA_F32", "CSA_BF16"]
+           "load_library", "launch_count", "device_status", "CsaError", "CSA_F32", "CSA_BF16"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libcsa_b200.so")
@@ -62,6 +62,7 @@ def load_library():
     lib.csa_last_error.restype = ctypes.c_char_p
     lib.csa_version.restype = ctypes.c_char_p
     lib.csa_launch_count.restype = ctypes.c_uint64
+    lib.csa_device_status.restype = ctypes.c_uint32
     _lib = lib
     return lib
 
@@ -69,6 +70,11 @@ def load_library():
 def launch_count() -> int:
     """Kernels the library has enqueued in this process."""
     return int(load_library().csa_launch_count())
+
+
+def device_status() -> int:
+    """Nonzero if a kernel gave up on a bounded wait since the last call (synchronises)."""
+    return int(load_library().csa_device_status())
 
 
 def _dtype_code(t: torch.Tensor) -> int:

@@ -39,6 +39,12 @@ csa_status_t attend_general(const AttendArgs &a, cudaStream_t st);
 // Scratch bytes the chosen path needs.
 size_t attend_workspace(const AttendArgs &a);
 
+// Tensor-core path (bf16, H = 64, D = 512): eligibility, workspace, launch.
+bool attend_tc_eligible(const AttendArgs &a);
+size_t attend_tc_workspace(const AttendArgs &a);
+csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st);
+unsigned int read_attend_tc_status();
+
 // Picks the kernel for a validated call.
 csa_status_t attend_dispatch(const AttendArgs &a, cudaStream_t st);
 

@@ -41,13 +41,24 @@ csa_status_t index_topk_dispatch(const void *qI, const void *w, const void *kI, 
                               scores_opt, dtype, st);
 }
 
-size_t attend_workspace(const AttendArgs &) { return 0; }
+size_t attend_workspace(const AttendArgs &a) {
+    return attend_tc_eligible(a) ? attend_tc_workspace(a) : 0;
+}
 
-csa_status_t attend_dispatch(const AttendArgs &a, cudaStream_t st) { return attend_general(a, st); }
+csa_status_t attend_dispatch(const AttendArgs &a, cudaStream_t st) {
+    if (attend_tc_eligible(a)) return attend_tc(a, st);
+    return attend_general(a, st);
+}
 
 }  // namespace csa
 
 extern "C" const char *csa_last_error(void) { return csa::g_error; }
+
+extern "C" uint32_t csa_device_status(void) {
+    uint32_t s = 0;
+    if (csa::read_attend_tc_status()) s |= 1u;
+    return s;
+}
 
 extern "C" uint64_t csa_launch_count(void) { return csa::g_launches.load(); }
 

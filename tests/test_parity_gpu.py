@@ -33,6 +33,14 @@ MID = [
     LayerSpec(name="mid_decode_bf16", dtype="bf16", B=3, S_q=1, S_kv=128, q_pos0=4095,
               kv_pos0=3968, H=64, D=512, R=64, base=160000.0, W=128, m=4, P=1024, kind="csa",
               H_I=64, d_I=128, topk=64, decode=True, workload=94),
+    # V4-Flash head shape on the tensor-core path: window-only layer, and a CSA layer
+    # whose key count per query is not a multiple of the 128-key tile
+    LayerSpec(name="mid_sliding_tc_bf16", dtype="bf16", B=2, S_q=333, S_kv=333, q_pos0=0,
+              kv_pos0=0, H=64, D=512, R=64, base=10000.0, W=128, m=4, P=0, kind="sliding",
+              workload=97),
+    LayerSpec(name="mid_csa_ragged_bf16", dtype="bf16", B=1, S_q=700, S_kv=700, q_pos0=0,
+              kv_pos0=0, H=64, D=512, R=64, base=160000.0, W=100, m=4, P=175, kind="csa",
+              H_I=64, d_I=128, topk=37, workload=98),
     # odd shapes: general path
     LayerSpec(name="odd_csa_bf16", dtype="bf16", B=1, S_q=77, S_kv=77, q_pos0=0, kv_pos0=0, H=5,
               D=40, R=8, base=10000.0, W=9, m=3, P=25, kind="csa", H_I=3, d_I=24, topk=7,
@@ -105,6 +113,26 @@ def test_attend_stagewise_parity(spec):
     torch.cuda.synchronize()
     ref = oracle_attend(spec, inp, rows, None if pool_in is None else to_np(pool_in), o_idx)
     assert rel_err(to_np(out), ref) <= TOL[spec.dtype]
+
+
+def test_tensor_core_path_selected():
+    """The V4-Flash prefill shapes take the tensor-core attention (it needs a workspace
+    for the rotated keys); decode-like and odd shapes take the general path."""
+    import sparse_attention_14_b200 as csa
+    for spec in MID + cs.WORKLOADS[1] + cs.WORKLOADS[2] + cs.WORKLOADS[3]:
+        ws = csa.csa_attend_workspace_bytes(0 if spec.kind == "csa" else 1, spec.B, spec.S_q,
+                                            spec.S_kv, spec.P, spec.H, spec.D, spec.topk,
+                                            spec.torch_dtype)
+        tc = spec.dtype == "bf16" and spec.H == 64 and spec.D == 512 and \
+            spec.S_q * 64 >= spec.S_kv + spec.P
+        assert (ws > 0) == tc, spec.name
+
+
+def test_no_kernel_gave_up():
+    import sparse_attention_14_b200 as csa
+    spec = MID[1]
+    _end_to_end(spec, list(range(spec.S_q)))
+    assert csa.device_status() == 0
 
 
 def _end_to_end(spec, rows, inp=None):
