@@ -141,6 +141,38 @@ csa_status_t hca_attend(const void *q, const void *kv, int64_t S_kv, int64_t kv_
                         void *workspace, size_t workspace_bytes, csa_dtype_t dtype,
                         void *stream);
 
+/*
+ * csa_attend_noalloc -- csa_attend for callers that cannot allocate device memory.
+ * The pages have no counterpart to this call; it exists for users of this library.
+ *
+ * Some callers cannot call cudaMalloc or pass a scratch buffer: a custom operator
+ * inside a host framework that hands the operator only its input and output buffers
+ * and owns every other byte of device memory through its own allocator (a raw
+ * cudaMalloc would bypass its accounting and can fail under its memory budget), or a
+ * latency-critical serving loop that must not allocate per call because cudaMalloc can
+ * synchronise the device.  This entry point takes the same arguments as csa_attend
+ * minus the workspace and allocates nothing: its scratch (the rotated window rows and
+ * compressed entries of the call) lives in one fixed device array of 16 MiB compiled
+ * into the library, created on each GPU that loads the library and held until the
+ * process exits.  The caller still provides q, kv, pool, idx, sink and out.
+ *
+ *  - Handles the bf16, H = 64, D = 512 prefill shape (S_q * 64 >= S_kv + P) with
+ *    B * (S_kv + P) <= 16384 rows of scratch; anything else returns
+ *    CSA_ERR_UNSUPPORTED with a message naming the limit.
+ *  - The first call on a device looks up the array's device address (set-up, once per
+ *    device, with that device current); make that first call before any stream capture.
+ *  - Every call on a device shares the one array, and it keeps the last call's contents
+ *    (every row a call reads is written by that call first).  Calls whose work overlaps
+ *    on the GPU (different streams, or different host threads) race on it: serialise
+ *    them, e.g. on one stream.
+ */
+csa_status_t csa_attend_noalloc(const void *q, const void *kv, int64_t S_kv, int64_t kv_pos0,
+                                const void *pool, int64_t P, const int32_t *idx, int32_t topk,
+                                const float *sink, void *out, int64_t B, int64_t S_q,
+                                int64_t q_pos0, int32_t H, int32_t D, int32_t rope_dim,
+                                double rope_base, int32_t window, int32_t ratio, float scale,
+                                csa_dtype_t dtype, void *stream);
+
 /* Scratch bytes csa_attend (mode 0) or hca_attend (mode 1) needs for these sizes. */
 size_t csa_attend_workspace_bytes(int32_t mode, int64_t B, int64_t S_q, int64_t S_kv,
                                   int64_t P, int32_t H, int32_t D, int32_t topk,

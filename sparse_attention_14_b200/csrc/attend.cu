@@ -224,7 +224,7 @@ csa_status_t attend_general(const AttendArgs &a, cudaStream_t st) {
     return a.dtype == CSA_F32 ? launch_simt<float>(a, st) : launch_simt<__nv_bfloat16>(a, st);
 }
 
-static csa_status_t attend_entry(AttendArgs &a, void *stream) {
+static csa_status_t attend_entry(AttendArgs &a, void *stream, bool no_alloc = false) {
     const char *fn = a.mode == 0 ? "csa_attend" : "hca_attend";
     CSA_REQUIRE(a.B >= 0 && a.S_q >= 0 && a.S_kv >= 0 && a.P >= 0, CSA_ERR_INVALID_ARG,
                 "%s: negative size", fn);
@@ -251,6 +251,10 @@ static csa_status_t attend_entry(AttendArgs &a, void *stream) {
     CSA_REQUIRE(aligned(a.q, 16) && aligned(a.kv, 16) && aligned(a.pool, 16) &&
                     aligned(a.out, 16) && aligned(a.idx, 4) && aligned(a.sink, 4),
                 CSA_ERR_INVALID_ARG, "%s: misaligned pointer", fn);
+    if (no_alloc) {
+        make_rope_table(&a.rope, a.D, a.rope_dim, a.rope_base);
+        return attend_tc_noalloc(a, reinterpret_cast<cudaStream_t>(stream));
+    }
     size_t need = attend_workspace(a);
     CSA_REQUIRE(a.workspace_bytes >= need && (need == 0 || a.workspace), CSA_ERR_WORKSPACE,
                 "%s: workspace of %zu B given, %zu B needed", fn, a.workspace_bytes, need);
@@ -285,6 +289,20 @@ extern "C" csa_status_t hca_attend(const void *q, const void *kv, int64_t S_kv, 
                       sink, out, B, S_q, q_pos0, H, D, rope_dim, rope_base, window, ratio,
                       scale, workspace, workspace_bytes, dtype, 1, {}};
     return csa::attend_entry(a, stream);
+}
+
+extern "C" csa_status_t csa_attend_noalloc(const void *q, const void *kv, int64_t S_kv,
+                                           int64_t kv_pos0, const void *pool, int64_t P,
+                                           const int32_t *idx, int32_t topk, const float *sink,
+                                           void *out, int64_t B, int64_t S_q, int64_t q_pos0,
+                                           int32_t H, int32_t D, int32_t rope_dim,
+                                           double rope_base, int32_t window, int32_t ratio,
+                                           float scale, csa_dtype_t dtype, void *stream) {
+    csa::clear_error();
+    csa::AttendArgs a{q,  kv, S_kv,  kv_pos0,  pool,      P,         idx,       topk,
+                      sink, out, B, S_q, q_pos0, H, D, rope_dim, rope_base, window, ratio,
+                      scale, nullptr, 0, dtype, 0, {}};
+    return csa::attend_entry(a, stream, true);
 }
 
 extern "C" size_t csa_attend_workspace_bytes(int32_t mode, int64_t B, int64_t S_q, int64_t S_kv,

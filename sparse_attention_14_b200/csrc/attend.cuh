@@ -44,6 +44,8 @@ bool attend_tc_eligible(const AttendArgs &a);
 size_t attend_tc_workspace(const AttendArgs &a);
 csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st);
 unsigned int read_attend_tc_status();
+// Same kernel with its scratch in a fixed device array (csa_attend_noalloc).
+csa_status_t attend_tc_noalloc(AttendArgs &a, cudaStream_t st);
 
 // Picks the kernel for a validated call.
 csa_status_t attend_dispatch(const AttendArgs &a, cudaStream_t st);

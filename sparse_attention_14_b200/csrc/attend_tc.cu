@@ -22,6 +22,8 @@
 //    the sink enters as the initial running max and once in the final sum;
 //  * epilogue: O^T / l, the -t de-rotation of the rope channels (partner channel via a
 //    lane shuffle), transposed through shared memory into coalesced 16-byte stores.
+#include <mutex>
+
 #include "attend.cuh"
 #include "umma.cuh"
 
@@ -462,6 +464,52 @@ csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st) {
         a.window, a.ratio, a.scale, a.rope);
     CSA_CHECK_LAUNCH(a.mode == 0 ? "csa_attend" : "hca_attend");
     return CSA_OK;
+}
+
+// ------------------------------------------------------------------ no-allocation variant
+// Scratch for csa_attend_noalloc: the rotated window rows and entries of one call live in
+// this fixed device array instead of a caller-provided workspace.  It is created when the
+// library is loaded on a device and kept until the process exits.
+constexpr size_t kNoAllocScratchBytes = (size_t)16 << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kMaxDevices];  // device address of g_noalloc_scratch, per device
+}  // namespace
+
+csa_status_t attend_tc_noalloc(AttendArgs &a, cudaStream_t st) {
+    CSA_REQUIRE(attend_tc_eligible(a), CSA_ERR_UNSUPPORTED,
+                "csa_attend_noalloc: only the bf16, 64-head, head_dim-512 prefill shape is "
+                "handled (S_q * 64 >= S_kv + P)");
+    const size_t need = attend_tc_workspace(a);
+    CSA_REQUIRE(need <= kNoAllocScratchBytes, CSA_ERR_UNSUPPORTED,
+                "csa_attend_noalloc: needs %zu B of scratch for B*(S_kv+P) rotated rows, the "
+                "fixed scratch holds %zu B (at most %zu rows of 512 bf16)",
+                need, kNoAllocScratchBytes, kNoAllocScratchBytes / 1024);
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    CSA_REQUIRE(e == cudaSuccess && dev >= 0 && dev < kMaxDevices, CSA_ERR_CUDA,
+                "csa_attend_noalloc: cudaGetDevice failed: %s", cudaGetErrorString(e));
+    void *ptr = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_noalloc_mu);
+        if (!g_noalloc_ptr[dev]) {
+            // one-time set-up on this device (the current one): the host-side symbol is a
+            // stand-in, the kernels need the array's device address
+            e = cudaGetSymbolAddress(&g_noalloc_ptr[dev], g_noalloc_scratch);
+            if (e != cudaSuccess) {
+                g_noalloc_ptr[dev] = nullptr;
+                set_error("csa_attend_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
+                return CSA_ERR_CUDA;
+            }
+        }
+        ptr = g_noalloc_ptr[dev];
+    }
+    a.workspace = ptr;
+    a.workspace_bytes = kNoAllocScratchBytes;
+    return attend_tc(a, st);
 }
 
 unsigned int read_attend_tc_status() {
