@@ -73,7 +73,11 @@ def algorithmic_work(spec):
             idx_flops += 2 * spec.H_I * spec.d_I * nv
     w["attend_flops"] = 4 * spec.B * spec.H * spec.D * keys
     w["index_flops"] = spec.B * idx_flops
-    w["attend_bytes"] = spec.B * (2 * spec.S_q * spec.H * spec.D + (spec.S_kv + spec.P) * spec.D) * e
+    # distinct rows an attention call must read: every window row it touches, and at most
+    # min(P, S_q*k) (CSA) / P (HCA) entries
+    ent_rows = min(spec.P, spec.S_q * spec.topk) if spec.kind == "csa" else spec.P
+    win_rows = min(spec.S_kv, spec.S_q + spec.W - 1)
+    w["attend_bytes"] = spec.B * (2 * spec.S_q * spec.H * spec.D + (win_rows + ent_rows) * spec.D) * e
     if spec.kind == "csa":
         w["index_bytes"] = spec.B * (spec.S_q * spec.H_I * (spec.d_I + 1) + spec.P * spec.d_I) * e \
             + spec.B * spec.S_q * spec.topk * 4
@@ -159,7 +163,8 @@ class LayerRunner:
         self.idx = torch.empty((s.B, s.S_q, s.topk), dtype=torch.int32, device=device) \
             if s.kind == "csa" else None
         self.out = torch.empty_like(self.inp["q"])
-        wsi = csa.csa_index_topk_workspace_bytes(s.B, s.S_q, s.P, s.H_I, s.d_I, s.topk, dt) \
+        wsi = csa.csa_index_topk_workspace_bytes(s.B, s.S_q, s.q_pos0, s.P, s.H_I, s.d_I, s.m,
+                                                 s.topk, dt) \
             if s.kind == "csa" else 0
         wsa = csa.csa_attend_workspace_bytes(0 if s.kind == "csa" else 1, s.B, s.S_q, s.S_kv, s.P,
                                              s.H, s.D, s.topk, dt)

@@ -77,8 +77,8 @@ csa_status_t csa_compress(const void *kv, const void *gate, void *pool, int64_t 
  *
  *   score[t,j] = sum_{h < H_I} w[b,i,h] * max(0, <q_I[b,i,h,:], k_I[b,j,:]>)
  *   for the visible entries j < n_vis(t) = min(P, floor((t+1)/ratio)), t = q_pos0 + i.
- *   idx[b,i,:] = the min(topk, n_vis) best entries, score descending (ties: lower j
- *   first), then -1 padding.
+ *   idx[b,i,:] = the min(topk, n_vis) best entries (ranked by score descending, equal
+ *   scores by lower j first), listed in ascending entry order, then -1 padding.
  *
  *   q_I : [B, S_q, H_I, d_I]   w : [B, S_q, H_I]   k_I : [B, P, d_I]
  *   idx : [B, S_q, topk] int32 output
@@ -93,8 +93,11 @@ csa_status_t csa_index_topk(const void *q_I, const void *w, const void *k_I, int
                             void *workspace, size_t workspace_bytes, csa_dtype_t dtype,
                             void *stream);
 
-size_t csa_index_topk_workspace_bytes(int64_t B, int64_t S_q, int64_t P, int32_t H_I,
-                                      int32_t d_I, int32_t topk, csa_dtype_t dtype);
+/* Scratch bytes csa_index_topk needs for these sizes (0 when the call needs none; a
+ * decode-sized call is split over entry ranges and merges through the workspace). */
+size_t csa_index_topk_workspace_bytes(int64_t B, int64_t S_q, int64_t q_pos0, int64_t P,
+                                      int32_t H_I, int32_t d_I, int32_t ratio, int32_t topk,
+                                      csa_dtype_t dtype);
 
 /*
  * csa_attend -- CSA attention: shared K=V single-head MQA over the sliding window plus
@@ -182,7 +185,7 @@ size_t csa_attend_workspace_bytes(int32_t mode, int64_t B, int64_t S_q, int64_t 
 const char *csa_last_error(void);
 
 /* Nonzero if a kernel of this library gave up on a bounded wait (and skipped the rest
- * of its work) since the last call; bit 0: attention.  Synchronises the device and
+ * of its work) since the last call; bit 0: attention, bit 1: indexer.  Synchronises the device and
  * clears the flags.  For tests and diagnostics. */
 uint32_t csa_device_status(void);
 

@@ -47,7 +47,8 @@ def load_library():
     lib.csa_compress.argtypes = [vp, vp, vp, i64, i64, i32, i32, i32, ctypes.c_int, vp]
     lib.csa_index_topk.argtypes = [vp, vp, vp, i64, i64, i64, i64, i32, i32, i32, i32, vp, vp, vp,
                                    sz, ctypes.c_int, vp]
-    lib.csa_index_topk_workspace_bytes.argtypes = [i64, i64, i64, i32, i32, i32, ctypes.c_int]
+    lib.csa_index_topk_workspace_bytes.argtypes = [i64, i64, i64, i64, i32, i32, i32, i32,
+                                                   ctypes.c_int]
     lib.csa_index_topk_workspace_bytes.restype = sz
     lib.csa_attend.argtypes = [vp, vp, i64, i64, vp, i64, vp, i32, vp, vp, i64, i64, i64, i32, i32,
                                i32, ctypes.c_double, i32, i32, ctypes.c_float, vp, sz,
@@ -129,9 +130,11 @@ def csa_compress(kv: torch.Tensor, gate: torch.Tensor, ratio: int, overlap: bool
     return pool
 
 
-def csa_index_topk_workspace_bytes(B, S_q, P, H_I, d_I, topk, dtype=torch.bfloat16) -> int:
+def csa_index_topk_workspace_bytes(B, S_q, q_pos0, P, H_I, d_I, ratio, topk,
+                                   dtype=torch.bfloat16) -> int:
     code = CSA_F32 if dtype == torch.float32 else CSA_BF16
-    return int(load_library().csa_index_topk_workspace_bytes(B, S_q, P, H_I, d_I, topk, code))
+    return int(load_library().csa_index_topk_workspace_bytes(B, S_q, q_pos0, P, H_I, d_I, ratio,
+                                                             topk, code))
 
 
 def csa_index_topk(q_I: torch.Tensor, w: torch.Tensor, k_I: torch.Tensor, q_pos0: int, ratio: int,
@@ -144,8 +147,8 @@ def csa_index_topk(q_I: torch.Tensor, w: torch.Tensor, k_I: torch.Tensor, q_pos0
     if idx is None:
         idx = torch.empty((B, S_q, topk), dtype=torch.int32, device=q_I.device)
     scores = torch.empty((B, S_q, topk), dtype=torch.float32, device=q_I.device) if want_scores else None
-    ws, wsb = _ws(csa_index_topk_workspace_bytes(B, S_q, P, H_I, d_I, topk, q_I.dtype), q_I.device,
-                  workspace)
+    ws, wsb = _ws(csa_index_topk_workspace_bytes(B, S_q, q_pos0, P, H_I, d_I, ratio, topk,
+                                                 q_I.dtype), q_I.device, workspace)
     _call("csa_index_topk", _ptr(q_I), _ptr(w), _ptr(k_I), B, S_q, q_pos0, P, H_I, d_I, ratio, topk,
           _ptr(idx), _ptr(scores), _ptr(ws), wsb, _dtype_code(q_I), _stream(stream))
     return (idx, scores) if want_scores else idx

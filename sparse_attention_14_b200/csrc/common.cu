@@ -31,12 +31,20 @@ void make_rope_table(RopeTable *t, int D, int R, double base) {
 }
 
 // ------------------------------------------------------------------ path selection
-size_t index_topk_workspace(int64_t, int64_t, int64_t, int, int, int, csa_dtype_t) { return 0; }
+size_t index_topk_workspace(int64_t B, int64_t S_q, int64_t q_pos0, int64_t P, int H_I,
+                            int d_I, int ratio, int topk, csa_dtype_t dtype) {
+    if (!index_tc_eligible(B, S_q, P, H_I, d_I, topk, dtype)) return 0;
+    return index_tc_workspace(B, S_q, q_pos0, P, ratio, topk);
+}
 
 csa_status_t index_topk_dispatch(const void *qI, const void *w, const void *kI, int64_t B,
                                  int64_t S_q, int64_t q_pos0, int64_t P, int H_I, int d_I,
-                                 int ratio, int topk, int32_t *idx, float *scores_opt, void *,
-                                 size_t, csa_dtype_t dtype, cudaStream_t st) {
+                                 int ratio, int topk, int32_t *idx, float *scores_opt,
+                                 void *workspace, size_t workspace_bytes, csa_dtype_t dtype,
+                                 cudaStream_t st) {
+    if (index_tc_eligible(B, S_q, P, H_I, d_I, topk, dtype))
+        return index_tc(qI, w, kI, B, S_q, q_pos0, P, ratio, topk, idx, scores_opt, workspace,
+                        workspace_bytes, st);
     return index_topk_general(qI, w, kI, B, S_q, q_pos0, P, H_I, d_I, ratio, topk, idx,
                               scores_opt, dtype, st);
 }
@@ -57,6 +65,7 @@ extern "C" const char *csa_last_error(void) { return csa::g_error; }
 extern "C" uint32_t csa_device_status(void) {
     uint32_t s = 0;
     if (csa::read_attend_tc_status()) s |= 1u;
+    if (csa::read_index_tc_status()) s |= 2u;
     return s;
 }
 

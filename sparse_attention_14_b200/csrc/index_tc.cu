@@ -1,0 +1,562 @@
+// index_tc.cu -- tensor-core Lightning Indexer + streaming top-k for the V4-Flash indexer
+// shape (H_I = 64 heads, d_I = 128, bf16).
+//
+//   score[t,j] = sum_h w[t,h] * max(0, <q_I[t,h], k_I[j]>)      (HF docs model_doc/
+//   deepseek_v4, section 2.3.1; the -1 marker of "Attention mask layout")
+//
+// Design:
+//  * the GEMM is transposed so that the per-thread epilogue is a private sum:
+//      D[j, (q,h)] = k_I[j, :] . q_I[q, h, :]     M = 128 entries (A = k_I tile, TMA,
+//      K-major, 128B swizzle), N = QB queries x 64 heads (B = q_I rows of the query
+//      block, loaded once), K = 128; fp32 accumulators in TMEM, double-buffered;
+//  * warp roles: warp 0 issues TMA loads into a ring of entry tiles, warp 1 issues the
+//    MMAs (one thread), the epilogue warps read D from TMEM (thread = entry row) and
+//    form sum_h w[q,h] ReLU(D) for their queries, while the next tile's MMA runs;
+//  * top-k without writing scores to HBM: each query keeps a candidate buffer of
+//    1024 64-bit keys (order-preserving score bits, then the complemented entry index,
+//    so that equal scores rank the lower index first) and a threshold; a tile inserts
+//    only keys above the threshold, and whenever the buffer could overflow it is cut
+//    back to exactly k by an exact radix select over the 64-bit keys (which then becomes
+//    the threshold);
+//  * output: the k survivors in ascending entry order (deterministic), or, for a
+//    decode-sized problem split over entry ranges, each range's candidates go to the
+//    workspace and a merge kernel selects the final k.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "index_topk.cuh"
+#include "topk.cuh"
+#include "umma.cuh"
+
+namespace csa {
+
+__device__ unsigned int g_index_tc_status;
+
+namespace {
+
+using namespace umma;
+
+constexpr int kDI = 128, kHI = 64, kTileE = 128, kCap = 1024;
+constexpr int kMaxTopk = kCap - kTileE;   // room for one tile after a cut to k
+
+struct Misc {
+    uint64_t full[4], empty[4], tfull[2], tempty[2], bfull;
+    uint32_t tmem_base;
+    unsigned cnt[4];
+    unsigned long long thr[4];
+    unsigned long long sel_prefix[4];
+    unsigned sel_remaining[4];
+    unsigned warp_part[4][8];
+    int abort_;
+};
+
+template <int QB>
+struct Cfg {
+    static constexpr int N = QB * 64;
+    static constexpr int NE = QB == 4 ? 8 : 4;          // epilogue warps
+    static constexpr int kThreads = (2 + NE) * 32;
+    static constexpr int NST = QB == 4 ? 3 : 4;          // entry-tile stages
+    static constexpr uint32_t kBChunk = QB * 64 * 128;   // one 64-column chunk of q_I rows
+    static constexpr uint32_t kBBytes = 2 * kBChunk;
+    static constexpr uint32_t kABytes = kTileE * kDI * 2;
+    static constexpr int GS = NE * 32 / QB;              // threads per query group
+    static constexpr int QPT = QB == 4 ? 2 : QB;         // queries per epilogue thread
+    static constexpr uint32_t kTmemCols = 2 * N <= 128 ? 128 : (2 * N <= 256 ? 256 : 512);
+    static constexpr uint32_t kOffB = 0;
+    static constexpr uint32_t kOffA = kBBytes;
+    static constexpr uint32_t kOffCand = kOffA + NST * kABytes;
+    static constexpr uint32_t kOffHist = kOffCand + QB * kCap * 8;
+    static constexpr uint32_t kOffW = kOffHist + QB * 256 * 4;
+    static constexpr uint32_t kOffMisc = kOffW + QB * 64 * 4;
+    static constexpr size_t kSmem = kOffMisc + sizeof(Misc) + 1024;
+};
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        :
+        : "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ float key_to_float(uint32_t key) {
+    uint32_t u = (key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key;
+    return __uint_as_float(u);
+}
+
+// ------------------------------------------------------------------ group selection
+// All GS threads of a group (named barrier `bar`) find the k-th largest of n unique
+// 64-bit keys by an MSB-first radix select, 8 bits per pass.
+template <int GS>
+__device__ unsigned long long group_kth(const unsigned long long *a, int n, int k, int gt, int bar,
+                                        unsigned *hist, Misc &ms, int g) {
+    constexpr int BPT = 256 / GS;
+    const int lane = gt & 31, wid = gt >> 5;
+    if (gt == 0) {
+        ms.sel_prefix[g] = 0ull;
+        ms.sel_remaining[g] = (unsigned)k;
+    }
+    for (int shift = 56; shift >= 0; shift -= 8) {
+        for (int i = gt; i < 256; i += GS) hist[i] = 0u;
+        named_sync(bar, GS);
+        const unsigned long long prefix = ms.sel_prefix[g];
+        const unsigned remaining = ms.sel_remaining[g];
+        const unsigned long long mask = shift == 56 ? 0ull : (~0ull << (shift + 8));
+        for (int e = gt; e < n; e += GS) {
+            const unsigned long long key = a[e];
+            if ((key & mask) == prefix) atomicAdd(&hist[(unsigned)(key >> shift) & 255u], 1u);
+        }
+        named_sync(bar, GS);
+        const int hi_bin = 256 - gt * BPT;   // my bins: [hi_bin - BPT, hi_bin)
+        unsigned local = 0;
+#pragma unroll
+        for (int b = 1; b <= BPT; ++b) local += hist[hi_bin - b];
+        unsigned incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            unsigned v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (lane == 31) ms.warp_part[g][wid] = incl;
+        named_sync(bar, GS);
+        unsigned cum = incl - local;
+        for (int w = 0; w < wid; ++w) cum += ms.warp_part[g][w];
+#pragma unroll
+        for (int b = 1; b <= BPT; ++b) {
+            const int bin = hi_bin - b;
+            const unsigned h = hist[bin];
+            if (cum < remaining && remaining <= cum + h) {
+                ms.sel_prefix[g] = prefix | ((unsigned long long)bin << shift);
+                ms.sel_remaining[g] = remaining - cum;
+            }
+            cum += h;
+        }
+        named_sync(bar, GS);
+    }
+    return ms.sel_prefix[g];
+}
+
+// Cut a query's candidate buffer back to its k largest keys (keys >= the k-th).
+template <int GS>
+__device__ void group_cut(unsigned long long *cand, int k, int gt, int bar, unsigned *hist, Misc &ms,
+                          int g, int q) {
+    constexpr int EPT = kCap / GS;
+    const int n = (int)ms.cnt[q];
+    if (n <= k) return;   // uniform within the group
+    const unsigned long long T = group_kth<GS>(cand, n, k, gt, bar, hist, ms, g);
+    unsigned long long mine[EPT];
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) {
+        const int e = gt + i * GS;
+        mine[i] = e < n ? cand[e] : 0ull;
+    }
+    named_sync(bar, GS);
+    if (gt == 0) ms.cnt[q] = 0;
+    named_sync(bar, GS);
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) {
+        if (mine[i] != 0ull && mine[i] >= T) {
+            const unsigned pos = atomicAdd(&ms.cnt[q], 1u);
+            cand[pos] = mine[i];
+        }
+    }
+    if (gt == 0) ms.thr[q] = T;
+    named_sync(bar, GS);
+}
+
+// Sort the first n keys by entry index ascending (low word descending) and write idx /
+// scores for one query row.
+template <int GS>
+__device__ void group_emit(unsigned long long *cand, int n, int k, int gt, int bar, int32_t *idx_row,
+                           float *score_row) {
+    const int N2 = pow2_ceil(n > 0 ? n : 1);
+    for (int e = n + gt; e < N2; e += GS) cand[e] = 0ull;
+    named_sync(bar, GS);
+    for (int size = 2; size <= N2; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int i = gt; i < N2 / 2; i += GS) {
+                const int lo = 2 * i - (i & (stride - 1));
+                const int hi = lo + stride;
+                const bool desc = (lo & size) == 0;
+                const unsigned long long a = cand[lo], b = cand[hi];
+                const uint32_t la = (uint32_t)a, lb = (uint32_t)b;
+                if ((la < lb) == desc) {
+                    cand[lo] = b;
+                    cand[hi] = a;
+                }
+            }
+            named_sync(bar, GS);
+        }
+    }
+    for (int r = gt; r < k; r += GS) {
+        if (r < n) {
+            const unsigned long long c = cand[r];
+            idx_row[r] = (int32_t)(0xFFFFFFFFu - (uint32_t)c);
+            if (score_row) score_row[r] = key_to_float((uint32_t)(c >> 32));
+        } else {
+            idx_row[r] = -1;
+            if (score_row) score_row[r] = __int_as_float(0x7fc00000);
+        }
+    }
+}
+
+// ------------------------------------------------------------------ main kernel
+template <int QB>
+__global__ void __launch_bounds__(Cfg<QB>::kThreads, 1) index_tc_kernel(
+    const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
+    const __nv_bfloat16 *__restrict__ w, int64_t B, int64_t S_q, int64_t q_pos0, int64_t P, int ratio,
+    int topk, int n_split, int32_t *__restrict__ idx, float *__restrict__ scores_opt,
+    unsigned long long *__restrict__ partial) {
+    using C = Cfg<QB>;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t base = smem_u32(smem);
+    unsigned long long *cand_all = reinterpret_cast<unsigned long long *>(smem + C::kOffCand);
+    unsigned *hist_all = reinterpret_cast<unsigned *>(smem + C::kOffHist);
+    float *w_s = reinterpret_cast<float *>(smem + C::kOffW);
+    Misc &ms = *reinterpret_cast<Misc *>(smem + C::kOffMisc);
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t qb_per_seq = (S_q + QB - 1) / QB;
+    const int64_t n_qb = B * qb_per_seq;
+    const int64_t blk = (int64_t)blockIdx.x / n_split;
+    const int split = (int)(blockIdx.x % n_split);
+    const int64_t qb = n_qb - 1 - blk;               // longest query blocks first
+    const int64_t b = qb / qb_per_seq;
+    const int64_t i0 = (qb % qb_per_seq) * QB;
+    const int nq_valid = (int)((S_q - i0) < QB ? (S_q - i0) : QB);
+    const int64_t t_last = q_pos0 + i0 + nq_valid - 1;
+    const int64_t nv_max = n_visible(t_last, ratio, P);
+    const int tiles_all = (int)((nv_max + kTileE - 1) / kTileE);
+    const int t0 = (int)((int64_t)tiles_all * split / n_split);
+    const int t1 = (int)((int64_t)tiles_all * (split + 1) / n_split);
+    const int n_tiles = t1 - t0;
+
+    if (tid == 0) {
+        for (int s = 0; s < C::NST; ++s) {
+            mbar_init(&ms.full[s], 1);
+            mbar_init(&ms.empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&ms.tfull[a], 1);
+            mbar_init(&ms.tempty[a], C::NE);
+        }
+        mbar_init(&ms.bfull, 1);
+        fence_mbar_init();
+        for (int q = 0; q < 4; ++q) {
+            ms.cnt[q] = 0;
+            ms.thr[q] = 0ull;
+        }
+        ms.abort_ = 0;
+    }
+    for (int e = tid; e < QB * 64; e += blockDim.x) {
+        const int q = e >> 6, h = e & 63;
+        w_s[e] = q < nq_valid ? __bfloat162float(w[((b * S_q) + i0 + q) * kHI + h]) : 0.f;
+    }
+    if (warp == 1) tmem_alloc(&ms.tmem_base, C::kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ms.tmem_base;
+    const uint32_t sB = base + C::kOffB, sA = base + C::kOffA;
+
+    if (warp == 0) {
+        // ---------------- producer
+        if (lane == 0 && n_tiles > 0) {
+            mbar_expect_tx(&ms.bfull, C::kBBytes);
+            const int yq = (int)((b * S_q + i0) * kHI);
+            tma_load_2d(sB, &map_q, 0, yq, &ms.bfull);
+            tma_load_2d(sB + C::kBChunk, &map_q, 64, yq, &ms.bfull);
+            for (int it = 0; it < n_tiles; ++it) {
+                const int s = it % C::NST;
+                if (it >= C::NST && !mbar_wait(&ms.empty[s], (uint32_t)((it / C::NST) - 1) & 1u)) {
+                    atomicOr(&g_index_tc_status, 1u);
+                    break;
+                }
+                mbar_expect_tx(&ms.full[s], C::kABytes);
+                const int ye = (int)(b * P + (int64_t)(t0 + it) * kTileE);
+                const uint32_t dst = sA + (uint32_t)s * C::kABytes;
+                tma_load_2d(dst, &map_k, 0, ye, &ms.full[s]);
+                tma_load_2d(dst + 16384u, &map_k, 64, ye, &ms.full[s]);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer
+        if (lane == 0 && n_tiles > 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(128, C::N, 0, 0);
+            bool ok = mbar_wait(&ms.bfull, 0);
+            for (int it = 0; ok && it < n_tiles; ++it) {
+                const int s = it % C::NST, acc = it & 1;
+                ok = mbar_wait(&ms.full[s], (uint32_t)(it / C::NST) & 1u);
+                if (ok && it >= 2) ok = mbar_wait(&ms.tempty[acc], (uint32_t)((it >> 1) - 1) & 1u);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t a0 = sA + (uint32_t)s * C::kABytes;
+#pragma unroll
+                for (int ks = 0; ks < kDI / 16; ++ks) {
+                    const uint64_t ad = sdesc_sw128(a0 + (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(sB + (uint32_t)(ks >> 2) * C::kBChunk + (uint32_t)(ks & 3) * 32u, 16, 1024);
+                    mma_bf16(tmem + (uint32_t)(acc * C::N), ad, bd, idesc, ks > 0 ? 1u : 0u);
+                }
+                mma_commit(&ms.empty[s]);
+                mma_commit(&ms.tfull[acc]);
+            }
+            if (!ok) atomicOr(&g_index_tc_status, 1u);
+        }
+    } else {
+        // ---------------- epilogue: scores, streaming top-k
+        const int e = warp - 2;                      // 0 .. NE-1
+        const int g4 = warp & 3;                     // TMEM lane group of this warp
+        const int row = g4 * 32 + lane;              // entry row inside the tile
+        const int qa = QB == 4 ? 2 * (e >> 2) : 0;   // first query of this thread
+        const int et = e * 32 + lane;                // epilogue thread id
+        const int grp = et / C::GS, gt = et % C::GS;
+        int64_t nvq[QB];
+#pragma unroll
+        for (int q = 0; q < QB; ++q) nvq[q] = q < nq_valid ? n_visible(q_pos0 + i0 + q, ratio, P) : 0;
+        bool ok = true;
+        for (int it = 0; it < n_tiles; ++it) {
+            const int acc = it & 1;
+            if (!mbar_wait(&ms.tfull[acc], (uint32_t)(it >> 1) & 1u)) {
+                atomicOr(&g_index_tc_status, 1u);
+                ok = false;
+            }
+            tc_fence_after();
+            const int64_t j = (int64_t)(t0 + it) * kTileE + row;
+            float sc[C::QPT];
+            const uint32_t trow = tmem + ((uint32_t)(g4 * 32) << 16) + (uint32_t)(acc * C::N);
+#pragma unroll
+            for (int qq = 0; qq < C::QPT; ++qq) {
+                const int q = qa + qq;
+                float v[32];
+                float s = 0.f;
+#pragma unroll
+                for (int hc = 0; hc < 2; ++hc) {
+                    tmem_ld32(trow + (uint32_t)(q * 64 + hc * 32), v);
+                    tmem_ld_wait();
+                    const float4 *wq = reinterpret_cast<const float4 *>(w_s + q * 64 + hc * 32);
+#pragma unroll
+                    for (int h4 = 0; h4 < 8; ++h4) {
+                        const float4 ww = wq[h4];
+                        s = fmaf(ww.x, fmaxf(v[4 * h4 + 0], 0.f), s);
+                        s = fmaf(ww.y, fmaxf(v[4 * h4 + 1], 0.f), s);
+                        s = fmaf(ww.z, fmaxf(v[4 * h4 + 2], 0.f), s);
+                        s = fmaf(ww.w, fmaxf(v[4 * h4 + 3], 0.f), s);
+                    }
+                }
+                sc[qq] = s;
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ms.tempty[acc]);
+#pragma unroll
+            for (int qq = 0; qq < C::QPT; ++qq) {
+                const int q = qa + qq;
+                if (j < nvq[q]) {
+                    const unsigned long long c = ((unsigned long long)order_key(sc[qq]) << 32) |
+                                                 (unsigned long long)(0xFFFFFFFFu - (uint32_t)j);
+                    if (c > ms.thr[q]) {
+                        const unsigned pos = atomicAdd(&ms.cnt[q], 1u);
+                        cand_all[q * kCap + pos] = c;
+                    }
+                }
+            }
+            named_sync(1, C::NE * 32);
+            // cut any buffer that another tile could overflow
+#pragma unroll
+            for (int q = 0; q < QB; ++q) {
+                if (ms.cnt[q] > (unsigned)(kCap - kTileE) && grp == q)
+                    group_cut<C::GS>(cand_all + q * kCap, topk, gt, 2 + q, hist_all + q * 256, ms, q, q);
+            }
+            named_sync(1, C::NE * 32);
+            if (!ok) break;
+        }
+        // final: this group's query
+        if (grp < nq_valid) {
+            const int q = grp;
+            unsigned long long *cand = cand_all + q * kCap;
+            group_cut<C::GS>(cand, topk, gt, 2 + q, hist_all + q * 256, ms, q, q);
+            const int n = (int)ms.cnt[q];
+            const int64_t qrow = b * S_q + i0 + q;
+            if (n_split == 1) {
+                group_emit<C::GS>(cand, n, topk, gt, 2 + q, idx + qrow * topk,
+                                  scores_opt ? scores_opt + qrow * topk : nullptr);
+            } else {
+                unsigned long long *dst = partial + (qrow * n_split + split) * (int64_t)topk;
+                for (int r = gt; r < topk; r += C::GS) dst[r] = r < n ? cand[r] : 0ull;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
+}
+
+// Merge the per-range candidates of one query row (decode split).
+constexpr int kMergeThreads = 256;
+__global__ void __launch_bounds__(kMergeThreads) index_merge_kernel(
+    const unsigned long long *__restrict__ partial, int n_split, int topk, int32_t *__restrict__ idx,
+    float *__restrict__ scores_opt) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int total = n_split * topk;
+    const int cap = pow2_ceil(total);
+    unsigned long long *cand = reinterpret_cast<unsigned long long *>(smem_raw);
+    unsigned long long *keep = cand + cap;                   // pow2_ceil(topk) slots
+    unsigned *hist = reinterpret_cast<unsigned *>(keep + pow2_ceil(topk));
+    Misc &ms = *reinterpret_cast<Misc *>(hist + 256);
+    const int64_t row = blockIdx.x;
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        ms.cnt[0] = 0;
+        ms.cnt[1] = 0;
+    }
+    __syncthreads();
+    for (int e = tid; e < total; e += kMergeThreads) {
+        const unsigned long long c = partial[row * total + e];
+        if (c != 0ull) cand[atomicAdd(&ms.cnt[0], 1u)] = c;
+    }
+    __syncthreads();
+    int n = (int)ms.cnt[0];
+    unsigned long long *src = cand;
+    if (n > topk) {
+        const unsigned long long T = group_kth<kMergeThreads>(cand, n, topk, tid, 1, hist, ms, 0);
+        for (int e = tid; e < n; e += kMergeThreads) {
+            const unsigned long long c = cand[e];
+            if (c >= T) keep[atomicAdd(&ms.cnt[1], 1u)] = c;
+        }
+        __syncthreads();
+        n = (int)ms.cnt[1];
+        src = keep;
+    }
+    group_emit<kMergeThreads>(src, n, topk, tid, 1, idx + row * topk,
+                              scores_opt ? scores_opt + row * topk : nullptr);
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint32_t box_rows) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)kDI, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)kDI * 2};
+    cuuint32_t box[2] = {64u, box_rows};
+    cuuint32_t es[2] = {1u, 1u};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int sm_count() {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms;
+}
+
+struct Plan {
+    int qb;
+    int n_split;
+};
+
+Plan plan(int64_t B, int64_t S_q, int64_t q_pos0, int64_t P, int ratio, int topk) {
+    Plan p;
+    p.qb = S_q >= 4 ? 4 : 1;
+    const int64_t n_qb = B * ((S_q + p.qb - 1) / p.qb);
+    const int64_t tiles = (n_visible(q_pos0 + S_q - 1, ratio, P) + kTileE - 1) / kTileE;
+    const int64_t want = 2 * (int64_t)sm_count();
+    int64_t ns = 1;
+    if (n_qb < want && tiles >= 8) ns = (want + n_qb - 1) / n_qb;
+    if (ns > tiles / 4) ns = tiles / 4 > 0 ? tiles / 4 : 1;
+    if (ns > 16) ns = 16;
+    while (ns > 1 && (int64_t)pow2_ceil((int)(ns * topk)) > 8192) --ns;
+    p.n_split = (int)(ns < 1 ? 1 : ns);
+    return p;
+}
+
+template <int QB>
+csa_status_t launch(const CUtensorMap &mk, const CUtensorMap &mq, const __nv_bfloat16 *w, int64_t B,
+                    int64_t S_q, int64_t q_pos0, int64_t P, int ratio, int topk, int n_split, int32_t *idx,
+                    float *scores_opt, unsigned long long *partial, cudaStream_t st) {
+    using C = Cfg<QB>;
+    const int64_t n_qb = B * ((S_q + QB - 1) / QB);
+    const int64_t grid = n_qb * n_split;
+    CSA_REQUIRE(grid < (1ll << 31), CSA_ERR_UNSUPPORTED, "csa_index_topk: grid too large");
+    auto kern = index_tc_kernel<QB>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
+    kern<<<(unsigned)grid, C::kThreads, C::kSmem, st>>>(mk, mq, w, B, S_q, q_pos0, P, ratio, topk, n_split,
+                                                        idx, scores_opt, partial);
+    CSA_CHECK_LAUNCH("csa_index_topk");
+    return CSA_OK;
+}
+
+}  // namespace
+
+bool index_tc_eligible(int64_t B, int64_t S_q, int64_t P, int H_I, int d_I, int topk,
+                       csa_dtype_t dtype) {
+    // TMA row coordinates are 32-bit: B*P rows of k_I and B*S_q*H_I rows of q_I
+    return dtype == CSA_BF16 && H_I == kHI && d_I == kDI && topk <= kMaxTopk && P > 0 &&
+           B * P + kTileE < (1ll << 31) && B * S_q * kHI + 256 < (1ll << 31);
+}
+
+size_t index_tc_workspace(int64_t B, int64_t S_q, int64_t q_pos0, int64_t P, int ratio, int topk) {
+    Plan p = plan(B, S_q, q_pos0, P, ratio, topk);
+    if (p.n_split <= 1) return 0;
+    return (size_t)B * S_q * p.n_split * topk * sizeof(unsigned long long);
+}
+
+csa_status_t index_tc(const void *qI, const void *w, const void *kI, int64_t B, int64_t S_q, int64_t q_pos0,
+                      int64_t P, int ratio, int topk, int32_t *idx, float *scores_opt, void *workspace,
+                      size_t workspace_bytes, cudaStream_t st) {
+    CUtensorMap mk, mq;
+    CSA_REQUIRE(make_map(&mk, kI, (uint64_t)B * P, kTileE), CSA_ERR_CUDA,
+                "csa_index_topk: cannot encode the k_I tensor map");
+    Plan p = plan(B, S_q, q_pos0, P, ratio, topk);
+    CSA_REQUIRE(make_map(&mq, qI, (uint64_t)B * S_q * kHI, (uint32_t)(p.qb * 64)), CSA_ERR_CUDA,
+                "csa_index_topk: cannot encode the q_I tensor map");
+    unsigned long long *partial = nullptr;
+    if (p.n_split > 1) {
+        const size_t need = (size_t)B * S_q * p.n_split * topk * sizeof(unsigned long long);
+        CSA_REQUIRE(workspace && workspace_bytes >= need, CSA_ERR_WORKSPACE,
+                    "csa_index_topk: workspace of %zu B given, %zu B needed", workspace_bytes, need);
+        partial = reinterpret_cast<unsigned long long *>(workspace);
+    }
+    csa_status_t r;
+    const __nv_bfloat16 *wb = reinterpret_cast<const __nv_bfloat16 *>(w);
+    if (p.qb == 4)
+        r = launch<4>(mk, mq, wb, B, S_q, q_pos0, P, ratio, topk, p.n_split, idx, scores_opt, partial, st);
+    else
+        r = launch<1>(mk, mq, wb, B, S_q, q_pos0, P, ratio, topk, p.n_split, idx, scores_opt, partial, st);
+    if (r != CSA_OK || p.n_split <= 1) return r;
+    const int total = p.n_split * topk;
+    const size_t smem = (size_t)(pow2_ceil(total) + pow2_ceil(topk)) * 8 + 256 * 4 + sizeof(Misc);
+    CSA_REQUIRE(smem <= 227 * 1024, CSA_ERR_UNSUPPORTED, "csa_index_topk: merge too large");
+    cudaFuncSetAttribute(index_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    index_merge_kernel<<<(unsigned)(B * S_q), kMergeThreads, smem, st>>>(partial, p.n_split, topk, idx, scores_opt);
+    CSA_CHECK_LAUNCH("csa_index_topk merge");
+    return CSA_OK;
+}
+
+unsigned int read_index_tc_status() {
+    unsigned int v = 0, z = 0;
+    cudaMemcpyFromSymbol(&v, g_index_tc_status, sizeof(v));
+    cudaMemcpyToSymbol(g_index_tc_status, &z, sizeof(z));
+    return v;
+}
+
+}  // namespace csa

@@ -121,9 +121,10 @@ csa_status_t index_topk_general(const void *qI, const void *w, const void *kI, i
 
 }  // namespace csa
 
-extern "C" size_t csa_index_topk_workspace_bytes(int64_t B, int64_t S_q, int64_t P, int32_t H_I,
-                                                 int32_t d_I, int32_t topk, csa_dtype_t dtype) {
-    return csa::index_topk_workspace(B, S_q, P, H_I, d_I, topk, dtype);
+extern "C" size_t csa_index_topk_workspace_bytes(int64_t B, int64_t S_q, int64_t q_pos0,
+                                                 int64_t P, int32_t H_I, int32_t d_I,
+                                                 int32_t ratio, int32_t topk, csa_dtype_t dtype) {
+    return csa::index_topk_workspace(B, S_q, q_pos0, P, H_I, d_I, ratio, topk, dtype);
 }
 
 extern "C" csa_status_t csa_index_topk(const void *q_I, const void *w, const void *k_I,
@@ -147,7 +148,7 @@ extern "C" csa_status_t csa_index_topk(const void *q_I, const void *w, const voi
     CSA_REQUIRE(aligned(q_I, 16) && aligned(k_I, 16) && aligned(w, (dtype == CSA_F32) ? 4 : 2) &&
                     aligned(idx, 4) && aligned(scores_opt, 4),
                 CSA_ERR_INVALID_ARG, "csa_index_topk: misaligned pointer");
-    size_t need = index_topk_workspace(B, S_q, P, H_I, d_I, topk, dtype);
+    size_t need = index_topk_workspace(B, S_q, q_pos0, P, H_I, d_I, ratio, topk, dtype);
     CSA_REQUIRE(workspace_bytes >= need && (need == 0 || workspace), CSA_ERR_WORKSPACE,
                 "csa_index_topk: workspace of %zu B given, %zu B needed", workspace_bytes, need);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

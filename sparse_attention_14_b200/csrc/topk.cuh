@@ -2,14 +2,14 @@
 //
 // Selection rule (HF docs model_doc/deepseek_v4, "Attention mask layout": the indexer
 // keeps index_topk entries per query and marks unused slots -1): the kk = min(k, n)
-// largest scores, ties broken by the lower entry index, output sorted by (score
-// descending, index ascending), then -1 padding.
+// largest scores, ties broken by the lower entry index, output in ascending entry
+// order, then -1 padding.
 //
 // Method: fp32 scores map to order-preserving uint32 keys; an 8-bit MSB-first radix
 // select (four histogram passes over the candidates that still match the prefix)
 // finds the kk-th largest key exactly; the keys above it are taken in any order and
 // the ties at it are taken in index order by a block-wide ordered scan; the kk winners
-// are then bitonic-sorted as 64-bit (key, ~index) words.  No global memory is used.
+// are then bitonic-sorted by entry index.  No global memory is used.
 #pragma once
 
 #include "common.cuh"
@@ -36,7 +36,7 @@ __host__ __device__ constexpr int pow2_ceil(int x) {
 // scores[0..n): candidate scores (entry index = position).  sel: scratch of
 // pow2_ceil(max(kk,1)) uint64 words.  Writes idx_out[0..k) and, if score_out != NULL,
 // score_out[0..k).  All threads of the block must call it.
-__device__ void block_topk(const float *scores, int n, int k, TopkSmem *ts,
+static __device__ void block_topk(const float *scores, int n, int k, TopkSmem *ts,
                            unsigned long long *sel, int32_t *idx_out, float *score_out) {
     const int tid = threadIdx.x, nt = blockDim.x;
     const int kk = n < k ? n : k;
@@ -114,7 +114,8 @@ __device__ void block_topk(const float *scores, int n, int k, TopkSmem *ts,
         for (int i = tid; i < n; i += nt)
             sel[i] = ((unsigned long long)order_key(scores[i]) << 32) | (0xFFFFFFFFu - (uint32_t)i);
     }
-    // bitonic sort, descending, over N = pow2_ceil(kk) words (padding sorts last)
+    // bitonic sort by entry index ascending (the low word ~index descending) over
+    // N = pow2_ceil(kk) words; the zero padding sorts last
     const int N = pow2_ceil(kk);
     for (int i = kk + tid; i < N; i += nt) sel[i] = 0ull;
     __syncthreads();
@@ -125,7 +126,7 @@ __device__ void block_topk(const float *scores, int n, int k, TopkSmem *ts,
                 int hi = lo + stride;
                 bool desc = ((lo & size) == 0);
                 unsigned long long a = sel[lo], b = sel[hi];
-                if ((a < b) == desc) { sel[lo] = b; sel[hi] = a; }
+                if (((uint32_t)a < (uint32_t)b) == desc) { sel[lo] = b; sel[hi] = a; }
             }
             __syncthreads();
         }

@@ -41,6 +41,11 @@ MID = [
     LayerSpec(name="mid_csa_ragged_bf16", dtype="bf16", B=1, S_q=700, S_kv=700, q_pos0=0,
               kv_pos0=0, H=64, D=512, R=64, base=160000.0, W=100, m=4, P=175, kind="csa",
               H_I=64, d_I=128, topk=37, workload=98),
+    # indexer buffer cuts (more than 1024 visible entries) and a top-k that is not a
+    # power of two
+    LayerSpec(name="mid_csa_cut_bf16", dtype="bf16", B=1, S_q=4801, S_kv=4801, q_pos0=0,
+              kv_pos0=0, H=64, D=512, R=64, base=160000.0, W=128, m=4, P=1200, kind="csa",
+              H_I=64, d_I=128, topk=200, workload=89),
     # odd shapes: general path
     LayerSpec(name="odd_csa_bf16", dtype="bf16", B=1, S_q=77, S_kv=77, q_pos0=0, kv_pos0=0, H=5,
               D=40, R=8, base=10000.0, W=9, m=3, P=25, kind="csa", H_I=3, d_I=24, topk=7,
@@ -90,10 +95,13 @@ def test_index_topk_parity(spec):
     g_sc = scores.cpu().numpy().astype(np.float64)
     for b in range(spec.B):
         check_topk(g_idx[b], o_idx[b], sc[b], kk_rows(spec, rows))
-        # scores of the kept entries, where the sets agree slot by slot
-        same = (g_idx[b] == o_idx[b]) & (o_idx[b] >= 0)
-        if same.any():
-            assert rel_err(g_sc[b][same], o_sel[b][same]) <= TOL[spec.dtype] * 0.05
+        # the kept entries come in ascending entry order, and each carries its own score
+        for r in range(len(rows)):
+            kk = kk_rows(spec, rows)[r]
+            assert (np.diff(g_idx[b, r, :kk]) > 0).all(), "row %d not in ascending order" % r
+        valid = g_idx[b] >= 0
+        ref = np.where(valid, np.take_along_axis(sc[b], np.maximum(g_idx[b], 0), axis=1), 0.0)
+        assert rel_err(np.where(valid, g_sc[b], 0.0), ref) <= TOL[spec.dtype] * 0.05
 
 
 @pytest.mark.parametrize("spec", MID, ids=[s.name for s in MID])
@@ -126,6 +134,24 @@ def test_tensor_core_path_selected():
         tc = spec.dtype == "bf16" and spec.H == 64 and spec.D == 512 and \
             spec.S_q * 64 >= spec.S_kv + spec.P
         assert (ws > 0) == tc, spec.name
+
+
+@pytest.mark.parametrize("S_q,q_pos0,P,topk", [(1203, 0, 1100, 300), (1, 8191, 2048, 512),
+                                               (3, 5000, 1500, 896)])
+def test_index_all_ties_take_lowest_entries(S_q, q_pos0, P, topk):
+    """q_I = 0 makes every score exactly 0: the kept entries must be the lowest visible
+    indices (equal scores rank the lower index first), in ascending order; exact."""
+    import sparse_attention_14_b200 as csa
+    B, m = 2, 4
+    q_I = torch.zeros((B, S_q, 64, 128), dtype=torch.bfloat16, device=DEV)
+    w = torch.randn((B, S_q, 64), device=DEV).to(torch.bfloat16)
+    k_I = torch.randn((B, P, 128), device=DEV).to(torch.bfloat16)
+    idx = csa.csa_index_topk(q_I, w, k_I, q_pos0, m, topk).cpu().numpy()
+    for i in range(S_q):
+        nv = min(P, (q_pos0 + i + 1) // m)
+        kk = min(topk, nv)
+        want = list(range(kk)) + [-1] * (topk - kk)
+        assert idx[0, i].tolist() == want and idx[1, i].tolist() == want, i
 
 
 def test_no_kernel_gave_up():
