@@ -6,22 +6,29 @@
 // mask layout" for the key sets).
 //
 // Design (one persistent CTA per SM, one query at a time, 64 heads per query):
-//  * keys are rotated once per call into the workspace (rope_rows_kernel), so a key
-//    tile is a plain gather of 128 rows of 1 KB (window rows are contiguous, selected
-//    entries are gathered by index) with 16-byte async copies into 128B-swizzled smem;
-//  * the MMAs are transposed so that M = 128 keys / 128 head-dims (full-rate M=128
-//    tcgen05 tiles) and N = 64 heads:
+//  * keys are rotated once per call into the workspace (rope_rows_kernel); a key tile is
+//    128 rows of 1 KB in 128B-swizzled shared memory, split into eight 16 KB chunks
+//    (64 dims each) with their own mbarriers: window rows (contiguous) arrive by 2-D TMA
+//    boxes, selected entries by 16-byte async copies from the loader warp;
+//  * warp roles: warp 0 loads (idx compaction, Q by TMA with its rope channels rotated in
+//    place, key tiles), warp 1 issues the MMAs (one thread), warps 2-9 run the softmax
+//    and the epilogue (two warps per TMEM lane group, 32 heads each);
+//  * the MMAs are transposed so that M = 128 keys / 128 head-dims (M=128 tcgen05 tiles)
+//    and N = 64 heads:
 //      S^T[key, h]  = K[key, :] . Qr[h, :]          (A = key tile, K-major; B = Q, K-major)
 //      O^T[d, h]   += V^T[d, key] . P^T[key, h]     (A = same key tile read MN-major,
 //                                                    B = P stored key-major, MN-major)
-//    both accumulate in TMEM (O^T: 4 x 64 columns, S^T: 64 columns);
-//  * softmax: one thread per key row holds its 64 head scores; the running max per head
-//    is only refreshed (exact cross-lane max, rescale of O^T and of the partial sums)
-//    when some score exceeds it by more than 2^8, so the common tile needs no
-//    cross-thread reduction; row sums stay per thread and are reduced once per query;
-//    the sink enters as the initial running max and once in the final sum;
-//  * epilogue: O^T / l, the -t de-rotation of the rope channels (partner channel via a
-//    lane shuffle), transposed through shared memory into coalesced 16-byte stores.
+//    both accumulate in TMEM (O^T: 4 x 64 columns, S^T: 64 columns); the first MMAs of a
+//    tile start as soon as its first chunk lands, and each pair of chunks is released to
+//    the loader as soon as the P.V MMAs reading it complete;
+//  * softmax: one thread per key row holds 32 head scores; the running max per head is
+//    only refreshed (exact cross-lane max, rescale of O^T and of the partial sums) when
+//    some score exceeds it by more than 2^8, so the common tile needs no cross-thread
+//    reduction; row sums stay per thread and are reduced once per query; the sink enters
+//    as the initial running max and once in the final sum;
+//  * epilogue: O^T / l and the -t de-rotation of the rope channels (partner channel via a
+//    lane shuffle), stored as bf16 pairs straight from registers while the next query's
+//    first tile loads and multiplies.
 #include <mutex>
 
 #include "attend.cuh"
@@ -35,24 +42,32 @@ namespace {
 
 using namespace umma;
 
-constexpr int kD = 512, kH = 64, kTile = 128, kThreads = 256;
-constexpr uint32_t kKvBytes = kTile * kD * 2;   // 8 chunks x 16 KB
-constexpr uint32_t kQBytes = kH * kD * 2;       // 8 chunks x 8 KB
-constexpr uint32_t kPBytes = kTile * kH * 2;    // 1 chunk of 128 rows
+constexpr int kD = 512, kH = 64, kTile = 128;
+constexpr int kThreads = 320;                    // warp 0 loads, warp 1 MMA, warps 2-9 softmax
+constexpr int kSoftThreads = 256;                // two warps per TMEM lane group, 32 heads each
+constexpr uint32_t kKvBytes = kTile * kD * 2;    // 8 chunks x 16 KB
+constexpr uint32_t kQBytes = kH * kD * 2;        // 8 chunks x 8 KB
+constexpr uint32_t kPBytes = kTile * kH * 2;     // 1 chunk of 128 rows
 constexpr uint32_t kOffKv = 0, kOffQ = kKvBytes, kOffP = kOffQ + kQBytes, kOffEnt = kOffP + kPBytes;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kRescaleThreshold = 8.0f;       // log2 units
+constexpr float kRescaleThreshold = 8.0f;        // log2 units
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 64, 0, 0);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 64, 1, 1);
 constexpr uint32_t kColO = 0, kColS = 256;
+constexpr uint32_t kWaitIter = 1u << 25;         // bounded waits (~seconds)
+
+struct Meta {
+    int n_ent;
+};
 
 struct Small {
-    uint64_t bar_mma;
+    uint64_t full[8], free_[4], s_full, p_full, o_full, q_tma, q_full, q_free, meta_full[2];
     uint32_t tmem_base;
     int flag;
-    int n_ent;
     int abort_;
-    int64_t row_off[kTile];
+    Meta meta[2];
+    int32_t rows[kTile];
+    float qcs[2][32];
     float m_used[kH];
     float alpha[kH];
     float red[4][kH];
@@ -93,13 +108,13 @@ __global__ void rope_rows_kernel(const __nv_bfloat16 *__restrict__ src, __nv_bfl
     store8(dst + ((int64_t)b * rows + r) * D + pc * 8, x);
 }
 
-// warp butterfly over 64 per-lane values: afterwards lane L holds the reduction over the
-// warp of heads 2L and 2L+1 in v[0], v[1].
+// warp butterfly over 32 per-lane values: afterwards lane L holds in v[0] the reduction
+// over the warp of value L.
 template <bool kMax>
-__device__ __forceinline__ void warp_reduce64(float *v) {
+__device__ __forceinline__ void warp_reduce32(float *v) {
     const int lane = threadIdx.x & 31;
 #pragma unroll
-    for (int half = 32, off = 16; off >= 1; half >>= 1, off >>= 1) {
+    for (int half = 16, off = 16; off >= 1; half >>= 1, off >>= 1) {
         const bool upper = (lane & off) != 0;
 #pragma unroll
         for (int i = 0; i < half; ++i) {
@@ -111,9 +126,37 @@ __device__ __forceinline__ void warp_reduce64(float *v) {
     }
 }
 
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        :
+        : "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+struct QueryGeom {
+    int64_t b, i, t, lo_w;
+    int n_win, n_wt;
+};
+
+__device__ __forceinline__ QueryGeom query_geom(int64_t qi, int64_t S_q, int64_t q_pos0, int64_t kv_pos0,
+                                                int64_t S_kv, int window) {
+    QueryGeom g;
+    g.b = qi / S_q;
+    g.i = qi % S_q;
+    g.t = q_pos0 + g.i;
+    int64_t lo = g.t - window + 1;
+    if (lo < kv_pos0) lo = kv_pos0;
+    int64_t hi = g.t < kv_pos0 + S_kv - 1 ? g.t : kv_pos0 + S_kv - 1;
+    g.lo_w = lo;
+    g.n_win = hi >= lo ? (int)(hi - lo + 1) : 0;
+    g.n_wt = (g.n_win + kTile - 1) / kTile;
+    return g;
+}
+
 __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
-    const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ kv_rot, int64_t S_kv,
-    int64_t kv_pos0, const __nv_bfloat16 *__restrict__ pool_rot, int64_t P,
+    const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kv,
+    const __nv_bfloat16 *__restrict__ pool_rot, int64_t S_kv, int64_t kv_pos0, int64_t P,
     const int32_t *__restrict__ idx, int topk, int mode, const float *__restrict__ sink,
     __nv_bfloat16 *__restrict__ out, int64_t B, int64_t S_q, int64_t q_pos0, int window, int ratio,
     float scale, RopeTable rope) {
@@ -123,304 +166,433 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     const uint32_t base = smem_u32(smem);
     const uint32_t s_kv = base + kOffKv, s_q = base + kOffQ, s_p = base + kOffP;
     int32_t *ent = reinterpret_cast<int32_t *>(smem + kOffEnt);
-    size_t ent_bytes = ((size_t)(topk > 0 ? topk : 1) * 4 + 15) & ~(size_t)15;
+    const size_t ent_bytes = ((size_t)(topk > 0 ? topk : 1) * 4 + 15) & ~(size_t)15;
     Small &sm = *reinterpret_cast<Small *>(smem + kOffEnt + ent_bytes);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const float c2 = scale * kLog2e;
+    const int64_t nq = B * S_q;
 
     if (tid == 0) {
-        mbar_init(&sm.bar_mma, 1);
+        for (int c = 0; c < 8; ++c) mbar_init(&sm.full[c], 1);
+        for (int c = 0; c < 4; ++c) mbar_init(&sm.free_[c], 1);
+        mbar_init(&sm.s_full, 1);
+        mbar_init(&sm.p_full, kSoftThreads);
+        mbar_init(&sm.o_full, 1);
+        mbar_init(&sm.q_tma, 1);
+        mbar_init(&sm.q_full, 1);
+        mbar_init(&sm.q_free, 1);
+        mbar_init(&sm.meta_full[0], 1);
+        mbar_init(&sm.meta_full[1], 1);
         fence_mbar_init();
         sm.flag = 0;
         sm.abort_ = 0;
     }
-    if (warp == 0) tmem_alloc(&sm.tmem_base, 512);
+    if (warp == 1) tmem_alloc(&sm.tmem_base, 512);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    uint32_t phase = 0;
 
-    for (int64_t qi = blockIdx.x; qi < B * S_q; qi += gridDim.x) {
-        const int64_t b = qi / S_q, i = qi % S_q;
-        const int64_t t = q_pos0 + i;
-        const int64_t nv = n_visible(t, ratio, P);
-        int64_t lo_w = t - window + 1;
-        if (lo_w < kv_pos0) lo_w = kv_pos0;
-        int64_t hi_w = t < kv_pos0 + S_kv - 1 ? t : kv_pos0 + S_kv - 1;
-        const int n_win = hi_w >= lo_w ? (int)(hi_w - lo_w + 1) : 0;
-
-        // entries of this query
-        if (mode == 0) {
-            if (warp == 0) {
+    if (warp == 0) {
+        // ===================================================== loader
+        uint32_t g = 0, qc = 0;
+        for (int64_t qi = blockIdx.x; qi < nq && !sm.abort_; qi += gridDim.x, ++qc) {
+            const QueryGeom qg = query_geom(qi, S_q, q_pos0, kv_pos0, S_kv, window);
+            const int64_t nv = n_visible(qg.t, ratio, P);
+            int n_ent;
+            if (mode == 0) {
+                // compact the valid idx values in slot order; eight loads per lane in flight
                 int cnt = 0;
                 const int32_t *ip = idx + qi * topk;
-                for (int c0 = 0; c0 < topk; c0 += 32) {
-                    int c = c0 + lane;
-                    int32_t j = c < topk ? ip[c] : -1;
-                    bool ok = j >= 0 && (int64_t)j < nv;
-                    unsigned ball = __ballot_sync(0xFFFFFFFFu, ok);
-                    if (ok) ent[cnt + __popc(ball & ((1u << lane) - 1u))] = j;
-                    cnt += __popc(ball);
-                }
-                if (lane == 0) sm.n_ent = cnt;
-            }
-        } else if (tid == 0) {
-            sm.n_ent = (int)nv;
-        }
-        // rotated Q into the swizzled B operand
-        const __nv_bfloat16 *qrow = q + qi * (int64_t)kH * kD;
-        for (int v = tid; v < kH * (kD / 8); v += kThreads) {
-            const int h = v >> 6, qp = v & 63;
-            float x[8];
-            load8(qrow + (int64_t)h * kD + qp * 8, x);
-            const int d0 = qp * 8;
-            if (d0 + 8 > rope.first) {
+                for (int c0 = 0; c0 < topk; c0 += 256) {
+                    int32_t jv[8];
 #pragma unroll
-                for (int c = 0; c < 8; c += 2) {
-                    int d = d0 + c;
-                    if (d >= rope.first) {
-                        float cs, sn;
-                        rope_cs((double)t, rope.inv_freq[(d - rope.first) >> 1], &cs, &sn);
-                        float a = x[c], bb = x[c + 1];
-                        x[c] = a * cs - bb * sn;
-                        x[c + 1] = a * sn + bb * cs;
+                    for (int k = 0; k < 8; ++k) {
+                        const int c = c0 + k * 32 + lane;
+                        jv[k] = c < topk ? ip[c] : -1;
+                    }
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const bool okj = jv[k] >= 0 && (int64_t)jv[k] < nv;
+                        const unsigned ball = __ballot_sync(0xFFFFFFFFu, okj);
+                        if (okj) ent[cnt + __popc(ball & ((1u << lane) - 1u))] = jv[k];
+                        cnt += __popc(ball);
                     }
                 }
+                n_ent = cnt;
+                // warm L2 with the next query's idx row
+                const int64_t qn = qi + gridDim.x;
+                if (qn < nq) {
+                    const char *np = reinterpret_cast<const char *>(idx + qn * topk);
+                    for (int off = lane * 128; off < topk * 4; off += 32 * 128)
+                        asm volatile("prefetch.global.L2 [%0];" ::"l"(np + off));
+                }
+            } else {
+                n_ent = (int)nv;
             }
-            uint4 u;
-            __nv_bfloat162 *hp = reinterpret_cast<__nv_bfloat162 *>(&u);
+            __syncwarp();
+            if (lane == 0) {
+                sm.meta[qc & 1].n_ent = n_ent;
+                mbar_arrive(&sm.meta_full[qc & 1]);
+            }
+            // Q of this query: start its TMA now, rotate it once the first tile is issued
+            if (qc > 0 && !mbar_wait(&sm.q_free, (qc - 1) & 1u, kWaitIter)) {
+                atomicOr(&g_attend_tc_status, 1u);
+                sm.abort_ = 1;
+                break;
+            }
+            if (lane == 0) {
+                mbar_expect_tx(&sm.q_tma, kQBytes);
+                for (int c = 0; c < 8; ++c)
+                    tma_load_2d(s_q + (uint32_t)c * 8192u, &map_q, 64 * c, (int)(qi * kH), &sm.q_tma);
+                // bring the next query's Q into L2 while this query runs
+                const int64_t qn = qi + gridDim.x;
+                if (qn < nq)
+                    for (int c = 0; c < 8; ++c)
+                        asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
+                                         reinterpret_cast<uint64_t>(&map_q)),
+                                     "r"(64 * c), "r"((int)(qn * kH))
+                                     : "memory");
+            }
+            if (lane < rope.n_pairs) {
+                float cs, sn;
+                rope_cs((double)qg.t, rope.inv_freq[lane], &cs, &sn);
+                sm.qcs[0][lane] = cs;
+                sm.qcs[1][lane] = sn;
+            }
+            const int n_tiles = qg.n_wt + (n_ent + kTile - 1) / kTile;
+            bool q_done = false;
+            bool ok = true;
+            for (int kt = 0; kt <= n_tiles && ok; ++kt) {
+                if (kt == 1 || (kt == n_tiles && !q_done)) {
+                    // rotate the rope channels of Q in place and publish it
+                    ok = mbar_wait(&sm.q_tma, qc & 1u, kWaitIter);
+                    if (!ok) break;
+                    __syncwarp();
+                    for (int v = lane; v < kH * 8; v += 32) {
+                        const int h = v >> 3, pc = v & 7;
+                        const int d0 = 7 * 64 + pc * 8;
+                        if (d0 + 8 <= rope.first) continue;
+                        const uint32_t addr = s_q + 7u * 8192u + sw128((uint32_t)h, (uint32_t)pc);
+                        uint32_t w0, w1, w2, w3;
+                        asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3) : "r"(addr));
+                        uint32_t wv[4] = {w0, w1, w2, w3};
 #pragma unroll
-            for (int k = 0; k < 4; ++k) hp[k] = __floats2bfloat162_rn(x[2 * k], x[2 * k + 1]);
-            const uint32_t dst = s_q + (uint32_t)(qp >> 3) * 8192u + sw128((uint32_t)h, (uint32_t)(qp & 7));
-            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(u.x), "r"(u.y), "r"(u.z),
-                         "r"(u.w)
-                         : "memory");
-        }
-        if (tid < kH) {
-            const float sk = sink[tid];
-            sm.m_used[tid] = sk == -INFINITY ? -INFINITY : sk * kLog2e;
-        }
-        __syncthreads();
-        const int n_keys = n_win + sm.n_ent;
-        const int n_tiles = (n_keys + kTile - 1) / kTile;
-
-        float l_part[kH];
+                        for (int k = 0; k < 4; ++k) {
+                            const int d = d0 + 2 * k;
+                            if (d >= rope.first) {
+                                __nv_bfloat162 hv = *reinterpret_cast<__nv_bfloat162 *>(&wv[k]);
+                                float2 f = __bfloat1622float2(hv);
+                                const int pr = (d - rope.first) >> 1;
+                                const float cs = sm.qcs[0][pr], sn = sm.qcs[1][pr];
+                                __nv_bfloat162 r = __floats2bfloat162_rn(f.x * cs - f.y * sn, f.x * sn + f.y * cs);
+                                wv[k] = *reinterpret_cast<uint32_t *>(&r);
+                            }
+                        }
+                        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(wv[0]), "r"(wv[1]),
+                                     "r"(wv[2]), "r"(wv[3])
+                                     : "memory");
+                    }
+                    fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm.q_full);
+                    q_done = true;
+                }
+                if (kt == n_tiles) break;
+                const bool win = kt < qg.n_wt;
+                if (win) {
+                    // window rows are contiguous: one 2-D TMA box of 128 rows per chunk
+                    const int y0 = (int)(qg.b * S_kv + (qg.lo_w - kv_pos0) + (int64_t)kt * kTile);
+                    for (int c = 0; c < 8 && ok; ++c) {
+                        if ((c & 1) == 0 && g > 0) ok = mbar_wait(&sm.free_[c >> 1], (g - 1) & 1u, kWaitIter);
+                        if (ok && lane == 0) {
+                            mbar_expect_tx(&sm.full[c], 16384u);
+                            tma_load_2d(s_kv + (uint32_t)c * 16384u, &map_kv, 64 * c, y0, &sm.full[c]);
+                        }
+                    }
+                } else {
+                    // selected entries: 16-byte async copies straight into the swizzled
+                    // layout.  Lane l always copies piece (l & 7) of rows 4k + (l >> 3), so its
+                    // 32 source rows and destinations are computed once per tile; up to four
+                    // chunks are in flight, each published (own copies complete, proxy fence,
+                    // warp sync) with one mbarrier arrive.
+                    const int et = kt - qg.n_wt;
+                    const int pc = lane & 7;
+                    const __nv_bfloat16 *src[32];
+                    uint32_t dsto[32];
 #pragma unroll
-        for (int h = 0; h < kH; ++h) l_part[h] = 0.f;
-
-        for (int kt = 0; kt < n_tiles; ++kt) {
-            const int x0 = kt * kTile;
-            const int tile_n = min(kTile, n_keys - x0);
-            if (tid < kTile) {
-                const int kx = x0 + tid;
-                int64_t off = 0;
-                if (tid < tile_n) {
-                    if (kx < n_win) {
-                        off = (b * S_kv + (lo_w - kv_pos0) + kx) * kD;
-                    } else {
-                        int64_t j = mode == 0 ? (int64_t)ent[kx - n_win] : (int64_t)(kx - n_win);
-                        off = -1 - (b * P + j) * kD;
+                    for (int k = 0; k < 32; ++k) {
+                        const int xr = 4 * k + (lane >> 3);
+                        const int r = et * kTile + xr;
+                        const int rr = r < n_ent ? r : 0;
+                        const int64_t j = mode == 0 ? (int64_t)ent[rr] : (int64_t)rr;
+                        src[k] = pool_rot + (qg.b * P + j) * kD + pc * 8;
+                        dsto[k] = sw128((uint32_t)xr, (uint32_t)pc);
+                    }
+                    for (int c = 0; c < 8 && ok; ++c) {
+                        if ((c & 1) == 0 && g > 0) ok = mbar_wait(&sm.free_[c >> 1], (g - 1) & 1u, kWaitIter);
+                        if (!ok) break;
+                        const uint32_t dst = s_kv + (uint32_t)c * 16384u;
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) cp_async16(dst + dsto[k], src[k] + c * 64, 16u);
+                        cp_async_commit();
+                        if (c >= 3) {
+                            asm volatile("cp.async.wait_group 3;" ::: "memory");
+                            fence_async_smem();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&sm.full[c - 3]);
+                        }
+                    }
+                    if (ok) {
+                        asm volatile("cp.async.wait_group 2;" ::: "memory");
+                        fence_async_smem();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sm.full[5]);
+                        asm volatile("cp.async.wait_group 1;" ::: "memory");
+                        fence_async_smem();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sm.full[6]);
+                        asm volatile("cp.async.wait_group 0;" ::: "memory");
+                        fence_async_smem();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sm.full[7]);
                     }
                 }
-                sm.row_off[tid] = off;
+                __syncwarp();
+                ++g;
             }
-            __syncthreads();
-            // gather the key tile (rows past tile_n are zero-filled)
-#pragma unroll 4
-            for (int r = 0; r < (kTile * 64) / kThreads; ++r) {
-                const int v = tid + r * kThreads;
-                const int x = v >> 6, qp = v & 63;
-                const int64_t off = sm.row_off[x];
-                const __nv_bfloat16 *src = off >= 0 ? kv_rot + off : pool_rot + (-1 - off);
-                const uint32_t bytes = x < tile_n ? 16u : 0u;
-                if (bytes == 0) src = kv_rot;
-                cp_async16(s_kv + (uint32_t)(qp >> 3) * 16384u + sw128((uint32_t)x, (uint32_t)(qp & 7)),
-                           src + qp * 8, bytes);
+            if (!ok) {
+                atomicOr(&g_attend_tc_status, 1u);
+                sm.abort_ = 1;
+                break;
             }
-            cp_async_commit();
-            cp_async_wait_all();
-            fence_async_smem();
-            __syncthreads();
-
-            // S^T = K . Qr^T
-            if (tid == 0) {
+        }
+    } else if (warp == 1) {
+        // ===================================================== MMA issuer
+        if (lane == 0) {
+            uint32_t g = 0, qc = 0;
+            bool ok = true;
+            for (int64_t qi = blockIdx.x; ok && qi < nq; qi += gridDim.x, ++qc) {
+                const QueryGeom qg = query_geom(qi, S_q, q_pos0, kv_pos0, S_kv, window);
+                ok = mbar_wait(&sm.meta_full[qc & 1], (qc >> 1) & 1u, kWaitIter);
+                if (!ok) break;
+                const int n_ent = sm.meta[qc & 1].n_ent;
+                const int n_tiles = qg.n_wt + (n_ent + kTile - 1) / kTile;
+                ok = mbar_wait(&sm.q_full, qc & 1u, kWaitIter);
+                if (!ok) break;
                 tc_fence_after();
+                for (int kt = 0; ok && kt < n_tiles; ++kt, ++g) {
+                    // S^T = K . Qr^T, chunk by chunk as the tile lands
+                    for (int c = 0; c < 8; ++c) {
+                        ok = mbar_wait(&sm.full[c], g & 1u, kWaitIter);
+                        if (!ok) break;
 #pragma unroll
-                for (int ks = 0; ks < kD / 16; ++ks) {
-                    const uint64_t a = sdesc_sw128(s_kv + (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u, 16, 1024);
-                    const uint64_t bq = sdesc_sw128(s_q + (uint32_t)(ks >> 2) * 8192u + (uint32_t)(ks & 3) * 32u, 16, 1024);
-                    mma_bf16(tmem + kColS, a, bq, kIdescQK, ks > 0);
+                        for (int k4 = 0; k4 < 4; ++k4) {
+                            const int ks = c * 4 + k4;
+                            const uint64_t a = sdesc_sw128(s_kv + (uint32_t)c * 16384u + (uint32_t)k4 * 32u, 16, 1024);
+                            const uint64_t bq = sdesc_sw128(s_q + (uint32_t)c * 8192u + (uint32_t)k4 * 32u, 16, 1024);
+                            mma_bf16(tmem + kColS, a, bq, kIdescQK, ks > 0 ? 1u : 0u);
+                        }
+                    }
+                    if (!ok) break;
+                    mma_commit(&sm.s_full);
+                    if (kt == n_tiles - 1) mma_commit(&sm.q_free);
+                    ok = mbar_wait(&sm.p_full, g & 1u, kWaitIter);
+                    if (!ok) break;
+                    tc_fence_after();
+                    // O^T += V^T . P^T, releasing each pair of key chunks when done
+#pragma unroll
+                    for (int mt = 0; mt < 4; ++mt) {
+#pragma unroll
+                        for (int kk = 0; kk < kTile / 16; ++kk) {
+                            const uint64_t a = sdesc_sw128(s_kv + (uint32_t)(2 * mt) * 16384u + (uint32_t)kk * 2048u, 16384, 1024);
+                            const uint64_t bp = sdesc_sw128(s_p + (uint32_t)kk * 2048u, 8192, 1024);
+                            mma_bf16(tmem + kColO + mt * 64, a, bp, kIdescPV, (kt > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        mma_commit(&sm.free_[mt]);
+                    }
                 }
-                mma_commit(&sm.bar_mma);
+                if (!ok) break;
+                if (n_tiles == 0) mma_commit(&sm.q_free);
+                mma_commit(&sm.o_full);
             }
-            if (!mbar_wait(&sm.bar_mma, phase)) {
+            if (!ok) {
                 atomicOr(&g_attend_tc_status, 1u);
                 sm.abort_ = 1;
             }
-            phase ^= 1;
-            tc_fence_after();
-
-            if (warp < 4) {
-                const int x = warp * 32 + lane;
-                float s[kH];
-                const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-                tmem_ld32(trow + kColS, s);
-                tmem_ld32(trow + kColS + 32, s + 32);
+        }
+    } else {
+        // ===================================================== softmax + epilogue
+        const int st = tid - 64;                 // 0..255
+        const int lg = warp & 3;                 // TMEM lane group
+        const int half = (warp - 2) >> 2;        // heads [32*half, 32*half + 32)
+        const int hb = half * 32;
+        const int x = lg * 32 + lane;            // key row / head-dim row of this thread
+        const uint32_t trow = tmem + ((uint32_t)(lg * 32) << 16);
+        const float c2 = scale * kLog2e;
+        uint32_t g = 0, qc = 0;
+        bool ok = true;
+        for (int64_t qi = blockIdx.x; ok && qi < nq; qi += gridDim.x, ++qc) {
+            const QueryGeom qg = query_geom(qi, S_q, q_pos0, kv_pos0, S_kv, window);
+            ok = mbar_wait(&sm.meta_full[qc & 1], (qc >> 1) & 1u, kWaitIter);
+            if (!ok) break;
+            const int n_ent = sm.meta[qc & 1].n_ent;
+            const int n_tiles = qg.n_wt + (n_ent + kTile - 1) / kTile;
+            if (st < kH) {
+                const float sk = sink[st];
+                sm.m_used[st] = sk == -INFINITY ? -INFINITY : sk * kLog2e;
+            }
+            named_sync(1, kSoftThreads);
+            float l_part[32];
+#pragma unroll
+            for (int h = 0; h < 32; ++h) l_part[h] = 0.f;
+            for (int kt = 0; kt < n_tiles; ++kt, ++g) {
+                ok = mbar_wait(&sm.s_full, g & 1u, kWaitIter);
+                if (!ok) break;
+                tc_fence_after();
+                const bool valid = kt < qg.n_wt ? (kt * kTile + x < qg.n_win)
+                                                : ((kt - qg.n_wt) * kTile + x < n_ent);
+                float s[32];
+                tmem_ld32(trow + kColS + hb, s);
                 tmem_ld_wait();
                 bool need = false;
 #pragma unroll
-                for (int h = 0; h < kH; ++h) {
-                    s[h] = x < tile_n ? s[h] * c2 : -INFINITY;
-                    need |= s[h] > sm.m_used[h] + kRescaleThreshold;
+                for (int h = 0; h < 32; ++h) {
+                    s[h] = valid ? s[h] * c2 : -INFINITY;
+                    need |= s[h] > sm.m_used[hb + h] + kRescaleThreshold;
                 }
                 if (need) atomicOr(&sm.flag, 1);
-                named_sync(1, 128);
+                named_sync(1, kSoftThreads);
                 const int flag = sm.flag;
-                named_sync(1, 128);
+                named_sync(1, kSoftThreads);
                 if (flag) {
-                    if (tid == 0) sm.flag = 0;
-                    float mx[kH];
+                    if (st == 0) sm.flag = 0;
+                    float mx[32];
 #pragma unroll
-                    for (int h = 0; h < kH; ++h) mx[h] = s[h];
-                    warp_reduce64<true>(mx);
-                    sm.red[warp][2 * lane] = mx[0];
-                    sm.red[warp][2 * lane + 1] = mx[1];
-                    named_sync(1, 128);
-                    if (tid < kH) {
-                        const float mt = fmaxf(fmaxf(sm.red[0][tid], sm.red[1][tid]),
-                                               fmaxf(sm.red[2][tid], sm.red[3][tid]));
-                        const float mo = sm.m_used[tid];
+                    for (int h = 0; h < 32; ++h) mx[h] = s[h];
+                    warp_reduce32<true>(mx);
+                    sm.red[lg][hb + lane] = mx[0];
+                    named_sync(1, kSoftThreads);
+                    if (st < kH) {
+                        const float mt = fmaxf(fmaxf(sm.red[0][st], sm.red[1][st]), fmaxf(sm.red[2][st], sm.red[3][st]));
+                        const float mo = sm.m_used[st];
                         const float mn = fmaxf(mo, mt);
-                        sm.alpha[tid] = mo == -INFINITY ? 0.f : exp2f(mo - mn);
-                        sm.m_used[tid] = mn;
+                        sm.alpha[st] = mo == -INFINITY ? 0.f : exp2f(mo - mn);
+                        sm.m_used[st] = mn;
                     }
-                    named_sync(1, 128);
+                    named_sync(1, kSoftThreads);
 #pragma unroll
-                    for (int h = 0; h < kH; ++h) l_part[h] *= sm.alpha[h];
+                    for (int h = 0; h < 32; ++h) l_part[h] *= sm.alpha[hb + h];
                     if (kt > 0) {
 #pragma unroll 1
                         for (int mt = 0; mt < 4; ++mt) {
                             float o[32];
-#pragma unroll 1
-                            for (int hh = 0; hh < 2; ++hh) {
-                                const uint32_t ta = trow + kColO + mt * 64 + hh * 32;
-                                tmem_ld32(ta, o);
-                                tmem_ld_wait();
+                            const uint32_t ta = trow + kColO + mt * 64 + hb;
+                            tmem_ld32(ta, o);
+                            tmem_ld_wait();
 #pragma unroll
-                                for (int h = 0; h < 32; ++h) o[h] *= sm.alpha[hh * 32 + h];
-                                tmem_st32(ta, o);
-                            }
+                            for (int h = 0; h < 32; ++h) o[h] *= sm.alpha[hb + h];
+                            tmem_st32(ta, o);
                         }
                         tmem_st_wait();
                     }
                 }
-                // P row of this key: 64 heads, bf16, swizzled
 #pragma unroll
-                for (int pc = 0; pc < 8; ++pc) {
+                for (int pc = 0; pc < 4; ++pc) {
                     float pv[8];
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         const int h = pc * 8 + k;
-                        pv[k] = exp2f(s[h] - sm.m_used[h]);
+                        pv[k] = exp2f(s[h] - sm.m_used[hb + h]);
                         l_part[h] += pv[k];
                     }
                     uint4 u;
                     __nv_bfloat162 *hp = reinterpret_cast<__nv_bfloat162 *>(&u);
 #pragma unroll
                     for (int k = 0; k < 4; ++k) hp[k] = __floats2bfloat162_rn(pv[2 * k], pv[2 * k + 1]);
-                    const uint32_t dst = s_p + sw128((uint32_t)x, (uint32_t)pc);
+                    const uint32_t dst = s_p + sw128((uint32_t)x, (uint32_t)(half * 4 + pc));
                     asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(u.x), "r"(u.y),
                                  "r"(u.z), "r"(u.w)
                                  : "memory");
                 }
                 fence_async_smem();
                 tc_fence_before();
+                mbar_arrive(&sm.p_full);
             }
-            __syncthreads();
-
-            // O^T += V^T . P^T
-            if (tid == 0) {
-                tc_fence_after();
-#pragma unroll
-                for (int mt = 0; mt < 4; ++mt) {
-#pragma unroll
-                    for (int kk = 0; kk < kTile / 16; ++kk) {
-                        const uint64_t a = sdesc_sw128(s_kv + (uint32_t)(2 * mt) * 16384u + (uint32_t)kk * 2048u, 16384, 1024);
-                        const uint64_t bp = sdesc_sw128(s_p + (uint32_t)kk * 2048u, 8192, 1024);
-                        mma_bf16(tmem + kColO + mt * 64, a, bp, kIdescPV, (kt > 0 || kk > 0) ? 1u : 0u);
-                    }
-                }
-                mma_commit(&sm.bar_mma);
+            if (!ok) break;
+            // ---- epilogue: l, normalisation, de-rotation, store
+            warp_reduce32<false>(l_part);
+            sm.red[lg][hb + lane] = l_part[0];
+            named_sync(1, kSoftThreads);
+            if (st < kH) {
+                float l = sm.red[0][st] + sm.red[1][st] + sm.red[2][st] + sm.red[3][st];
+                const float sk = sink[st];
+                if (sk != -INFINITY) l += exp2f(sk * kLog2e - sm.m_used[st]);
+                sm.inv_l[st] = l > 0.f ? 1.f / l : 0.f;
             }
-            if (!mbar_wait(&sm.bar_mma, phase)) {
-                atomicOr(&g_attend_tc_status, 1u);
-                sm.abort_ = 1;
-            }
-            phase ^= 1;
+            ok = mbar_wait(&sm.o_full, qc & 1u, kWaitIter);
+            named_sync(1, kSoftThreads);
+            if (!ok) break;
             tc_fence_after();
-            __syncthreads();
-            if (sm.abort_) break;
-        }
-        if (sm.abort_) break;
-
-        // ---- epilogue: l, normalisation, de-rotation, store
-        __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(smem + kOffKv);  // [64][512]
-        if (warp < 4) {
-            warp_reduce64<false>(l_part);
-            sm.red[warp][2 * lane] = l_part[0];
-            sm.red[warp][2 * lane + 1] = l_part[1];
-            named_sync(1, 128);
-            if (tid < kH) {
-                float l = sm.red[0][tid] + sm.red[1][tid] + sm.red[2][tid] + sm.red[3][tid];
-                const float sk = sink[tid];
-                if (sk != -INFINITY) l += exp2f(sk * kLog2e - sm.m_used[tid]);
-                sm.inv_l[tid] = l > 0.f ? 1.f / l : 0.f;
-            }
-            named_sync(1, 128);
-            const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+            __nv_bfloat16 *orow = out + qi * (int64_t)kH * kD;
+            float inv_l[32];
+#pragma unroll
+            for (int h = 0; h < 32; ++h) inv_l[h] = sm.inv_l[hb + h];
 #pragma unroll 1
             for (int mt = 0; mt < 4; ++mt) {
-                const int d = mt * 128 + warp * 32 + lane;
+                const int d = mt * 128 + x;
                 float cs = 1.f, sn = 0.f;
                 const bool rot = d >= rope.first;
-                if (rot) rope_cs(-(double)t, rope.inv_freq[(d - rope.first) >> 1], &cs, &sn);
-#pragma unroll 1
-                for (int hh = 0; hh < 2; ++hh) {
-                    float o[32];
-                    tmem_ld32(trow + kColO + mt * 64 + hh * 32, o);
+                if (rot) rope_cs(-(double)qg.t, rope.inv_freq[(d - rope.first) >> 1], &cs, &sn);
+                float o[32];
+                if (n_tiles > 0) {
+                    tmem_ld32(trow + kColO + mt * 64 + hb, o);
                     tmem_ld_wait();
+                } else {
+#pragma unroll
+                    for (int h = 0; h < 32; ++h) o[h] = 0.f;
+                }
+                float pr[32];
+#pragma unroll
+                for (int h = 0; h < 32; ++h) {
+                    o[h] *= inv_l[h];
+                    pr[h] = __shfl_xor_sync(0xFFFFFFFFu, o[h], 1);
+                }
+                if ((lane & 1) == 0) {
 #pragma unroll
                     for (int h = 0; h < 32; ++h) {
-                        float v = o[h] * sm.inv_l[hh * 32 + h];
-                        float partner = __shfl_xor_sync(0xFFFFFFFFu, v, 1);
-                        if (rot) v = (d & 1) == 0 ? v * cs - partner * sn : partner * sn + v * cs;
-                        stage[(hh * 32 + h) * kD + d] = __float2bfloat16_rn(v);
+                        const float a = o[h], bb = pr[h];
+                        const float ra = rot ? a * cs - bb * sn : a;
+                        const float rb = rot ? a * sn + bb * cs : bb;
+                        *reinterpret_cast<__nv_bfloat162 *>(orow + (int64_t)(hb + h) * kD + d) =
+                            __floats2bfloat162_rn(ra, rb);
                     }
                 }
             }
             tc_fence_before();
         }
-        __syncthreads();
-        uint4 *dst = reinterpret_cast<uint4 *>(out + qi * (int64_t)kH * kD);
-        const uint4 *src4 = reinterpret_cast<const uint4 *>(stage);
-        for (int v = tid; v < kH * kD / 8; v += kThreads) dst[v] = src4[v];
-        __syncthreads();
+        if (!ok) {
+            atomicOr(&g_attend_tc_status, 1u);
+            sm.abort_ = 1;
+        }
     }
 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 0) tmem_dealloc(tmem, 512);
+    if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace
 
 bool attend_tc_eligible(const AttendArgs &a) {
     if (a.dtype != CSA_BF16 || a.H != kH || a.D != kD) return false;
-    if (a.rope_dim > a.D) return false;
+    if (a.rope_dim > 64) return false;               // rope channels inside the last chunk
     if (a.mode == 0 && a.topk > 2048) return false;
+    // TMA row coordinates are 32-bit
+    if (a.B * a.S_q * kH >= (1ll << 31) || a.B * a.S_kv + kTile >= (1ll << 31) ||
+        a.B * a.P >= (1ll << 31))
+        return false;
     // keys are rotated once per call: worth it when the queries outnumber the key rows
     // (prefill); a few queries over a long cache take the general path
     return (double)a.S_q * 64.0 >= (double)(a.S_kv + a.P);
@@ -450,6 +622,11 @@ csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st) {
                                             a.D, a.rope);
         CSA_CHECK_LAUNCH("attend: rotate entries");
     }
+    CUtensorMap map_q, map_kv;
+    const uint64_t kv_rows = (uint64_t)(a.B * a.S_kv > 0 ? a.B * a.S_kv : 1);
+    CSA_REQUIRE(encode_map_bf16_2d(&map_q, a.q, kD, (uint64_t)(a.B * a.S_q * kH), 64u, 64u) &&
+                    encode_map_bf16_2d(&map_kv, kv_rot, kD, kv_rows, 64u, (uint32_t)kTile),
+                CSA_ERR_CUDA, "attend: cannot encode the TMA tensor maps");
     const size_t smem = tc_smem_bytes(a.mode == 0 ? a.topk : 1);
     CSA_REQUIRE(smem <= 232448, CSA_ERR_UNSUPPORTED, "attend: shared memory %zu B too large", smem);
     cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -459,9 +636,8 @@ csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st) {
     const int64_t nq = a.B * a.S_q;
     const int grid = (int)(nq < sms ? nq : sms);
     attend_tc_kernel<<<grid, kThreads, smem, st>>>(
-        (const __nv_bfloat16 *)a.q, kv_rot, a.S_kv, a.kv_pos0, pool_rot, a.P, a.idx,
-        a.mode == 0 ? a.topk : 0, a.mode, a.sink, (__nv_bfloat16 *)a.out, a.B, a.S_q, a.q_pos0,
-        a.window, a.ratio, a.scale, a.rope);
+        map_q, map_kv, pool_rot, a.S_kv, a.kv_pos0, a.P, a.idx, a.mode == 0 ? a.topk : 0, a.mode,
+        a.sink, (__nv_bfloat16 *)a.out, a.B, a.S_q, a.q_pos0, a.window, a.ratio, a.scale, a.rope);
     CSA_CHECK_LAUNCH(a.mode == 0 ? "csa_attend" : "hca_attend");
     return CSA_OK;
 }

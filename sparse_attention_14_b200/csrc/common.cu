@@ -1,6 +1,9 @@
 // common.cu -- error state, RoPE tables and path selection of libcsa_b200.
+#include <cudaTypedefs.h>
 #include <stdarg.h>
+
 #include <atomic>
+#include <mutex>
 #include <string.h>
 
 #include "attend.cuh"
@@ -22,6 +25,27 @@ void set_error(const char *fmt, ...) {
 }
 
 void clear_error() { g_error[0] = '\0'; }
+
+bool encode_map_bf16_2d(CUtensorMap *map, const void *ptr, uint64_t cols, uint64_t rows,
+                        uint32_t box_cols, uint32_t box_rows) {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t es[2] = {1u, 1u};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 void make_rope_table(RopeTable *t, int D, int R, double base) {
     memset(t, 0, sizeof(*t));

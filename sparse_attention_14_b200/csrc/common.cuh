@@ -2,6 +2,7 @@
 // RoPE angles, argument checks.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -98,6 +99,13 @@ __device__ __forceinline__ void rope_cs(double pos, double inv_freq, float *c, f
     phi -= two_pi * rint(phi * (1.0 / two_pi));
     sincosf((float)phi, s, c);
 }
+
+// ---------------------------------------------------------------- TMA descriptors
+// 2-D bf16 tensor map over `rows` rows of `cols` elements (row pitch cols*2 bytes), box
+// {box_cols, box_rows}, 128-byte swizzle, zero fill out of bounds.  The driver entry
+// point is looked up once through the runtime, so the library links no driver library.
+bool encode_map_bf16_2d(CUtensorMap *map, const void *ptr, uint64_t cols, uint64_t rows,
+                        uint32_t box_cols, uint32_t box_rows);
 
 // ---------------------------------------------------------------- misc
 __host__ __device__ __forceinline__ int64_t n_visible(int64_t t, int64_t ratio, int64_t P) {

@@ -41,6 +41,10 @@ MID = [
     LayerSpec(name="mid_csa_ragged_bf16", dtype="bf16", B=1, S_q=700, S_kv=700, q_pos0=0,
               kv_pos0=0, H=64, D=512, R=64, base=160000.0, W=100, m=4, P=175, kind="csa",
               H_I=64, d_I=128, topk=37, workload=98),
+    # a window longer than one 128-key tile, HCA-style entries
+    LayerSpec(name="mid_hca_w200_bf16", dtype="bf16", B=2, S_q=600, S_kv=600, q_pos0=0,
+              kv_pos0=0, H=64, D=512, R=64, base=160000.0, W=200, m=16, P=37, kind="hca",
+              workload=88),
     # indexer buffer cuts (more than 1024 visible entries) and a top-k that is not a
     # power of two
     LayerSpec(name="mid_csa_cut_bf16", dtype="bf16", B=1, S_q=4801, S_kv=4801, q_pos0=0,
