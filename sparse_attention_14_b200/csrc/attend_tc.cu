@@ -108,6 +108,111 @@ __global__ void rope_rows_kernel(const __nv_bfloat16 *__restrict__ src, __nv_bfl
     store8(dst + ((int64_t)b * rows + r) * D + pc * 8, x);
 }
 
+// Decode-sized calls: gather each query's keys (window rows, then its valid entries in
+// slot order / every visible entry) into a packed buffer [B*S_q][kmax][D], rotated at
+// their positions, and record the key count per query.  Only the rows a query reads are
+// touched, instead of rotating the whole cache.  Two kernels: one warp per query lists
+// the key sources; then (query, 16-row slice) blocks copy and rotate the rows.
+__global__ void __launch_bounds__(32) pack_list_kernel(const int32_t *__restrict__ idx, int topk, int mode,
+                                                       int64_t S_kv, int64_t kv_pos0, int64_t P, int64_t S_q,
+                                                       int64_t q_pos0, int window, int ratio, int kmax,
+                                                       int32_t *__restrict__ ent_ws, int32_t *__restrict__ n_keys) {
+    const int64_t qi = blockIdx.x;
+    const int lane = threadIdx.x;
+    const int64_t t = q_pos0 + qi % S_q;
+    const int64_t nv = n_visible(t, ratio, P);
+    int64_t lo = t - window + 1;
+    if (lo < kv_pos0) lo = kv_pos0;
+    const int64_t hi = t < kv_pos0 + S_kv - 1 ? t : kv_pos0 + S_kv - 1;
+    const int n_win = hi >= lo ? (int)(hi - lo + 1) : 0;
+    int n_ent;
+    if (mode == 0) {
+        int cnt = 0;
+        const int32_t *ip = idx + qi * topk;
+        int32_t *ep = ent_ws + qi * (int64_t)kmax;
+        for (int c0 = 0; c0 < topk; c0 += 256) {
+            int32_t jv[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int c = c0 + k * 32 + lane;
+                jv[k] = c < topk ? ip[c] : -1;
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const bool ok = jv[k] >= 0 && (int64_t)jv[k] < nv;
+                const unsigned ball = __ballot_sync(0xFFFFFFFFu, ok);
+                if (ok) ep[cnt + __popc(ball & ((1u << lane) - 1u))] = jv[k];
+                cnt += __popc(ball);
+            }
+        }
+        n_ent = cnt;
+    } else {
+        n_ent = (int)nv;
+    }
+    int nk = n_win + n_ent;
+    if (nk > kmax) nk = kmax;
+    if (lane == 0) n_keys[qi] = nk;
+}
+
+constexpr int kPackRows = 16;
+__global__ void __launch_bounds__(128) pack_rows_kernel(
+    const __nv_bfloat16 *__restrict__ kv, int64_t S_kv, int64_t kv_pos0, const __nv_bfloat16 *__restrict__ pool,
+    int64_t P, int mode, int64_t S_q, int64_t q_pos0, int window, int ratio, RopeTable rope,
+    const int32_t *__restrict__ ent_ws, const int32_t *__restrict__ n_keys, __nv_bfloat16 *__restrict__ packed,
+    int kmax) {
+    const int64_t qi = blockIdx.x;
+    const int x0 = blockIdx.y * kPackRows;
+    const int nk = n_keys[qi];
+    if (x0 >= nk) return;
+    const int64_t b = qi / S_q, t = q_pos0 + qi % S_q;
+    int64_t lo = t - window + 1;
+    if (lo < kv_pos0) lo = kv_pos0;
+    const int64_t hi = t < kv_pos0 + S_kv - 1 ? t : kv_pos0 + S_kv - 1;
+    const int n_win = hi >= lo ? (int)(hi - lo + 1) : 0;
+    constexpr int kPieces = kD / 8;
+    constexpr int kPer = kPackRows * kPieces / 128;       // 8 pieces per thread
+    float e[kPer][8];
+    double pos[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int v = threadIdx.x + u * 128;
+        const int x = x0 + v / kPieces, pc = v % kPieces;
+        if (x < nk) {
+            const __nv_bfloat16 *src;
+            if (x < n_win) {
+                src = kv + (b * S_kv + (lo - kv_pos0) + x) * kD;
+                pos[u] = (double)(lo + x);
+            } else {
+                const int64_t j = mode == 0 ? (int64_t)ent_ws[qi * (int64_t)kmax + (x - n_win)] : (int64_t)(x - n_win);
+                src = pool + (b * P + j) * kD;
+                pos[u] = (double)j * (double)ratio;
+            }
+            load8(src + pc * 8, e[u]);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int v = threadIdx.x + u * 128;
+        const int x = x0 + v / kPieces, pc = v % kPieces;
+        if (x >= nk) continue;
+        const int d0 = pc * 8;
+        if (d0 + 8 > rope.first) {
+#pragma unroll
+            for (int c = 0; c < 8; c += 2) {
+                const int d = d0 + c;
+                if (d >= rope.first) {
+                    float cs, sn;
+                    rope_cs(pos[u], rope.inv_freq[(d - rope.first) >> 1], &cs, &sn);
+                    const float a0 = e[u][c], a1 = e[u][c + 1];
+                    e[u][c] = a0 * cs - a1 * sn;
+                    e[u][c + 1] = a0 * sn + a1 * cs;
+                }
+            }
+        }
+        store8(packed + (qi * kmax + x) * kD + pc * 8, e[u]);
+    }
+}
+
 // warp butterfly over 32 per-lane values: afterwards lane L holds in v[0] the reduction
 // over the warp of value L.
 template <bool kMax>
@@ -139,12 +244,20 @@ struct QueryGeom {
     int n_win, n_wt;
 };
 
+// packed != nullptr: the keys of query qi are the n_keys[qi] rows qi*kmax... of a packed,
+// already rotated buffer (decode-sized calls), all loaded like window rows.
 __device__ __forceinline__ QueryGeom query_geom(int64_t qi, int64_t S_q, int64_t q_pos0, int64_t kv_pos0,
-                                                int64_t S_kv, int window) {
+                                                int64_t S_kv, int window, const int32_t *packed_n) {
     QueryGeom g;
     g.b = qi / S_q;
     g.i = qi % S_q;
     g.t = q_pos0 + g.i;
+    if (packed_n) {
+        g.lo_w = 0;
+        g.n_win = packed_n[qi];
+        g.n_wt = (g.n_win + kTile - 1) / kTile;
+        return g;
+    }
     int64_t lo = g.t - window + 1;
     if (lo < kv_pos0) lo = kv_pos0;
     int64_t hi = g.t < kv_pos0 + S_kv - 1 ? g.t : kv_pos0 + S_kv - 1;
@@ -159,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     const __nv_bfloat16 *__restrict__ pool_rot, int64_t S_kv, int64_t kv_pos0, int64_t P,
     const int32_t *__restrict__ idx, int topk, int mode, const float *__restrict__ sink,
     __nv_bfloat16 *__restrict__ out, int64_t B, int64_t S_q, int64_t q_pos0, int window, int ratio,
-    float scale, RopeTable rope) {
+    float scale, RopeTable rope, const int32_t *__restrict__ packed_n, int kmax) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     unsigned char *smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -197,10 +310,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         // ===================================================== loader
         uint32_t g = 0, qc = 0;
         for (int64_t qi = blockIdx.x; qi < nq && !sm.abort_; qi += gridDim.x, ++qc) {
-            const QueryGeom qg = query_geom(qi, S_q, q_pos0, kv_pos0, S_kv, window);
+            const QueryGeom qg = query_geom(qi, S_q, q_pos0, kv_pos0, S_kv, window, packed_n);
             const int64_t nv = n_visible(qg.t, ratio, P);
             int n_ent;
-            if (mode == 0) {
+            if (packed_n) {
+                n_ent = 0;
+            } else if (mode == 0) {
                 // compact the valid idx values in slot order; eight loads per lane in flight
                 int cnt = 0;
                 const int32_t *ip = idx + qi * topk;
@@ -302,7 +417,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 const bool win = kt < qg.n_wt;
                 if (win) {
                     // window rows are contiguous: one 2-D TMA box of 128 rows per chunk
-                    const int y0 = (int)(qg.b * S_kv + (qg.lo_w - kv_pos0) + (int64_t)kt * kTile);
+                    const int y0 = packed_n ? (int)(qi * kmax + (int64_t)kt * kTile)
+                                            : (int)(qg.b * S_kv + (qg.lo_w - kv_pos0) + (int64_t)kt * kTile);
                     for (int c = 0; c < 8 && ok; ++c) {
                         if ((c & 1) == 0 && g > 0) ok = mbar_wait(&sm.free_[c >> 1], (g - 1) & 1u, kWaitIter);
                         if (ok && lane == 0) {
@@ -373,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             uint32_t g = 0, qc = 0;
             bool ok = true;
             for (int64_t qi = blockIdx.x; ok && qi < nq; qi += gridDim.x, ++qc) {
-                const QueryGeom qg = query_geom(qi, S_q, q_pos0, kv_pos0, S_kv, window);
+                const QueryGeom qg = query_geom(qi, S_q, q_pos0, kv_pos0, S_kv, window, packed_n);
                 ok = mbar_wait(&sm.meta_full[qc & 1], (qc >> 1) & 1u, kWaitIter);
                 if (!ok) break;
                 const int n_ent = sm.meta[qc & 1].n_ent;
@@ -433,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         uint32_t g = 0, qc = 0;
         bool ok = true;
         for (int64_t qi = blockIdx.x; ok && qi < nq; qi += gridDim.x, ++qc) {
-            const QueryGeom qg = query_geom(qi, S_q, q_pos0, kv_pos0, S_kv, window);
+            const QueryGeom qg = query_geom(qi, S_q, q_pos0, kv_pos0, S_kv, window, packed_n);
             ok = mbar_wait(&sm.meta_full[qc & 1], (qc >> 1) & 1u, kWaitIter);
             if (!ok) break;
             const int n_ent = sm.meta[qc & 1].n_ent;
@@ -593,12 +709,28 @@ bool attend_tc_eligible(const AttendArgs &a) {
     if (a.B * a.S_q * kH >= (1ll << 31) || a.B * a.S_kv + kTile >= (1ll << 31) ||
         a.B * a.P >= (1ll << 31))
         return false;
-    // keys are rotated once per call: worth it when the queries outnumber the key rows
-    // (prefill); a few queries over a long cache take the general path
-    return (double)a.S_q * 64.0 >= (double)(a.S_kv + a.P);
+    if (attend_tc_packed(a) && a.B * a.S_q * (int64_t)attend_tc_kmax(a) + kTile >= (1ll << 31)) return false;
+    return true;
+}
+
+// Prefill (the queries outnumber the key rows): every window row and entry is rotated once
+// into the workspace and tiles gather from there.  Decode-sized calls (few queries over a
+// long cache) instead pack just the rows each query reads.
+bool attend_tc_packed(const AttendArgs &a) { return (double)a.S_q * 64.0 < (double)(a.S_kv + a.P); }
+
+int attend_tc_kmax(const AttendArgs &a) {
+    // an upper bound that needs no window size (the workspace query does not take one):
+    // every raw row given plus every entry the query can list
+    const int64_t e = a.mode == 0 ? (a.topk < a.P ? a.topk : a.P) : a.P;
+    return (int)(a.S_kv + e > 0 ? a.S_kv + e : 1);
 }
 
 size_t attend_tc_workspace(const AttendArgs &a) {
+    if (attend_tc_packed(a)) {
+        const size_t rows = (size_t)a.B * a.S_q * attend_tc_kmax(a);
+        return ((rows * kD * 2 + 255) & ~(size_t)255) + (((size_t)a.B * a.S_q * 4 + 255) & ~(size_t)255) +
+               rows * 4;   // packed keys, key counts, entry lists
+    }
     size_t kv = ((size_t)a.B * a.S_kv * a.D * 2 + 255) & ~(size_t)255;
     size_t pl = ((size_t)a.B * a.P * a.D * 2 + 255) & ~(size_t)255;
     return kv + pl;
@@ -606,28 +738,49 @@ size_t attend_tc_workspace(const AttendArgs &a) {
 
 csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st) {
     char *ws = reinterpret_cast<char *>(a.workspace);
+    const bool packed = attend_tc_packed(a);
+    const int kmax = packed ? attend_tc_kmax(a) : 0;
     __nv_bfloat16 *kv_rot = reinterpret_cast<__nv_bfloat16 *>(ws);
-    __nv_bfloat16 *pool_rot = reinterpret_cast<__nv_bfloat16 *>(
-        ws + (((size_t)a.B * a.S_kv * a.D * 2 + 255) & ~(size_t)255));
+    __nv_bfloat16 *pool_rot = nullptr;
+    int32_t *n_keys = nullptr;
+    uint64_t kv_rows;
     const int pieces = a.D / 8;
-    if (a.S_kv > 0) {
-        dim3 g((unsigned)ceil_div(a.S_kv * pieces, 256), (unsigned)a.B);
-        rope_rows_kernel<<<g, 256, 0, st>>>((const __nv_bfloat16 *)a.kv, kv_rot, a.S_kv, a.kv_pos0, 1,
-                                            a.D, a.rope);
-        CSA_CHECK_LAUNCH("attend: rotate window rows");
-    }
-    if (a.P > 0) {
-        dim3 g((unsigned)ceil_div(a.P * pieces, 256), (unsigned)a.B);
-        rope_rows_kernel<<<g, 256, 0, st>>>((const __nv_bfloat16 *)a.pool, pool_rot, a.P, 0, a.ratio,
-                                            a.D, a.rope);
-        CSA_CHECK_LAUNCH("attend: rotate entries");
+    if (packed) {
+        const size_t rows = (size_t)a.B * a.S_q * kmax;
+        const size_t keys_bytes = (rows * kD * 2 + 255) & ~(size_t)255;
+        n_keys = reinterpret_cast<int32_t *>(ws + keys_bytes);
+        int32_t *ent_ws = reinterpret_cast<int32_t *>(ws + keys_bytes + (((size_t)a.B * a.S_q * 4 + 255) & ~(size_t)255));
+        kv_rows = rows;
+        pack_list_kernel<<<(unsigned)(a.B * a.S_q), 32, 0, st>>>(a.idx, a.mode == 0 ? a.topk : 0, a.mode, a.S_kv,
+                                                                 a.kv_pos0, a.P, a.S_q, a.q_pos0, a.window, a.ratio,
+                                                                 kmax, ent_ws, n_keys);
+        CSA_CHECK_LAUNCH("attend: list keys");
+        dim3 pg((unsigned)(a.B * a.S_q), (unsigned)ceil_div(kmax, kPackRows));
+        pack_rows_kernel<<<pg, 128, 0, st>>>((const __nv_bfloat16 *)a.kv, a.S_kv, a.kv_pos0,
+                                            (const __nv_bfloat16 *)a.pool, a.P, a.mode, a.S_q, a.q_pos0, a.window,
+                                            a.ratio, a.rope, ent_ws, n_keys, kv_rot, kmax);
+        CSA_CHECK_LAUNCH("attend: pack keys");
+    } else {
+        pool_rot = reinterpret_cast<__nv_bfloat16 *>(ws + (((size_t)a.B * a.S_kv * a.D * 2 + 255) & ~(size_t)255));
+        kv_rows = (uint64_t)(a.B * a.S_kv > 0 ? a.B * a.S_kv : 1);
+        if (a.S_kv > 0) {
+            dim3 g((unsigned)ceil_div(a.S_kv * pieces, 256), (unsigned)a.B);
+            rope_rows_kernel<<<g, 256, 0, st>>>((const __nv_bfloat16 *)a.kv, kv_rot, a.S_kv, a.kv_pos0, 1,
+                                                a.D, a.rope);
+            CSA_CHECK_LAUNCH("attend: rotate window rows");
+        }
+        if (a.P > 0) {
+            dim3 g((unsigned)ceil_div(a.P * pieces, 256), (unsigned)a.B);
+            rope_rows_kernel<<<g, 256, 0, st>>>((const __nv_bfloat16 *)a.pool, pool_rot, a.P, 0, a.ratio,
+                                                a.D, a.rope);
+            CSA_CHECK_LAUNCH("attend: rotate entries");
+        }
     }
     CUtensorMap map_q, map_kv;
-    const uint64_t kv_rows = (uint64_t)(a.B * a.S_kv > 0 ? a.B * a.S_kv : 1);
     CSA_REQUIRE(encode_map_bf16_2d(&map_q, a.q, kD, (uint64_t)(a.B * a.S_q * kH), 64u, 64u) &&
                     encode_map_bf16_2d(&map_kv, kv_rot, kD, kv_rows, 64u, (uint32_t)kTile),
                 CSA_ERR_CUDA, "attend: cannot encode the TMA tensor maps");
-    const size_t smem = tc_smem_bytes(a.mode == 0 ? a.topk : 1);
+    const size_t smem = tc_smem_bytes(a.mode == 0 && !packed ? a.topk : 1);
     CSA_REQUIRE(smem <= 232448, CSA_ERR_UNSUPPORTED, "attend: shared memory %zu B too large", smem);
     cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     int dev = 0, sms = 148;
@@ -636,8 +789,8 @@ csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st) {
     const int64_t nq = a.B * a.S_q;
     const int grid = (int)(nq < sms ? nq : sms);
     attend_tc_kernel<<<grid, kThreads, smem, st>>>(
-        map_q, map_kv, pool_rot, a.S_kv, a.kv_pos0, a.P, a.idx, a.mode == 0 ? a.topk : 0, a.mode,
-        a.sink, (__nv_bfloat16 *)a.out, a.B, a.S_q, a.q_pos0, a.window, a.ratio, a.scale, a.rope);
+        map_q, map_kv, pool_rot, a.S_kv, a.kv_pos0, a.P, a.idx, a.mode == 0 && !packed ? a.topk : 0, a.mode,
+        a.sink, (__nv_bfloat16 *)a.out, a.B, a.S_q, a.q_pos0, a.window, a.ratio, a.scale, a.rope, n_keys, kmax);
     CSA_CHECK_LAUNCH(a.mode == 0 ? "csa_attend" : "hca_attend");
     return CSA_OK;
 }
@@ -656,7 +809,7 @@ void *g_noalloc_ptr[kMaxDevices];  // device address of g_noalloc_scratch, per d
 }  // namespace
 
 csa_status_t attend_tc_noalloc(AttendArgs &a, cudaStream_t st) {
-    CSA_REQUIRE(attend_tc_eligible(a), CSA_ERR_UNSUPPORTED,
+    CSA_REQUIRE(attend_tc_eligible(a) && !attend_tc_packed(a), CSA_ERR_UNSUPPORTED,
                 "csa_attend_noalloc: only the bf16, 64-head, head_dim-512 prefill shape is "
                 "handled (S_q * 64 >= S_kv + P)");
     const size_t need = attend_tc_workspace(a);

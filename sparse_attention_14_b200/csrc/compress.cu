@@ -10,9 +10,9 @@
 // (8 bf16 or 4+4 fp32 as two vectors), a warp covers 256 contiguous channels of one row,
 // and each thread keeps a running (max, sum of weights, weighted sum) per channel --
 // an online softmax -- so the window is read exactly once, in one pass.
-//  * short windows (CSA: 2m = 8 tokens): one thread per (entry, 8 channels), the
-//    window loop fully in registers;
-//  * long windows (HCA: 128 tokens): the window is split over `split` thread rows of
+//  * short windows (up to 8 tokens, e.g. CSA: 2m = 8): one thread per (entry, 8
+//    channels), the window loaded four tokens at a time into registers;
+//  * longer windows (HCA: 128 tokens): the window is split over `split` thread rows of
 //    one CTA, each row reads every split-th token (so a warp-row reads consecutive rows
 //    of HBM), and the partial softmax states are merged through shared memory.
 #include "common.cuh"
@@ -49,8 +49,10 @@ struct SoftPool8 {
     }
 };
 
-// One thread per (b, j, 8-channel group); window loop in registers.
-template <typename T>
+// One thread per (b, j, 8-channel group).  The window (at most WIN tokens) is read in
+// batches of four tokens, the eight 16-byte loads of a batch issued together before their
+// tokens are folded into the running softmax.
+template <typename T, int WIN>
 __global__ void __launch_bounds__(256) compress_rows_kernel(const T *__restrict__ kv,
                                                             const T *__restrict__ gate,
                                                             T *__restrict__ pool, int64_t B,
@@ -65,17 +67,24 @@ __global__ void __launch_bounds__(256) compress_rows_kernel(const T *__restrict_
     int64_t b = gid / ((int64_t)groups * P);
     int64_t lo = overlap ? (j - 1) * ratio : j * ratio;
     if (lo < 0) lo = 0;
-    int64_t hi = (j + 1) * ratio;
-    const T *kv_p = kv + (b * S) * D + g8 * 8;
-    const T *g_p = gate + (b * S) * D + g8 * 8;
+    const int n = (int)((j + 1) * ratio - lo);   // <= WIN
+    const T *kv_p = kv + (b * S + lo) * D + g8 * 8;
+    const T *g_p = gate + (b * S + lo) * D + g8 * 8;
     SoftPool8 st;
     st.init();
-    float gv[8], vv[8];
-#pragma unroll 4
-    for (int64_t s = lo; s < hi; ++s) {
-        load8(g_p + s * D, gv);
-        load8(kv_p + s * D, vv);
-        st.add(gv, vv);
+#pragma unroll
+    for (int s0 = 0; s0 < WIN; s0 += 4) {
+        float gv[4][8], vv[4][8];
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            if (s0 + s < n) {
+                load8(g_p + (int64_t)(s0 + s) * D, gv[s]);
+                load8(kv_p + (int64_t)(s0 + s) * D, vv[s]);
+            }
+        }
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            if (s0 + s < n) st.add(gv[s], vv[s]);
     }
     float o[8];
 #pragma unroll
@@ -139,12 +148,12 @@ template <typename T>
 csa_status_t launch_compress(const T *kv, const T *gate, T *pool, int64_t B, int64_t S, int D,
                              int ratio, int overlap, int64_t P, cudaStream_t st) {
     const int64_t win = overlap ? 2 * (int64_t)ratio : ratio;
-    if (win <= 16) {
+    if (win <= 8) {
         int64_t total = B * P * (D / 8);
         int64_t blocks = ceil_div(total, 256);
         CSA_REQUIRE(blocks < (1ll << 31), CSA_ERR_UNSUPPORTED, "csa_compress: too many entries");
-        compress_rows_kernel<T><<<(unsigned)blocks, 256, 0, st>>>(kv, gate, pool, B, S, D, ratio,
-                                                                  overlap, P);
+        compress_rows_kernel<T, 8><<<(unsigned)blocks, 256, 0, st>>>(kv, gate, pool, B, S, D, ratio,
+                                                                     overlap, P);
     } else {
         int split = 8;
         while (split > 1 && win / split < 4) split /= 2;

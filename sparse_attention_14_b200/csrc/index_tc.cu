@@ -55,14 +55,16 @@ struct Misc {
 template <int QB>
 struct Cfg {
     static constexpr int N = QB * 64;
-    static constexpr int NE = QB == 4 ? 8 : 4;          // epilogue warps
+    static constexpr int NE = 8;                         // epilogue warps (two per TMEM lane group)
     static constexpr int kThreads = (2 + NE) * 32;
-    static constexpr int NST = QB == 4 ? 3 : 4;          // entry-tile stages
+    static constexpr int NST = QB == 4 ? 3 : 2;          // entry-tile stages (QB=1: two CTAs per SM)
+    static constexpr int kMinBlocks = QB == 4 ? 1 : 2;
     static constexpr uint32_t kBChunk = QB * 64 * 128;   // one 64-column chunk of q_I rows
     static constexpr uint32_t kBBytes = 2 * kBChunk;
     static constexpr uint32_t kABytes = kTileE * kDI * 2;
     static constexpr int GS = NE * 32 / QB;              // threads per query group
-    static constexpr int QPT = QB == 4 ? 2 : QB;         // queries per epilogue thread
+    static constexpr int QPT = QB == 4 ? 2 : 1;          // queries per epilogue thread
+    static constexpr int CPT = QB == 4 ? 64 : 32;        // head columns per query per thread
     static constexpr uint32_t kTmemCols = 2 * N <= 128 ? 128 : (2 * N <= 256 ? 256 : 512);
     static constexpr uint32_t kOffB = 0;
     static constexpr uint32_t kOffA = kBBytes;
@@ -204,7 +206,7 @@ __device__ void group_emit(unsigned long long *cand, int n, int k, int gt, int b
 
 // ------------------------------------------------------------------ main kernel
 template <int QB>
-__global__ void __launch_bounds__(Cfg<QB>::kThreads, 1) index_tc_kernel(
+__global__ void __launch_bounds__(Cfg<QB>::kThreads, Cfg<QB>::kMinBlocks) index_tc_kernel(
     const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
     const __nv_bfloat16 *__restrict__ w, int64_t B, int64_t S_q, int64_t q_pos0, int64_t P, int ratio,
     int topk, int n_split, int32_t *__restrict__ idx, float *__restrict__ scores_opt,
@@ -311,6 +313,7 @@ __global__ void __launch_bounds__(Cfg<QB>::kThreads, 1) index_tc_kernel(
         const int g4 = warp & 3;                     // TMEM lane group of this warp
         const int row = g4 * 32 + lane;              // entry row inside the tile
         const int qa = QB == 4 ? 2 * (e >> 2) : 0;   // first query of this thread
+        const int cb = QB == 4 ? 0 : 32 * (e >> 2);  // first head column (QB=1: half of 64)
         const int et = e * 32 + lane;                // epilogue thread id
         const int grp = et / C::GS, gt = et % C::GS;
         int64_t nvq[QB];
@@ -333,10 +336,10 @@ __global__ void __launch_bounds__(Cfg<QB>::kThreads, 1) index_tc_kernel(
                 float v[32];
                 float s = 0.f;
 #pragma unroll
-                for (int hc = 0; hc < 2; ++hc) {
-                    tmem_ld32(trow + (uint32_t)(q * 64 + hc * 32), v);
+                for (int hc = 0; hc < C::CPT / 32; ++hc) {
+                    tmem_ld32(trow + (uint32_t)(q * 64 + cb + hc * 32), v);
                     tmem_ld_wait();
-                    const float4 *wq = reinterpret_cast<const float4 *>(w_s + q * 64 + hc * 32);
+                    const float4 *wq = reinterpret_cast<const float4 *>(w_s + q * 64 + cb + hc * 32);
 #pragma unroll
                     for (int h4 = 0; h4 < 8; ++h4) {
                         const float4 ww = wq[h4];
@@ -351,9 +354,18 @@ __global__ void __launch_bounds__(Cfg<QB>::kThreads, 1) index_tc_kernel(
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&ms.tempty[acc]);
+            if (QB == 1) {
+                // QB=1: warps e and e+4 hold the two halves of the head sum of the same rows
+                float *part = reinterpret_cast<float *>(hist_all);   // 128 floats, free here
+                if (e >= 4) part[row] = sc[0];
+                named_sync(1, C::NE * 32);
+                if (e < 4) sc[0] += part[row];
+                named_sync(1, C::NE * 32);
+            }
 #pragma unroll
             for (int qq = 0; qq < C::QPT; ++qq) {
                 const int q = qa + qq;
+                if (QB == 1 && e >= 4) break;
                 if (j < nvq[q]) {
                     const unsigned long long c = ((unsigned long long)order_key(sc[qq]) << 32) |
                                                  (unsigned long long)(0xFFFFFFFFu - (uint32_t)j);

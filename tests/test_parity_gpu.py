@@ -128,15 +128,15 @@ def test_attend_stagewise_parity(spec):
 
 
 def test_tensor_core_path_selected():
-    """The V4-Flash prefill shapes take the tensor-core attention (it needs a workspace
-    for the rotated keys); decode-like and odd shapes take the general path."""
+    """The V4-Flash head shape takes the tensor-core attention, which needs a workspace
+    (rotated keys for prefill, packed keys for decode-sized calls); other shapes take the
+    general path."""
     import sparse_attention_14_b200 as csa
     for spec in MID + cs.WORKLOADS[1] + cs.WORKLOADS[2] + cs.WORKLOADS[3]:
         ws = csa.csa_attend_workspace_bytes(0 if spec.kind == "csa" else 1, spec.B, spec.S_q,
                                             spec.S_kv, spec.P, spec.H, spec.D, spec.topk,
                                             spec.torch_dtype)
-        tc = spec.dtype == "bf16" and spec.H == 64 and spec.D == 512 and \
-            spec.S_q * 64 >= spec.S_kv + spec.P
+        tc = spec.dtype == "bf16" and spec.H == 64 and spec.D == 512 and spec.R <= 64
         assert (ws > 0) == tc, spec.name
 
 
