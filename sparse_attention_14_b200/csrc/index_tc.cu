@@ -48,6 +48,7 @@ struct Misc {
     unsigned long long thr[4];
     unsigned long long sel_prefix[4];
     unsigned sel_remaining[4];
+    int sel_done[4];
     unsigned warp_part[4][8];
     int abort_;
 };
@@ -89,32 +90,47 @@ __device__ __forceinline__ float key_to_float(uint32_t key) {
 }
 
 // ------------------------------------------------------------------ group selection
-// All GS threads of a group (named barrier `bar`) find the k-th largest of n unique
-// 64-bit keys by an MSB-first radix select, 8 bits per pass.
+// All GS threads of a group (named barrier `bar`) find a threshold T such that exactly k
+// of n unique 64-bit keys are >= T, by an MSB-first radix select, 8 bits per pass.  The
+// histogram is built with warp-aggregated atomics (lanes with the same bin add once), and
+// the select stops at the first pass whose chosen bin is taken whole: T is then that
+// bin's prefix with the lower bits zero.
 template <int GS>
 __device__ unsigned long long group_kth(const unsigned long long *a, int n, int k, int gt, int bar,
                                         unsigned *hist, Misc &ms, int g) {
-    constexpr int BPT = 256 / GS;
+    constexpr int BPT = 256 / GS > 0 ? 256 / GS : 1;
     const int lane = gt & 31, wid = gt >> 5;
     if (gt == 0) {
         ms.sel_prefix[g] = 0ull;
         ms.sel_remaining[g] = (unsigned)k;
+        ms.sel_done[g] = 0;
     }
     for (int shift = 56; shift >= 0; shift -= 8) {
         for (int i = gt; i < 256; i += GS) hist[i] = 0u;
         named_sync(bar, GS);
+        if (ms.sel_done[g]) break;   // uniform: written before the previous barrier
         const unsigned long long prefix = ms.sel_prefix[g];
         const unsigned remaining = ms.sel_remaining[g];
         const unsigned long long mask = shift == 56 ? 0ull : (~0ull << (shift + 8));
-        for (int e = gt; e < n; e += GS) {
-            const unsigned long long key = a[e];
-            if ((key & mask) == prefix) atomicAdd(&hist[(unsigned)(key >> shift) & 255u], 1u);
+        for (int e0 = 0; e0 < n; e0 += GS) {
+            const int e = e0 + gt;
+            unsigned long long key = 0ull;
+            bool m = false;
+            if (e < n) {
+                key = a[e];
+                m = (key & mask) == prefix;
+            }
+            const unsigned bin = (unsigned)(key >> shift) & 255u;
+            const unsigned peers = __match_any_sync(0xFFFFFFFFu, m ? bin : 0xFFFFFFFFu);
+            if (m && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (unsigned)__popc(peers));
         }
         named_sync(bar, GS);
         const int hi_bin = 256 - gt * BPT;   // my bins: [hi_bin - BPT, hi_bin)
         unsigned local = 0;
+        if (gt * BPT < 256) {
 #pragma unroll
-        for (int b = 1; b <= BPT; ++b) local += hist[hi_bin - b];
+            for (int bb = 1; bb <= BPT; ++bb) local += hist[hi_bin - bb];
+        }
         unsigned incl = local;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -125,15 +141,18 @@ __device__ unsigned long long group_kth(const unsigned long long *a, int n, int 
         named_sync(bar, GS);
         unsigned cum = incl - local;
         for (int w = 0; w < wid; ++w) cum += ms.warp_part[g][w];
+        if (gt * BPT < 256) {
 #pragma unroll
-        for (int b = 1; b <= BPT; ++b) {
-            const int bin = hi_bin - b;
-            const unsigned h = hist[bin];
-            if (cum < remaining && remaining <= cum + h) {
-                ms.sel_prefix[g] = prefix | ((unsigned long long)bin << shift);
-                ms.sel_remaining[g] = remaining - cum;
+            for (int bb = 1; bb <= BPT; ++bb) {
+                const int bin = hi_bin - bb;
+                const unsigned h = hist[bin];
+                if (cum < remaining && remaining <= cum + h) {
+                    ms.sel_prefix[g] = prefix | ((unsigned long long)bin << shift);
+                    ms.sel_remaining[g] = remaining - cum;
+                    if (remaining - cum == h) ms.sel_done[g] = 1;
+                }
+                cum += h;
             }
-            cum += h;
         }
         named_sync(bar, GS);
     }
@@ -201,6 +220,53 @@ __device__ void group_emit(unsigned long long *cand, int n, int k, int gt, int b
             idx_row[r] = -1;
             if (score_row) score_row[r] = __int_as_float(0x7fc00000);
         }
+    }
+}
+
+// Write n survivor keys (n <= k) as idx / scores in ascending entry order using a bitmap
+// over [0, nv): set a bit per survivor, count bits per thread range, scan, and let each
+// survivor compute its own output slot.  bitmap holds ceil(nv/32) words; base >= GS ints.
+template <int GS>
+__device__ void group_emit_bitmap(const unsigned long long *cand, int n, int k, int64_t nv, int gt, int bar,
+                                  unsigned *bitmap, unsigned *base, Misc &ms, int g, int32_t *idx_row,
+                                  float *score_row) {
+    const int nwords = (int)((nv + 31) >> 5);
+    const int wpt = (nwords + GS - 1) / GS;
+    const int lane = gt & 31, wid = gt >> 5;
+    for (int w = gt; w < nwords; w += GS) bitmap[w] = 0u;
+    named_sync(bar, GS);
+    for (int e = gt; e < n; e += GS) {
+        const uint32_t j = 0xFFFFFFFFu - (uint32_t)cand[e];
+        atomicOr(&bitmap[j >> 5], 1u << (j & 31));
+    }
+    named_sync(bar, GS);
+    unsigned local = 0;
+    for (int w = gt * wpt; w < (gt + 1) * wpt && w < nwords; ++w) local += __popc(bitmap[w]);
+    unsigned incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        unsigned v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) ms.warp_part[g][wid] = incl;
+    named_sync(bar, GS);
+    unsigned pre = incl - local;
+    for (int w = 0; w < wid; ++w) pre += ms.warp_part[g][w];
+    base[gt] = pre;
+    named_sync(bar, GS);
+    for (int e = gt; e < n; e += GS) {
+        const unsigned long long c = cand[e];
+        const uint32_t j = 0xFFFFFFFFu - (uint32_t)c;
+        const int w = (int)(j >> 5), o = w / wpt;
+        unsigned pos = base[o];
+        for (int w2 = o * wpt; w2 < w; ++w2) pos += __popc(bitmap[w2]);
+        pos += __popc(bitmap[w] & ((1u << (j & 31)) - 1u));
+        idx_row[pos] = (int32_t)j;
+        if (score_row) score_row[pos] = key_to_float((uint32_t)(c >> 32));
+    }
+    for (int r = n + gt; r < k; r += GS) {
+        idx_row[r] = -1;
+        if (score_row) score_row[r] = __int_as_float(0x7fc00000);
     }
 }
 
@@ -392,7 +458,12 @@ __global__ void __launch_bounds__(Cfg<QB>::kThreads, Cfg<QB>::kMinBlocks) index_
             group_cut<C::GS>(cand, topk, gt, 2 + q, hist_all + q * 256, ms, q, q);
             const int n = (int)ms.cnt[q];
             const int64_t qrow = b * S_q + i0 + q;
-            if (n_split == 1) {
+            if (n_split == 1 && topk <= kCap / 2 && nvq[q] <= (int64_t)kCap / 2 * 64) {
+                // survivors occupy the lower half of the buffer, the bitmap the upper half
+                group_emit_bitmap<C::GS>(cand, n, topk, nvq[q], gt, 2 + q,
+                                         reinterpret_cast<unsigned *>(cand + kCap / 2), hist_all + q * 256, ms, q,
+                                         idx + qrow * topk, scores_opt ? scores_opt + qrow * topk : nullptr);
+            } else if (n_split == 1) {
                 group_emit<C::GS>(cand, n, topk, gt, 2 + q, idx + qrow * topk,
                                   scores_opt ? scores_opt + qrow * topk : nullptr);
             } else {
