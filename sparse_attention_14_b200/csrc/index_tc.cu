@@ -38,7 +38,7 @@ namespace {
 
 using namespace umma;
 
-constexpr int kDI = 128, kHI = 64, kTileE = 128, kCap = 1024;
+constexpr int kDI = 128, kHI = 64, kTileE = 128, kCap = 2048;
 constexpr int kMaxTopk = kCap - kTileE;   // room for one tile after a cut to k
 
 struct Misc {
@@ -58,7 +58,7 @@ struct Cfg {
     static constexpr int N = QB * 64;
     static constexpr int NE = 8;                         // epilogue warps (two per TMEM lane group)
     static constexpr int kThreads = (2 + NE) * 32;
-    static constexpr int NST = QB == 4 ? 3 : 2;          // entry-tile stages (QB=1: two CTAs per SM)
+    static constexpr int NST = 2;                        // entry-tile stages
     static constexpr int kMinBlocks = QB == 4 ? 1 : 2;
     static constexpr uint32_t kBChunk = QB * 64 * 128;   // one 64-column chunk of q_I rows
     static constexpr uint32_t kBBytes = 2 * kBChunk;
@@ -159,29 +159,37 @@ __device__ unsigned long long group_kth(const unsigned long long *a, int n, int 
     return ms.sel_prefix[g];
 }
 
-// Cut a query's candidate buffer back to its k largest keys (keys >= the k-th).
+// Cut a query's candidate buffer back to its k largest keys (keys >= the k-th).  The
+// survivors are compacted to the front in chunks of 8 keys per thread: a chunk is read
+// into registers before any of it is overwritten, and survivors never pass the read point.
 template <int GS>
 __device__ void group_cut(unsigned long long *cand, int k, int gt, int bar, unsigned *hist, Misc &ms,
                           int g, int q) {
-    constexpr int EPT = kCap / GS;
     const int n = (int)ms.cnt[q];
     if (n <= k) return;   // uniform within the group
     const unsigned long long T = group_kth<GS>(cand, n, k, gt, bar, hist, ms, g);
-    unsigned long long mine[EPT];
-#pragma unroll
-    for (int i = 0; i < EPT; ++i) {
-        const int e = gt + i * GS;
-        mine[i] = e < n ? cand[e] : 0ull;
-    }
+    const int lane = gt & 31;
     named_sync(bar, GS);
     if (gt == 0) ms.cnt[q] = 0;
     named_sync(bar, GS);
+    for (int c0 = 0; c0 < n; c0 += 8 * GS) {
+        unsigned long long mine[8];
 #pragma unroll
-    for (int i = 0; i < EPT; ++i) {
-        if (mine[i] != 0ull && mine[i] >= T) {
-            const unsigned pos = atomicAdd(&ms.cnt[q], 1u);
-            cand[pos] = mine[i];
+        for (int i = 0; i < 8; ++i) {
+            const int e = c0 + gt + i * GS;
+            mine[i] = e < n ? cand[e] : 0ull;
         }
+        named_sync(bar, GS);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const bool keep = mine[i] != 0ull && mine[i] >= T;
+            const unsigned ball = __ballot_sync(0xFFFFFFFFu, keep);
+            unsigned base = 0;
+            if (lane == 0 && ball) base = atomicAdd(&ms.cnt[q], (unsigned)__popc(ball));
+            base = __shfl_sync(0xFFFFFFFFu, base, 0);
+            if (keep) cand[base + __popc(ball & ((1u << lane) - 1u))] = mine[i];
+        }
+        named_sync(bar, GS);
     }
     if (gt == 0) ms.thr[q] = T;
     named_sync(bar, GS);
@@ -428,17 +436,19 @@ __global__ void __launch_bounds__(Cfg<QB>::kThreads, Cfg<QB>::kMinBlocks) index_
                 if (e < 4) sc[0] += part[row];
                 named_sync(1, C::NE * 32);
             }
+            if (!(QB == 1 && e >= 4)) {
 #pragma unroll
-            for (int qq = 0; qq < C::QPT; ++qq) {
-                const int q = qa + qq;
-                if (QB == 1 && e >= 4) break;
-                if (j < nvq[q]) {
+                for (int qq = 0; qq < C::QPT; ++qq) {
+                    const int q = qa + qq;
                     const unsigned long long c = ((unsigned long long)order_key(sc[qq]) << 32) |
                                                  (unsigned long long)(0xFFFFFFFFu - (uint32_t)j);
-                    if (c > ms.thr[q]) {
-                        const unsigned pos = atomicAdd(&ms.cnt[q], 1u);
-                        cand_all[q * kCap + pos] = c;
-                    }
+                    const bool ins = j < nvq[q] && c > ms.thr[q];
+                    // one counter update per warp: reserve the warp's slots, then scatter
+                    const unsigned ball = __ballot_sync(0xFFFFFFFFu, ins);
+                    unsigned base = 0;
+                    if (lane == 0 && ball) base = atomicAdd(&ms.cnt[q], (unsigned)__popc(ball));
+                    base = __shfl_sync(0xFFFFFFFFu, base, 0);
+                    if (ins) cand_all[q * kCap + base + __popc(ball & ((1u << lane) - 1u))] = c;
                 }
             }
             named_sync(1, C::NE * 32);
