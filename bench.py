@@ -143,8 +143,19 @@ def workload_specs(workload: int):
 
 
 def rank_spec(spec, rank):
-    # each rank: its own independent sequence (seeded per rank)
+    """Rank r runs its own independent layer instance: same shape, its own seeded inputs."""
     return dataclasses.replace(spec, workload=spec.workload + 10 * rank) if rank else spec
+
+
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """Device time of the slowest rank (one all-reduce of a scalar; no data-path traffic)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 class LayerRunner:
@@ -276,11 +287,7 @@ def gpu_arm(args, rank, world, local_rank):
         dist.barrier()
     clocks = clk.stop()
     launches = csa.launch_count() - launches0
-    ms_total = t0.elapsed_time(t1)
-    if world > 1:
-        tt = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total = float(tt.item())
+    ms_total = max_over_ranks(t0.elapsed_time(t1), world, dev)
     ms_step = ms_total / args.steps
     stage_ms = {"%d:%s" % key: sum(a.elapsed_time(b) for a, b in ev[key]) / args.steps
                 for key in stage_names}
@@ -392,11 +399,7 @@ def e2e_arm(args, runners, stage_names, stream, world, dev):
         one()
     b.record(stream)
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / steps
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(a.elapsed_time(b) / steps, world, dev)
     tokens = runners[0].spec.B * runners[0].spec.S_q * world
     return {"value": round(tokens / (ms * 1e-3), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3),
@@ -434,7 +437,7 @@ def oracle_rows(spec, n):
     # evenly spaced query rows: the same causal mix of window/entry counts as the workload
     S = spec.S_q
     n = min(n, S)
-    return sorted({int(round(x)) for x in [(k + 0.5) * S / n for k in range(n)]})
+    return sorted({min(S - 1, int((k + 0.5) * S / n)) for k in range(n)})
 
 
 def oracle_threads():
