@@ -253,16 +253,44 @@ def gpu_arm(args, rank, world, local_rank):
     tokens_per_step = sum(s.B * s.S_q for s in specs[:1])  # the block processes S tokens once
     stage_names = [(li, st) for li, r in enumerate(runners) for st in r.stages()]
 
-    def step(events=None):
-        for li, st in stage_names:
-            if events is not None:
-                events[(li, st)][0].record(stream)
-            runners[li].run_stage(st)
-            if events is not None:
-                events[(li, st)][1].record(stream)
-
     for _ in range(args.warmup):
-        step()
+        for li, st in stage_names:
+            runners[li].run_stage(st)
+    torch.cuda.synchronize()
+
+    # each stage captured once into a CUDA graph (the library only enqueues work on the
+    # current stream, so a call is capturable); the timed steps replay the graphs with CUDA
+    # events between them, which removes host launch overhead from the measurement
+    graphs = None
+    launches_per_step = None
+    if not args.eager:
+        try:
+            l0 = csa.launch_count()
+            graphs = {}
+            for key in stage_names:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    runners[key[0]].run_stage(key[1])
+                graphs[key] = g
+            launches_per_step = csa.launch_count() - l0
+            torch.cuda.synchronize()
+        except Exception as exc:  # pragma: no cover - falls back to eager launches
+            print("graph capture failed (%s); timing eager launches" % exc, file=sys.stderr)
+            graphs = None
+            torch.cuda.synchronize()
+
+    def step(events=None):
+        for key in stage_names:
+            if events is not None:
+                events[key][0].record(stream)
+            if graphs is not None:
+                graphs[key].replay()
+            else:
+                runners[key[0]].run_stage(key[1])
+            if events is not None:
+                events[key][1].record(stream)
+
+    step()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -287,6 +315,8 @@ def gpu_arm(args, rank, world, local_rank):
         dist.barrier()
     clocks = clk.stop()
     launches = csa.launch_count() - launches0
+    if graphs is not None:
+        launches = launches_per_step * args.steps
     ms_total = max_over_ranks(t0.elapsed_time(t1), world, dev)
     ms_step = ms_total / args.steps
     stage_ms = {"%d:%s" % key: sum(a.elapsed_time(b) for a, b in ev[key]) / args.steps
@@ -344,7 +374,8 @@ def gpu_arm(args, rank, world, local_rank):
                    "layers": [s.kind for s in specs], "m": [s.m for s in specs],
                    "P": [s.P for s in specs], "topk": spec0.topk, "H_I": spec0.H_I,
                    "d_I": spec0.d_I, "parallelism": "independent layer instance per GPU",
-                   "l2": "inputs larger than L2 (q/out/q_I > 126 MB per step); no flush"},
+                   "l2": "inputs larger than L2 (q/out/q_I > 126 MB per step); no flush",
+                   "launch": "CUDA graph per stage" if graphs is not None else "eager"},
         "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
         "roofline": roof,
         "gpu_launches": int(launches),
@@ -503,6 +534,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="time eager launches instead of CUDA graphs")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

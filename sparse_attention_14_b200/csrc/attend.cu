@@ -199,7 +199,7 @@ csa_status_t launch_simt_n(const AttendArgs &a, cudaStream_t st) {
     CSA_REQUIRE(smem <= 227 * 1024, CSA_ERR_UNSUPPORTED, "attend: D=%d too large", a.D);
     CSA_REQUIRE(a.S_q < (1ll << 31) && a.B < 65536, CSA_ERR_UNSUPPORTED, "attend: grid too large");
     auto kern = attend_simt_kernel<T, NACC>;
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    ensure_smem((const void *)kern, smem);
     dim3 grid((unsigned)a.S_q, (unsigned)a.B, (unsigned)ceil_div(a.H, kHG));
     kern<<<grid, kThreads, smem, st>>>(
         (const T *)a.q, (const T *)a.kv, a.S_kv, a.kv_pos0, (const T *)a.pool, a.P, a.idx, a.topk,

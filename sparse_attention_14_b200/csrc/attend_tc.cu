@@ -154,12 +154,14 @@ __global__ void __launch_bounds__(32) pack_list_kernel(const int32_t *__restrict
     if (lane == 0) n_keys[qi] = nk;
 }
 
-constexpr int kPackRows = 16;
-__global__ void __launch_bounds__(128) pack_rows_kernel(
+constexpr int kPackRows = 64;
+__global__ void __launch_bounds__(256) pack_rows_kernel(
     const __nv_bfloat16 *__restrict__ kv, int64_t S_kv, int64_t kv_pos0, const __nv_bfloat16 *__restrict__ pool,
     int64_t P, int mode, int64_t S_q, int64_t q_pos0, int window, int ratio, RopeTable rope,
     const int32_t *__restrict__ ent_ws, const int32_t *__restrict__ n_keys, __nv_bfloat16 *__restrict__ packed,
     int kmax) {
+    __shared__ const __nv_bfloat16 *row_src[kPackRows];
+    __shared__ double row_pos[kPackRows];
     const int64_t qi = blockIdx.x;
     const int x0 = blockIdx.y * kPackRows;
     const int nk = n_keys[qi];
@@ -169,47 +171,56 @@ __global__ void __launch_bounds__(128) pack_rows_kernel(
     if (lo < kv_pos0) lo = kv_pos0;
     const int64_t hi = t < kv_pos0 + S_kv - 1 ? t : kv_pos0 + S_kv - 1;
     const int n_win = hi >= lo ? (int)(hi - lo + 1) : 0;
-    constexpr int kPieces = kD / 8;
-    constexpr int kPer = kPackRows * kPieces / 128;       // 8 pieces per thread
-    float e[kPer][8];
-    double pos[kPer];
-#pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-        const int v = threadIdx.x + u * 128;
-        const int x = x0 + v / kPieces, pc = v % kPieces;
-        if (x < nk) {
-            const __nv_bfloat16 *src;
-            if (x < n_win) {
-                src = kv + (b * S_kv + (lo - kv_pos0) + x) * kD;
-                pos[u] = (double)(lo + x);
-            } else {
-                const int64_t j = mode == 0 ? (int64_t)ent_ws[qi * (int64_t)kmax + (x - n_win)] : (int64_t)(x - n_win);
-                src = pool + (b * P + j) * kD;
-                pos[u] = (double)j * (double)ratio;
-            }
-            load8(src + pc * 8, e[u]);
+    const int rows = nk - x0 < kPackRows ? nk - x0 : kPackRows;
+    // resolve this slice's source rows once
+    if (threadIdx.x < rows) {
+        const int x = x0 + threadIdx.x;
+        if (x < n_win) {
+            row_src[threadIdx.x] = kv + (b * S_kv + (lo - kv_pos0) + x) * kD;
+            row_pos[threadIdx.x] = (double)(lo + x);
+        } else {
+            const int64_t j = mode == 0 ? (int64_t)ent_ws[qi * (int64_t)kmax + (x - n_win)] : (int64_t)(x - n_win);
+            row_src[threadIdx.x] = pool + (b * P + j) * kD;
+            row_pos[threadIdx.x] = (double)j * (double)ratio;
         }
     }
+    __syncthreads();
+    constexpr int kPieces = kD / 8;                       // 64 pieces of 16 bytes per row
+    const int rope_p0 = rope.first / 8;                   // first piece holding rope channels
+    // un-rotated pieces: raw 16-byte copies, eight in flight per thread
+    const int plain = rows * rope_p0;
+    for (int v0 = 0; v0 < plain; v0 += 8 * 256) {
+        uint4 w[8];
 #pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-        const int v = threadIdx.x + u * 128;
-        const int x = x0 + v / kPieces, pc = v % kPieces;
-        if (x >= nk) continue;
-        const int d0 = pc * 8;
-        if (d0 + 8 > rope.first) {
+        for (int u = 0; u < 8; ++u) {
+            const int v = v0 + u * 256 + threadIdx.x;
+            if (v < plain) w[u] = *reinterpret_cast<const uint4 *>(row_src[v / rope_p0] + (v % rope_p0) * 8);
+        }
 #pragma unroll
-            for (int c = 0; c < 8; c += 2) {
-                const int d = d0 + c;
-                if (d >= rope.first) {
-                    float cs, sn;
-                    rope_cs(pos[u], rope.inv_freq[(d - rope.first) >> 1], &cs, &sn);
-                    const float a0 = e[u][c], a1 = e[u][c + 1];
-                    e[u][c] = a0 * cs - a1 * sn;
-                    e[u][c + 1] = a0 * sn + a1 * cs;
-                }
+        for (int u = 0; u < 8; ++u) {
+            const int v = v0 + u * 256 + threadIdx.x;
+            if (v < plain)
+                *reinterpret_cast<uint4 *>(packed + (qi * kmax + x0 + v / rope_p0) * kD + (v % rope_p0) * 8) = w[u];
+        }
+    }
+    // rope pieces: every lane rotates whole pieces (no divergence around the angle math)
+    const int rp = kPieces - rope_p0;
+    for (int v = threadIdx.x; v < rows * rp; v += 256) {
+        const int xr = v / rp, pc = rope_p0 + v % rp;
+        float e[8];
+        load8(row_src[xr] + pc * 8, e);
+#pragma unroll
+        for (int c = 0; c < 8; c += 2) {
+            const int d = pc * 8 + c;
+            if (d >= rope.first) {
+                float cs, sn;
+                rope_cs(row_pos[xr], rope.inv_freq[(d - rope.first) >> 1], &cs, &sn);
+                const float a0 = e[c], a1 = e[c + 1];
+                e[c] = a0 * cs - a1 * sn;
+                e[c + 1] = a0 * sn + a1 * cs;
             }
         }
-        store8(packed + (qi * kmax + x) * kD + pc * 8, e[u]);
+        store8(packed + (qi * kmax + x0 + xr) * kD + pc * 8, e);
     }
 }
 
@@ -756,7 +767,7 @@ csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st) {
                                                                  kmax, ent_ws, n_keys);
         CSA_CHECK_LAUNCH("attend: list keys");
         dim3 pg((unsigned)(a.B * a.S_q), (unsigned)ceil_div(kmax, kPackRows));
-        pack_rows_kernel<<<pg, 128, 0, st>>>((const __nv_bfloat16 *)a.kv, a.S_kv, a.kv_pos0,
+        pack_rows_kernel<<<pg, 256, 0, st>>>((const __nv_bfloat16 *)a.kv, a.S_kv, a.kv_pos0,
                                             (const __nv_bfloat16 *)a.pool, a.P, a.mode, a.S_q, a.q_pos0, a.window,
                                             a.ratio, a.rope, ent_ws, n_keys, kv_rot, kmax);
         CSA_CHECK_LAUNCH("attend: pack keys");
@@ -782,10 +793,8 @@ csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st) {
                 CSA_ERR_CUDA, "attend: cannot encode the TMA tensor maps");
     const size_t smem = tc_smem_bytes(a.mode == 0 && !packed ? a.topk : 1);
     CSA_REQUIRE(smem <= 232448, CSA_ERR_UNSUPPORTED, "attend: shared memory %zu B too large", smem);
-    cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    ensure_smem((const void *)attend_tc_kernel, smem);
+    const int sms = device_sm_count();
     const int64_t nq = a.B * a.S_q;
     const int grid = (int)(nq < sms ? nq : sms);
     attend_tc_kernel<<<grid, kThreads, smem, st>>>(

@@ -47,6 +47,48 @@ bool encode_map_bf16_2d(CUtensorMap *map, const void *ptr, uint64_t cols, uint64
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+namespace {
+constexpr int kMaxDev = 64;
+std::mutex g_dev_mu;
+int g_sm_count[kMaxDev];
+struct SmemEntry {
+    const void *fn;
+    int dev;
+    size_t bytes;
+};
+SmemEntry g_smem[256];
+int g_n_smem = 0;
+}  // namespace
+
+int device_sm_count() {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= kMaxDev) return 148;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (g_sm_count[dev] == 0) {
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) sms = 148;
+        g_sm_count[dev] = sms;
+    }
+    return g_sm_count[dev];
+}
+
+void ensure_smem(const void *kernel, size_t bytes) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    for (int i = 0; i < g_n_smem; ++i) {
+        if (g_smem[i].fn == kernel && g_smem[i].dev == dev) {
+            if (g_smem[i].bytes >= bytes) return;
+            cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+            g_smem[i].bytes = bytes;
+            return;
+        }
+    }
+    cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (g_n_smem < 256) g_smem[g_n_smem++] = SmemEntry{kernel, dev, bytes};
+}
+
 void make_rope_table(RopeTable *t, int D, int R, double base) {
     memset(t, 0, sizeof(*t));
     t->n_pairs = R / 2;

@@ -108,6 +108,13 @@ __device__ __forceinline__ void rope_cs(double pos, double inv_freq, float *c, f
 bool encode_map_bf16_2d(CUtensorMap *map, const void *ptr, uint64_t cols, uint64_t rows,
                         uint32_t box_cols, uint32_t box_rows);
 
+// ---------------------------------------------------------------- per-device launch state
+// SM count of the current device, looked up once per device.
+int device_sm_count();
+// Raise a kernel's dynamic shared-memory limit to at least `bytes` (once per kernel, device
+// and size; the attribute call is skipped when it is already high enough).
+void ensure_smem(const void *kernel, size_t bytes);
+
 // ---------------------------------------------------------------- misc
 __host__ __device__ __forceinline__ int64_t n_visible(int64_t t, int64_t ratio, int64_t P) {
     if (t < 0) return 0;

@@ -492,7 +492,7 @@ __global__ void __launch_bounds__(Cfg<QB>::kThreads, Cfg<QB>::kMinBlocks) index_
 constexpr int kMergeThreads = 256;
 __global__ void __launch_bounds__(kMergeThreads) index_merge_kernel(
     const unsigned long long *__restrict__ partial, int n_split, int topk, int32_t *__restrict__ idx,
-    float *__restrict__ scores_opt) {
+    float *__restrict__ scores_opt, int64_t S_q, int64_t q_pos0, int ratio, int64_t P) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int total = n_split * topk;
     const int cap = pow2_ceil(total);
@@ -500,7 +500,9 @@ __global__ void __launch_bounds__(kMergeThreads) index_merge_kernel(
     unsigned long long *keep = cand + cap;                   // pow2_ceil(topk) slots
     unsigned *hist = reinterpret_cast<unsigned *>(keep + pow2_ceil(topk));
     Misc &ms = *reinterpret_cast<Misc *>(hist + 256);
+    unsigned *bitmap = reinterpret_cast<unsigned *>(&ms + 1);  // ceil(P/32) words
     const int64_t row = blockIdx.x;
+    const int64_t nv = n_visible(q_pos0 + row % S_q, ratio, P);
     const int tid = threadIdx.x;
     if (tid == 0) {
         ms.cnt[0] = 0;
@@ -524,8 +526,8 @@ __global__ void __launch_bounds__(kMergeThreads) index_merge_kernel(
         n = (int)ms.cnt[1];
         src = keep;
     }
-    group_emit<kMergeThreads>(src, n, topk, tid, 1, idx + row * topk,
-                              scores_opt ? scores_opt + row * topk : nullptr);
+    group_emit_bitmap<kMergeThreads>(src, n, topk, nv, tid, 1, bitmap, hist, ms, 0, idx + row * topk,
+                                     scores_opt ? scores_opt + row * topk : nullptr);
 }
 
 // ------------------------------------------------------------------ host side
@@ -534,10 +536,7 @@ bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint32_t box_rows)
 }
 
 int sm_count() {
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    return sms;
+    return device_sm_count();
 }
 
 struct Plan {
@@ -550,9 +549,11 @@ Plan plan(int64_t B, int64_t S_q, int64_t q_pos0, int64_t P, int ratio, int topk
     p.qb = S_q >= 4 ? 4 : 1;
     const int64_t n_qb = B * ((S_q + p.qb - 1) / p.qb);
     const int64_t tiles = (n_visible(q_pos0 + S_q - 1, ratio, P) + kTileE - 1) / kTileE;
+    // decode-sized calls: split each query's entry range so that all CTAs run in one wave
+    // (the single-query kernel fits two CTAs per SM)
     const int64_t want = 2 * (int64_t)sm_count();
     int64_t ns = 1;
-    if (n_qb < want && tiles >= 8) ns = (want + n_qb - 1) / n_qb;
+    if (n_qb < want && tiles >= 8) ns = want / n_qb > 1 ? want / n_qb : 2;
     if (ns > tiles / 4) ns = tiles / 4 > 0 ? tiles / 4 : 1;
     if (ns > 16) ns = 16;
     while (ns > 1 && (int64_t)pow2_ceil((int)(ns * topk)) > 8192) --ns;
@@ -569,7 +570,7 @@ csa_status_t launch(const CUtensorMap &mk, const CUtensorMap &mq, const __nv_bfl
     const int64_t grid = n_qb * n_split;
     CSA_REQUIRE(grid < (1ll << 31), CSA_ERR_UNSUPPORTED, "csa_index_topk: grid too large");
     auto kern = index_tc_kernel<QB>;
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
+    ensure_smem((const void *)kern, C::kSmem);
     kern<<<(unsigned)grid, C::kThreads, C::kSmem, st>>>(mk, mq, w, B, S_q, q_pos0, P, ratio, topk, n_split,
                                                         idx, scores_opt, partial);
     CSA_CHECK_LAUNCH("csa_index_topk");
@@ -615,10 +616,12 @@ csa_status_t index_tc(const void *qI, const void *w, const void *kI, int64_t B, 
         r = launch<1>(mk, mq, wb, B, S_q, q_pos0, P, ratio, topk, p.n_split, idx, scores_opt, partial, st);
     if (r != CSA_OK || p.n_split <= 1) return r;
     const int total = p.n_split * topk;
-    const size_t smem = (size_t)(pow2_ceil(total) + pow2_ceil(topk)) * 8 + 256 * 4 + sizeof(Misc);
+    const size_t smem = (size_t)(pow2_ceil(total) + pow2_ceil(topk)) * 8 + 256 * 4 + sizeof(Misc) +
+                        (size_t)((P + 31) / 32) * 4;
     CSA_REQUIRE(smem <= 227 * 1024, CSA_ERR_UNSUPPORTED, "csa_index_topk: merge too large");
-    cudaFuncSetAttribute(index_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    index_merge_kernel<<<(unsigned)(B * S_q), kMergeThreads, smem, st>>>(partial, p.n_split, topk, idx, scores_opt);
+    ensure_smem((const void *)index_merge_kernel, smem);
+    index_merge_kernel<<<(unsigned)(B * S_q), kMergeThreads, smem, st>>>(partial, p.n_split, topk, idx, scores_opt,
+                                                                         S_q, q_pos0, ratio, P);
     CSA_CHECK_LAUNCH("csa_index_topk merge");
     return CSA_OK;
 }

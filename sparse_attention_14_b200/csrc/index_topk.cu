@@ -98,7 +98,7 @@ csa_status_t launch_simt(const T *qI, const T *w, const T *kI, int64_t B, int64_
                 "general path", (long long)P, H_I * d_I, smem);
     CSA_REQUIRE(S_q < (1ll << 31) && B < 65536, CSA_ERR_UNSUPPORTED, "csa_index_topk: grid too large");
     auto kern = index_topk_simt_kernel<T>;
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    ensure_smem((const void *)kern, smem);
     kern<<<dim3((unsigned)S_q, (unsigned)B), kIdxThreads, smem, st>>>(
         qI, w, kI, S_q, q_pos0, P, H_I, d_I, ratio, topk, idx, scores_opt);
     CSA_CHECK_LAUNCH("csa_index_topk");
