@@ -497,6 +497,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     } else if (warp == 1) {
         // ===================================================== MMA issuer
         if (lane == 0) {
+            // Loop-invariant descriptor words; per K-step only a constant is added to the
+            // low word (see mma_bf16_w).
+            const uint64_t d_kv = sdesc_sw128(s_kv, 16, 1024), d_q = sdesc_sw128(s_q, 16, 1024);
+            const uint64_t d_v = sdesc_sw128(s_kv, 16384, 1024), d_p = sdesc_sw128(s_p, 8192, 1024);
+            const uint32_t kv_lo = (uint32_t)d_kv, q_lo = (uint32_t)d_q, v_lo = (uint32_t)d_v, p_lo = (uint32_t)d_p;
+            const uint32_t hi = (uint32_t)(d_kv >> 32);   // SBO 1024, version, swizzle: shared
             uint32_t g = 0, qc = 0;
             bool ok = true;
             for (int64_t qi = blockIdx.x; ok && qi < nq; qi += gridDim.x, ++qc) {
@@ -510,16 +516,15 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 tc_fence_after();
                 for (int kt = 0; ok && kt < n_tiles; ++kt, ++g) {
                     // S^T = K . Qr^T, chunk by chunk as the tile lands
+#pragma unroll
                     for (int c = 0; c < 8; ++c) {
                         ok = mbar_wait(&sm.full[c], g & 1u, kWaitIter);
                         if (!ok) break;
 #pragma unroll
-                        for (int k4 = 0; k4 < 4; ++k4) {
-                            const int ks = c * 4 + k4;
-                            const uint64_t a = sdesc_sw128(s_kv + (uint32_t)c * 16384u + (uint32_t)k4 * 32u, 16, 1024);
-                            const uint64_t bq = sdesc_sw128(s_q + (uint32_t)c * 8192u + (uint32_t)k4 * 32u, 16, 1024);
-                            mma_bf16(tmem + kColS, a, bq, kIdescQK, ks > 0 ? 1u : 0u);
-                        }
+                        for (int k4 = 0; k4 < 4; ++k4)
+                            mma_bf16_w(tmem + kColS, kv_lo + (uint32_t)((c * 16384 + k4 * 32) >> 4), hi,
+                                       q_lo + (uint32_t)((c * 8192 + k4 * 32) >> 4), hi, kIdescQK,
+                                       (c | k4) ? 1u : 0u);
                     }
                     if (!ok) break;
                     mma_commit(&sm.s_full);
@@ -528,14 +533,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                     if (!ok) break;
                     tc_fence_after();
                     // O^T += V^T . P^T, releasing each pair of key chunks when done
+                    const uint32_t acc0 = kt > 0 ? 1u : 0u;
 #pragma unroll
                     for (int mt = 0; mt < 4; ++mt) {
 #pragma unroll
-                        for (int kk = 0; kk < kTile / 16; ++kk) {
-                            const uint64_t a = sdesc_sw128(s_kv + (uint32_t)(2 * mt) * 16384u + (uint32_t)kk * 2048u, 16384, 1024);
-                            const uint64_t bp = sdesc_sw128(s_p + (uint32_t)kk * 2048u, 8192, 1024);
-                            mma_bf16(tmem + kColO + mt * 64, a, bp, kIdescPV, (kt > 0 || kk > 0) ? 1u : 0u);
-                        }
+                        for (int kk = 0; kk < kTile / 16; ++kk)
+                            mma_bf16_w(tmem + kColO + mt * 64, v_lo + (uint32_t)((2 * mt * 16384 + kk * 2048) >> 4), hi,
+                                       p_lo + (uint32_t)((kk * 2048) >> 4), hi, kIdescPV, kk > 0 ? 1u : acc0);
                         mma_commit(&sm.free_[mt]);
                     }
                 }

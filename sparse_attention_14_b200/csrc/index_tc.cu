@@ -362,6 +362,9 @@ __global__ void __launch_bounds__(Cfg<QB>::kThreads, Cfg<QB>::kMinBlocks) index_
         // ---------------- MMA issuer
         if (lane == 0 && n_tiles > 0) {
             constexpr uint32_t idesc = idesc_bf16_f32(128, C::N, 0, 0);
+            // loop-invariant descriptor words (see mma_bf16_w)
+            const uint64_t d_a = sdesc_sw128(sA, 16, 1024), d_b = sdesc_sw128(sB, 16, 1024);
+            const uint32_t a_lo0 = (uint32_t)d_a, b_lo0 = (uint32_t)d_b, hi = (uint32_t)(d_a >> 32);
             bool ok = mbar_wait(&ms.bfull, 0);
             for (int it = 0; ok && it < n_tiles; ++it) {
                 const int s = it % C::NST, acc = it & 1;
@@ -369,13 +372,12 @@ __global__ void __launch_bounds__(Cfg<QB>::kThreads, Cfg<QB>::kMinBlocks) index_
                 if (ok && it >= 2) ok = mbar_wait(&ms.tempty[acc], (uint32_t)((it >> 1) - 1) & 1u);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t a0 = sA + (uint32_t)s * C::kABytes;
+                const uint32_t a_lo = a_lo0 + (uint32_t)s * (C::kABytes >> 4);
 #pragma unroll
-                for (int ks = 0; ks < kDI / 16; ++ks) {
-                    const uint64_t ad = sdesc_sw128(a0 + (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u, 16, 1024);
-                    const uint64_t bd = sdesc_sw128(sB + (uint32_t)(ks >> 2) * C::kBChunk + (uint32_t)(ks & 3) * 32u, 16, 1024);
-                    mma_bf16(tmem + (uint32_t)(acc * C::N), ad, bd, idesc, ks > 0 ? 1u : 0u);
-                }
+                for (int ks = 0; ks < kDI / 16; ++ks)
+                    mma_bf16_w(tmem + (uint32_t)(acc * C::N), a_lo + (uint32_t)(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4), hi,
+                               b_lo0 + (uint32_t)(((ks >> 2) * C::kBChunk + (ks & 3) * 32) >> 4), hi, idesc,
+                               ks > 0 ? 1u : 0u);
                 mma_commit(&ms.empty[s]);
                 mma_commit(&ms.tfull[acc]);
             }

@@ -46,6 +46,26 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_maj
 }
 
 // ------------------------------------------------------------------ MMA and TMEM
+// The same MMA with each descriptor passed as two 32-bit words.  Only the low word
+// (start address and LBO) changes between the K-steps of a tile, so an issue loop can
+// keep the high words and a base low word in registers and add a compile-time
+// (byte offset >> 4) per step: one integer add per operand, which keeps the single
+// issuing thread well ahead of the tensor pipe.  Valid while every start address stays
+// below 256 KB (the 14-bit field cannot carry into LBO), which shared memory guarantees.
+__device__ __forceinline__ void mma_bf16_w(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi,
+                                           uint32_t b_lo, uint32_t b_hi, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "mov.b64 da, {%1, %2};\n\t"
+        "mov.b64 db, {%3, %4};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}\n"
+        :
+        : "r"(d_tmem), "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                          uint32_t idesc, uint32_t accumulate) {
     asm volatile(
