@@ -63,12 +63,11 @@ struct Meta {
 struct Small {
     uint64_t full[8], free_[4], s_full, p_full, o_full, q_tma, q_full, q_free, meta_full[2];
     uint32_t tmem_base;
-    int flag;
     int abort_;
     Meta meta[2];
     int32_t rows[kTile];
     float qcs[2][32];
-    float m_used[kH];
+    alignas(16) float m_used[kH];
     float alpha[kH];
     float red[4][kH];
     float inv_l[kH];
@@ -242,6 +241,28 @@ __device__ __forceinline__ void warp_reduce32(float *v) {
     }
 }
 
+// Named barrier over `count` threads that also ORs a predicate across them.
+__device__ __forceinline__ bool named_sync_any(uint32_t id, uint32_t count, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\t"
+        "setp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.or.pred po, %2, %3, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}\n"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
+}
+
+// 2^x by the hardware approximation (relative error about 2^-22, flushes subnormal
+// results to zero): P is rounded to bf16 right after, so this is exact enough.
+__device__ __forceinline__ float ex2_fast(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
@@ -308,7 +329,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         mbar_init(&sm.meta_full[0], 1);
         mbar_init(&sm.meta_full[1], 1);
         fence_mbar_init();
-        sm.flag = 0;
         sm.abort_ = 0;
     }
     if (warp == 1) tmem_alloc(&sm.tmem_base, 512);
@@ -577,6 +597,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             float l_part[32];
 #pragma unroll
             for (int h = 0; h < 32; ++h) l_part[h] = 0.f;
+            // the running maxima of this thread's 32 heads, read as broadcast 16-byte loads
+            const float4 *m4 = reinterpret_cast<const float4 *>(&sm.m_used[hb]);
             for (int kt = 0; kt < n_tiles; ++kt, ++g) {
                 ok = mbar_wait(&sm.s_full, g & 1u, kWaitIter);
                 if (!ok) break;
@@ -588,16 +610,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 tmem_ld_wait();
                 bool need = false;
 #pragma unroll
-                for (int h = 0; h < 32; ++h) {
-                    s[h] = valid ? s[h] * c2 : -INFINITY;
-                    need |= s[h] > sm.m_used[hb + h] + kRescaleThreshold;
+                for (int h4 = 0; h4 < 8; ++h4) {
+                    const float4 m = m4[h4];
+                    const float mm[4] = {m.x, m.y, m.z, m.w};
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int h = 4 * h4 + k;
+                        s[h] = valid ? s[h] * c2 : -INFINITY;
+                        need |= s[h] > mm[k] + kRescaleThreshold;
+                    }
                 }
-                if (need) atomicOr(&sm.flag, 1);
-                named_sync(1, kSoftThreads);
-                const int flag = sm.flag;
-                named_sync(1, kSoftThreads);
-                if (flag) {
-                    if (st == 0) sm.flag = 0;
+                if (named_sync_any(1, kSoftThreads, need)) {
                     float mx[32];
 #pragma unroll
                     for (int h = 0; h < 32; ++h) mx[h] = s[h];
@@ -631,10 +654,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
 #pragma unroll
                 for (int pc = 0; pc < 4; ++pc) {
                     float pv[8];
+                    const float4 ma = m4[2 * pc], mb = m4[2 * pc + 1];
+                    const float mm[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         const int h = pc * 8 + k;
-                        pv[k] = exp2f(s[h] - sm.m_used[hb + h]);
+                        pv[k] = ex2_fast(s[h] - mm[k]);
                         l_part[h] += pv[k];
                     }
                     uint4 u;
