@@ -271,6 +271,14 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
+// Key tiles [kt0, kt1) of a query that work item `sp` of `n_split` handles.
+__device__ __forceinline__ void split_range(int n_tiles, int n_split, int sp, int *kt0, int *kt1) {
+    const int per = (n_tiles + n_split - 1) / n_split;
+    const int a = sp * per < n_tiles ? sp * per : n_tiles;
+    *kt0 = a;
+    *kt1 = a + per < n_tiles ? a + per : n_tiles;
+}
+
 struct QueryGeom {
     int64_t b, i, t, lo_w;
     int n_win, n_wt;
@@ -304,7 +312,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     const __nv_bfloat16 *__restrict__ pool_rot, int64_t S_kv, int64_t kv_pos0, int64_t P,
     const int32_t *__restrict__ idx, int topk, int mode, const float *__restrict__ sink,
     __nv_bfloat16 *__restrict__ out, int64_t B, int64_t S_q, int64_t q_pos0, int window, int ratio,
-    float scale, RopeTable rope, const int32_t *__restrict__ packed_n, int kmax) {
+    float scale, RopeTable rope, const int32_t *__restrict__ packed_n, int kmax, int n_split,
+    float *__restrict__ part) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     unsigned char *smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -315,7 +324,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     Small &sm = *reinterpret_cast<Small *>(smem + kOffEnt + ent_bytes);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t nq = B * S_q;
+    // work item w = query w / n_split, key-tile range w % n_split of it (n_split > 1 only for
+    // decode-sized calls, whose partial results the combine kernel merges)
+    const int64_t nw = B * S_q * n_split;
 
     if (tid == 0) {
         for (int c = 0; c < 8; ++c) mbar_init(&sm.full[c], 1);
@@ -340,7 +351,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     if (warp == 0) {
         // ===================================================== loader
         uint32_t g = 0, qc = 0;
-        for (int64_t qi = blockIdx.x; qi < nq && !sm.abort_; qi += gridDim.x, ++qc) {
+        for (int64_t w = blockIdx.x; w < nw && !sm.abort_; w += gridDim.x, ++qc) {
+            const int64_t qi = w / n_split;
+            const int64_t qn = (w + gridDim.x) / n_split;   // query of the next work item
             const QueryGeom qg = query_geom(qi, S_q, q_pos0, kv_pos0, S_kv, window, packed_n);
             const int64_t nv = n_visible(qg.t, ratio, P);
             int n_ent;
@@ -367,8 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 }
                 n_ent = cnt;
                 // warm L2 with the next query's idx row
-                const int64_t qn = qi + gridDim.x;
-                if (qn < nq) {
+                if (w + gridDim.x < nw) {
                     const char *np = reinterpret_cast<const char *>(idx + qn * topk);
                     for (int off = lane * 128; off < topk * 4; off += 32 * 128)
                         asm volatile("prefetch.global.L2 [%0];" ::"l"(np + off));
@@ -392,8 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 for (int c = 0; c < 8; ++c)
                     tma_load_2d(s_q + (uint32_t)c * 8192u, &map_q, 64 * c, (int)(qi * kH), &sm.q_tma);
                 // bring the next query's Q into L2 while this query runs
-                const int64_t qn = qi + gridDim.x;
-                if (qn < nq)
+                if (w + gridDim.x < nw)
                     for (int c = 0; c < 8; ++c)
                         asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
                                          reinterpret_cast<uint64_t>(&map_q)),
@@ -406,11 +417,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 sm.qcs[0][lane] = cs;
                 sm.qcs[1][lane] = sn;
             }
-            const int n_tiles = qg.n_wt + (n_ent + kTile - 1) / kTile;
+            int kt0, kt1;
+            split_range(qg.n_wt + (n_ent + kTile - 1) / kTile, n_split, (int)(w % n_split), &kt0, &kt1);
             bool q_done = false;
             bool ok = true;
-            for (int kt = 0; kt <= n_tiles && ok; ++kt) {
-                if (kt == 1 || (kt == n_tiles && !q_done)) {
+            for (int kt = kt0; kt <= kt1 && ok; ++kt) {
+                if (kt == kt0 + 1 || (kt == kt1 && !q_done)) {
                     // rotate the rope channels of Q in place and publish it
                     ok = mbar_wait(&sm.q_tma, qc & 1u, kWaitIter);
                     if (!ok) break;
@@ -444,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                     if (lane == 0) mbar_arrive(&sm.q_full);
                     q_done = true;
                 }
-                if (kt == n_tiles) break;
+                if (kt == kt1) break;
                 const bool win = kt < qg.n_wt;
                 if (win) {
                     // window rows are contiguous: one 2-D TMA box of 128 rows per chunk
@@ -525,16 +537,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             const uint32_t hi = (uint32_t)(d_kv >> 32);   // SBO 1024, version, swizzle: shared
             uint32_t g = 0, qc = 0;
             bool ok = true;
-            for (int64_t qi = blockIdx.x; ok && qi < nq; qi += gridDim.x, ++qc) {
-                const QueryGeom qg = query_geom(qi, S_q, q_pos0, kv_pos0, S_kv, window, packed_n);
+            for (int64_t w = blockIdx.x; ok && w < nw; w += gridDim.x, ++qc) {
+                const QueryGeom qg = query_geom(w / n_split, S_q, q_pos0, kv_pos0, S_kv, window, packed_n);
                 ok = mbar_wait(&sm.meta_full[qc & 1], (qc >> 1) & 1u, kWaitIter);
                 if (!ok) break;
                 const int n_ent = sm.meta[qc & 1].n_ent;
-                const int n_tiles = qg.n_wt + (n_ent + kTile - 1) / kTile;
+                int kt0, kt1;
+                split_range(qg.n_wt + (n_ent + kTile - 1) / kTile, n_split, (int)(w % n_split), &kt0, &kt1);
                 ok = mbar_wait(&sm.q_full, qc & 1u, kWaitIter);
                 if (!ok) break;
                 tc_fence_after();
-                for (int kt = 0; ok && kt < n_tiles; ++kt, ++g) {
+                for (int kt = kt0; ok && kt < kt1; ++kt, ++g) {
                     // S^T = K . Qr^T, chunk by chunk as the tile lands
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
@@ -548,12 +561,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                     }
                     if (!ok) break;
                     mma_commit(&sm.s_full);
-                    if (kt == n_tiles - 1) mma_commit(&sm.q_free);
+                    if (kt == kt1 - 1) mma_commit(&sm.q_free);
                     ok = mbar_wait(&sm.p_full, g & 1u, kWaitIter);
                     if (!ok) break;
                     tc_fence_after();
                     // O^T += V^T . P^T, releasing each pair of key chunks when done
-                    const uint32_t acc0 = kt > 0 ? 1u : 0u;
+                    const uint32_t acc0 = kt > kt0 ? 1u : 0u;
 #pragma unroll
                     for (int mt = 0; mt < 4; ++mt) {
 #pragma unroll
@@ -564,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                     }
                 }
                 if (!ok) break;
-                if (n_tiles == 0) mma_commit(&sm.q_free);
+                if (kt1 == kt0) mma_commit(&sm.q_free);
                 mma_commit(&sm.o_full);
             }
             if (!ok) {
@@ -583,12 +596,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         const float c2 = scale * kLog2e;
         uint32_t g = 0, qc = 0;
         bool ok = true;
-        for (int64_t qi = blockIdx.x; ok && qi < nq; qi += gridDim.x, ++qc) {
+        for (int64_t w = blockIdx.x; ok && w < nw; w += gridDim.x, ++qc) {
+            const int64_t qi = w / n_split;
             const QueryGeom qg = query_geom(qi, S_q, q_pos0, kv_pos0, S_kv, window, packed_n);
             ok = mbar_wait(&sm.meta_full[qc & 1], (qc >> 1) & 1u, kWaitIter);
             if (!ok) break;
             const int n_ent = sm.meta[qc & 1].n_ent;
-            const int n_tiles = qg.n_wt + (n_ent + kTile - 1) / kTile;
+            int kt0, kt1;
+            split_range(qg.n_wt + (n_ent + kTile - 1) / kTile, n_split, (int)(w % n_split), &kt0, &kt1);
             if (st < kH) {
                 const float sk = sink[st];
                 sm.m_used[st] = sk == -INFINITY ? -INFINITY : sk * kLog2e;
@@ -599,7 +614,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             for (int h = 0; h < 32; ++h) l_part[h] = 0.f;
             // the running maxima of this thread's 32 heads, read as broadcast 16-byte loads
             const float4 *m4 = reinterpret_cast<const float4 *>(&sm.m_used[hb]);
-            for (int kt = 0; kt < n_tiles; ++kt, ++g) {
+            for (int kt = kt0; kt < kt1; ++kt, ++g) {
                 ok = mbar_wait(&sm.s_full, g & 1u, kWaitIter);
                 if (!ok) break;
                 tc_fence_after();
@@ -637,7 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                     named_sync(1, kSoftThreads);
 #pragma unroll
                     for (int h = 0; h < 32; ++h) l_part[h] *= sm.alpha[hb + h];
-                    if (kt > 0) {
+                    if (kt > kt0) {
 #pragma unroll 1
                         for (int mt = 0; mt < 4; ++mt) {
                             float o[32];
@@ -680,6 +695,35 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             warp_reduce32<false>(l_part);
             sm.red[lg][hb + lane] = l_part[0];
             named_sync(1, kSoftThreads);
+            if (part) {
+                // a key range of a split query: unnormalised O^T, the running maxima (log2
+                // units) and the row sums without the sink, for the combine kernel
+                float *pml = part + nw * (int64_t)(kH * kD) + w * (2 * kH);
+                if (st < kH) {
+                    pml[st] = sm.m_used[st];
+                    pml[kH + st] = sm.red[0][st] + sm.red[1][st] + sm.red[2][st] + sm.red[3][st];
+                }
+                ok = mbar_wait(&sm.o_full, qc & 1u, kWaitIter);
+                named_sync(1, kSoftThreads);
+                if (!ok) break;
+                tc_fence_after();
+                float *po = part + w * (int64_t)(kH * kD);
+#pragma unroll 1
+                for (int mt = 0; mt < 4; ++mt) {
+                    float o[32];
+                    if (kt1 > kt0) {
+                        tmem_ld32(trow + kColO + mt * 64 + hb, o);
+                        tmem_ld_wait();
+                    } else {
+#pragma unroll
+                        for (int h = 0; h < 32; ++h) o[h] = 0.f;
+                    }
+#pragma unroll
+                    for (int h = 0; h < 32; ++h) po[(int64_t)(hb + h) * kD + mt * 128 + x] = o[h];
+                }
+                tc_fence_before();
+                continue;
+            }
             if (st < kH) {
                 float l = sm.red[0][st] + sm.red[1][st] + sm.red[2][st] + sm.red[3][st];
                 const float sk = sink[st];
@@ -701,7 +745,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 const bool rot = d >= rope.first;
                 if (rot) rope_cs(-(double)qg.t, rope.inv_freq[(d - rope.first) >> 1], &cs, &sn);
                 float o[32];
-                if (n_tiles > 0) {
+                if (kt1 > kt0) {
                     tmem_ld32(trow + kColO + mt * 64 + hb, o);
                     tmem_ld_wait();
                 } else {
@@ -739,6 +783,78 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
+// Merges the key-range partials of split queries: per head, M = max over the ranges (and
+// the sink), weights 2^(m_s - M), l = sum of weighted row sums plus the sink term, then
+// O = sum of weighted O_s / l, the -t de-rotation of the rope channels and the bf16 store.
+// Block (query, group of 8 heads); every thread loads its 8 channel pairs of every range
+// before combining them, so the reads of a block are all in flight together.
+constexpr int kMaxSplit = 4;
+constexpr int kCombHeads = 8;
+__global__ void __launch_bounds__(256) attend_combine_kernel(const float *__restrict__ part, int n_split,
+                                                             int64_t nq, const float *__restrict__ sink,
+                                                             __nv_bfloat16 *__restrict__ out, int64_t S_q,
+                                                             int64_t q_pos0, RopeTable rope) {
+    __shared__ float wgt[kCombHeads][kMaxSplit];
+    __shared__ float inv_l[kCombHeads];
+    __shared__ float rcs[2][32];
+    const int64_t qi = blockIdx.x;
+    const int h0 = blockIdx.y * kCombHeads;
+    const int tid = threadIdx.x;
+    const float *pml = part + nq * n_split * (int64_t)(kH * kD);
+    if (tid < kCombHeads) {
+        const int h = h0 + tid;
+        const float sk = sink[h];
+        float M = sk == -INFINITY ? -INFINITY : sk * kLog2e;
+        for (int sp = 0; sp < n_split; ++sp) M = fmaxf(M, pml[(qi * n_split + sp) * (2 * kH) + h]);
+        float l = 0.f;
+        for (int sp = 0; sp < n_split; ++sp) {
+            const float *ml = pml + (qi * n_split + sp) * (2 * kH);
+            const float wv = M == -INFINITY ? 0.f : exp2f(ml[h] - M);
+            wgt[tid][sp] = wv;
+            l += wv * ml[kH + h];
+        }
+        if (sk != -INFINITY && M != -INFINITY) l += exp2f(sk * kLog2e - M);
+        inv_l[tid] = l > 0.f ? 1.f / l : 0.f;
+    }
+    if (tid >= 32 && tid - 32 < rope.n_pairs) {
+        float cs, sn;
+        rope_cs(-(double)(q_pos0 + qi % S_q), rope.inv_freq[tid - 32], &cs, &sn);
+        rcs[0][tid - 32] = cs;
+        rcs[1][tid - 32] = sn;
+    }
+    // thread: channel pair d = 2 * tid of the 8 heads
+    const int d = 2 * tid;
+    float2 v[kMaxSplit][kCombHeads];
+#pragma unroll
+    for (int sp = 0; sp < kMaxSplit; ++sp)
+        if (sp < n_split)
+#pragma unroll
+            for (int hh = 0; hh < kCombHeads; ++hh)
+                v[sp][hh] = *reinterpret_cast<const float2 *>(part + (qi * n_split + sp) * (int64_t)(kH * kD) +
+                                                            (int64_t)(h0 + hh) * kD + d);
+    __syncthreads();
+    float cs = 1.f, sn = 0.f;
+    const bool rot = d >= rope.first;
+    if (rot) {
+        cs = rcs[0][(d - rope.first) >> 1];
+        sn = rcs[1][(d - rope.first) >> 1];
+    }
+#pragma unroll
+    for (int hh = 0; hh < kCombHeads; ++hh) {
+        float a = 0.f, b = 0.f;
+#pragma unroll
+        for (int sp = 0; sp < kMaxSplit; ++sp)
+            if (sp < n_split) {
+                a += wgt[hh][sp] * v[sp][hh].x;
+                b += wgt[hh][sp] * v[sp][hh].y;
+            }
+        a *= inv_l[hh];
+        b *= inv_l[hh];
+        const float ra = rot ? a * cs - b * sn : a, rb = rot ? a * sn + b * cs : b;
+        *reinterpret_cast<__nv_bfloat162 *>(out + (qi * kH + h0 + hh) * (int64_t)kD + d) = __floats2bfloat162_rn(ra, rb);
+    }
+}
+
 }  // namespace
 
 bool attend_tc_eligible(const AttendArgs &a) {
@@ -765,11 +881,25 @@ int attend_tc_kmax(const AttendArgs &a) {
     return (int)(a.S_kv + e > 0 ? a.S_kv + e : 1);
 }
 
+// Decode-sized calls with few queries split each query's key tiles over two CTAs (the
+// device has 148 SMs) and merge the partials in a second kernel.
+static int attend_tc_split(const AttendArgs &a) {
+    if (!attend_tc_packed(a)) return 1;
+    const int64_t nq = a.B * a.S_q;
+    return (nq * 2 <= 148 && attend_tc_kmax(a) > kTile) ? 2 : 1;
+}
+
+static size_t split_part_bytes(const AttendArgs &a, int n_split) {
+    if (n_split <= 1) return 0;
+    return (size_t)a.B * a.S_q * n_split * (size_t)(kH * kD + 2 * kH) * sizeof(float);
+}
+
 size_t attend_tc_workspace(const AttendArgs &a) {
     if (attend_tc_packed(a)) {
         const size_t rows = (size_t)a.B * a.S_q * attend_tc_kmax(a);
+        // packed keys, key counts, entry lists, then the split partials
         return ((rows * kD * 2 + 255) & ~(size_t)255) + (((size_t)a.B * a.S_q * 4 + 255) & ~(size_t)255) +
-               rows * 4;   // packed keys, key counts, entry lists
+               ((rows * 4 + 255) & ~(size_t)255) + split_part_bytes(a, attend_tc_split(a));
     }
     size_t kv = ((size_t)a.B * a.S_kv * a.D * 2 + 255) & ~(size_t)255;
     size_t pl = ((size_t)a.B * a.P * a.D * 2 + 255) & ~(size_t)255;
@@ -825,11 +955,26 @@ csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st) {
     ensure_smem((const void *)attend_tc_kernel, smem);
     const int sms = device_sm_count();
     const int64_t nq = a.B * a.S_q;
-    const int grid = (int)(nq < sms ? nq : sms);
+    const int n_split = attend_tc_split(a);
+    float *part = nullptr;
+    if (n_split > 1) {
+        const size_t rows = (size_t)a.B * a.S_q * kmax;
+        part = reinterpret_cast<float *>(ws + ((rows * kD * 2 + 255) & ~(size_t)255) +
+                                         (((size_t)a.B * a.S_q * 4 + 255) & ~(size_t)255) +
+                                         ((rows * 4 + 255) & ~(size_t)255));
+    }
+    const int64_t nw = nq * n_split;
+    const int grid = (int)(nw < sms ? nw : sms);
     attend_tc_kernel<<<grid, kThreads, smem, st>>>(
         map_q, map_kv, pool_rot, a.S_kv, a.kv_pos0, a.P, a.idx, a.mode == 0 && !packed ? a.topk : 0, a.mode,
-        a.sink, (__nv_bfloat16 *)a.out, a.B, a.S_q, a.q_pos0, a.window, a.ratio, a.scale, a.rope, n_keys, kmax);
+        a.sink, (__nv_bfloat16 *)a.out, a.B, a.S_q, a.q_pos0, a.window, a.ratio, a.scale, a.rope, n_keys, kmax,
+        n_split, part);
     CSA_CHECK_LAUNCH(a.mode == 0 ? "csa_attend" : "hca_attend");
+    if (n_split > 1) {
+        attend_combine_kernel<<<dim3((unsigned)nq, kH / kCombHeads), kD / 2, 0, st>>>(
+            part, n_split, nq, a.sink, (__nv_bfloat16 *)a.out, a.S_q, a.q_pos0, a.rope);
+        CSA_CHECK_LAUNCH("attend: combine key ranges");
+    }
     return CSA_OK;
 }
 
