@@ -258,26 +258,55 @@ def gpu_arm(args, rank, world, local_rank):
             runners[li].run_stage(st)
     torch.cuda.synchronize()
 
-    # each stage captured once into a CUDA graph (the library only enqueues work on the
-    # current stream, so a call is capturable); the timed steps replay the graphs with CUDA
-    # events between them, which removes host launch overhead from the measurement
+    # The timed region is one CUDA graph holding all K steps (the library only enqueues work
+    # on the current stream, so its calls are capturable), with timing events recorded inside
+    # the graph around every stage of every step: no host launch gaps between kernels, and
+    # the per-stage times still come from device events over the timed region.  Fallbacks:
+    # one graph per stage replayed with events between them, then eager launches.
+    ev = {k: [(torch.cuda.Event(enable_timing=True, external=True),
+               torch.cuda.Event(enable_timing=True, external=True))
+              for _ in range(args.steps)] for k in stage_names}
+    whole = None
     graphs = None
     launches_per_step = None
+    launch_mode = "eager"
     if not args.eager:
         try:
             l0 = csa.launch_count()
-            graphs = {}
-            for key in stage_names:
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g):
-                    runners[key[0]].run_stage(key[1])
-                graphs[key] = g
-            launches_per_step = csa.launch_count() - l0
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for k in range(args.steps):
+                    for key in stage_names:
+                        ev[key][k][0].record()
+                        runners[key[0]].run_stage(key[1])
+                        ev[key][k][1].record()
+            launches_per_step = (csa.launch_count() - l0) // args.steps
             torch.cuda.synchronize()
-        except Exception as exc:  # pragma: no cover - falls back to eager launches
-            print("graph capture failed (%s); timing eager launches" % exc, file=sys.stderr)
-            graphs = None
+            g.replay()   # one untimed replay: first-launch costs of the graph itself
             torch.cuda.synchronize()
+            whole = g
+            launch_mode = "one CUDA graph for the K timed steps"
+        except Exception as exc:  # pragma: no cover - falls back to per-stage graphs
+            print("whole-run graph capture failed (%s); trying per-stage graphs" % exc, file=sys.stderr)
+            whole = None
+            torch.cuda.synchronize()
+            ev = {k: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                      for _ in range(args.steps)] for k in stage_names}
+            try:
+                l0 = csa.launch_count()
+                graphs = {}
+                for key in stage_names:
+                    gs = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(gs):
+                        runners[key[0]].run_stage(key[1])
+                    graphs[key] = gs
+                launches_per_step = csa.launch_count() - l0
+                torch.cuda.synchronize()
+                launch_mode = "CUDA graph per stage"
+            except Exception as exc2:  # pragma: no cover - falls back to eager launches
+                print("graph capture failed (%s); timing eager launches" % exc2, file=sys.stderr)
+                graphs = None
+                torch.cuda.synchronize()
 
     def step(events=None):
         for key in stage_names:
@@ -290,7 +319,8 @@ def gpu_arm(args, rank, world, local_rank):
             if events is not None:
                 events[key][1].record(stream)
 
-    step()
+    if whole is None:
+        step()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -299,23 +329,24 @@ def gpu_arm(args, rank, world, local_rank):
     clk = ClockSampler(local_rank)
     clk.start()
     time.sleep(0.3)
-    ev = {k: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)] for k in stage_names}
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     t0.record(stream)
-    for k in range(args.steps):
-        step({key: ev[key][k] for key in stage_names})
+    if whole is not None:
+        whole.replay()
+    else:
+        for k in range(args.steps):
+            step({key: ev[key][k] for key in stage_names})
     t1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clocks = clk.stop()
     launches = csa.launch_count() - launches0
-    if graphs is not None:
+    if launches_per_step is not None:
         launches = launches_per_step * args.steps
     ms_total = max_over_ranks(t0.elapsed_time(t1), world, dev)
     ms_step = ms_total / args.steps
@@ -375,7 +406,7 @@ def gpu_arm(args, rank, world, local_rank):
                    "P": [s.P for s in specs], "topk": spec0.topk, "H_I": spec0.H_I,
                    "d_I": spec0.d_I, "parallelism": "independent layer instance per GPU",
                    "l2": "inputs larger than L2 (q/out/q_I > 126 MB per step); no flush",
-                   "launch": "CUDA graph per stage" if graphs is not None else "eager"},
+                   "launch": launch_mode},
         "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
         "roofline": roof,
         "gpu_launches": int(launches),

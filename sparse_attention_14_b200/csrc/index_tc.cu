@@ -278,6 +278,39 @@ __device__ void group_emit_bitmap(const unsigned long long *cand, int n, int k, 
     }
 }
 
+// Merge of a decode-split query row: the candidate ranges' survivors (0 = empty slot) are
+// compacted into `cand`, cut to the topk largest into `keep`, and emitted in ascending
+// entry order through a bitmap of the nv visible entries.  All GS threads of the group
+// (named barrier `bar`) call it.
+template <int GS>
+__device__ void merge_ranges(const unsigned long long *__restrict__ partial_row, int total, int topk, int64_t nv,
+                             int gt, int bar, unsigned long long *cand, unsigned long long *keep, unsigned *bitmap,
+                             unsigned *hist, Misc &ms, int32_t *idx_row, float *score_row) {
+    if (gt == 0) {
+        ms.cnt[0] = 0;
+        ms.cnt[1] = 0;
+    }
+    named_sync(bar, GS);
+    for (int e = gt; e < total; e += GS) {
+        const unsigned long long c = __ldcg(partial_row + e);
+        if (c != 0ull) cand[atomicAdd(&ms.cnt[0], 1u)] = c;
+    }
+    named_sync(bar, GS);
+    int n = (int)ms.cnt[0];
+    const unsigned long long *src = cand;
+    if (n > topk) {
+        const unsigned long long T = group_kth<GS>(cand, n, topk, gt, bar, hist, ms, 0);
+        for (int e = gt; e < n; e += GS) {
+            const unsigned long long c = cand[e];
+            if (c >= T) keep[atomicAdd(&ms.cnt[1], 1u)] = c;
+        }
+        named_sync(bar, GS);
+        n = (int)ms.cnt[1];
+        src = keep;
+    }
+    group_emit_bitmap<GS>(src, n, topk, nv, gt, bar, bitmap, hist, ms, 0, idx_row, score_row);
+}
+
 // ------------------------------------------------------------------ main kernel
 template <int QB>
 __global__ void __launch_bounds__(Cfg<QB>::kThreads, Cfg<QB>::kMinBlocks) index_tc_kernel(
@@ -497,39 +530,15 @@ __global__ void __launch_bounds__(kMergeThreads) index_merge_kernel(
     float *__restrict__ scores_opt, int64_t S_q, int64_t q_pos0, int ratio, int64_t P) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int total = n_split * topk;
-    const int cap = pow2_ceil(total);
     unsigned long long *cand = reinterpret_cast<unsigned long long *>(smem_raw);
-    unsigned long long *keep = cand + cap;                   // pow2_ceil(topk) slots
+    unsigned long long *keep = cand + pow2_ceil(total);
     unsigned *hist = reinterpret_cast<unsigned *>(keep + pow2_ceil(topk));
     Misc &ms = *reinterpret_cast<Misc *>(hist + 256);
     unsigned *bitmap = reinterpret_cast<unsigned *>(&ms + 1);  // ceil(P/32) words
     const int64_t row = blockIdx.x;
-    const int64_t nv = n_visible(q_pos0 + row % S_q, ratio, P);
-    const int tid = threadIdx.x;
-    if (tid == 0) {
-        ms.cnt[0] = 0;
-        ms.cnt[1] = 0;
-    }
-    __syncthreads();
-    for (int e = tid; e < total; e += kMergeThreads) {
-        const unsigned long long c = partial[row * total + e];
-        if (c != 0ull) cand[atomicAdd(&ms.cnt[0], 1u)] = c;
-    }
-    __syncthreads();
-    int n = (int)ms.cnt[0];
-    unsigned long long *src = cand;
-    if (n > topk) {
-        const unsigned long long T = group_kth<kMergeThreads>(cand, n, topk, tid, 1, hist, ms, 0);
-        for (int e = tid; e < n; e += kMergeThreads) {
-            const unsigned long long c = cand[e];
-            if (c >= T) keep[atomicAdd(&ms.cnt[1], 1u)] = c;
-        }
-        __syncthreads();
-        n = (int)ms.cnt[1];
-        src = keep;
-    }
-    group_emit_bitmap<kMergeThreads>(src, n, topk, nv, tid, 1, bitmap, hist, ms, 0, idx + row * topk,
-                                     scores_opt ? scores_opt + row * topk : nullptr);
+    merge_ranges<kMergeThreads>(partial + row * total, total, topk, n_visible(q_pos0 + row % S_q, ratio, P),
+                                threadIdx.x, 1, cand, keep, bitmap, hist, ms, idx + row * topk,
+                                scores_opt ? scores_opt + row * topk : nullptr);
 }
 
 // ------------------------------------------------------------------ host side
@@ -588,10 +597,14 @@ bool index_tc_eligible(int64_t B, int64_t S_q, int64_t P, int H_I, int d_I, int 
            B * P + kTileE < (1ll << 31) && B * S_q * kHI + 256 < (1ll << 31);
 }
 
+static size_t partial_bytes(const Plan &p, int64_t B, int64_t S_q, int topk) {
+    return ((size_t)B * S_q * p.n_split * topk * sizeof(unsigned long long) + 255) & ~(size_t)255;
+}
+
 size_t index_tc_workspace(int64_t B, int64_t S_q, int64_t q_pos0, int64_t P, int ratio, int topk) {
     Plan p = plan(B, S_q, q_pos0, P, ratio, topk);
     if (p.n_split <= 1) return 0;
-    return (size_t)B * S_q * p.n_split * topk * sizeof(unsigned long long);
+    return partial_bytes(p, B, S_q, topk);   // candidates per (row, range)
 }
 
 csa_status_t index_tc(const void *qI, const void *w, const void *kI, int64_t B, int64_t S_q, int64_t q_pos0,
@@ -605,7 +618,7 @@ csa_status_t index_tc(const void *qI, const void *w, const void *kI, int64_t B, 
                 "csa_index_topk: cannot encode the q_I tensor map");
     unsigned long long *partial = nullptr;
     if (p.n_split > 1) {
-        const size_t need = (size_t)B * S_q * p.n_split * topk * sizeof(unsigned long long);
+        const size_t need = partial_bytes(p, B, S_q, topk);
         CSA_REQUIRE(workspace && workspace_bytes >= need, CSA_ERR_WORKSPACE,
                     "csa_index_topk: workspace of %zu B given, %zu B needed", workspace_bytes, need);
         partial = reinterpret_cast<unsigned long long *>(workspace);
