@@ -1,5 +1,5 @@
 // attend_tc.cu -- tensor-core (tcgen05 / TMEM) sink attention for the V4-Flash head shape
-// (64 query heads sharing one K=V head of dim 512, bf16), prefill.
+// (64 query heads sharing one K=V head of dim 512, bf16), prefill and decode.
 //
 // Same semantics as attend.cu (HF docs model_doc/deepseek_v4, section 2.3: shared K=V
 // MQA, partial RoPE with the -i output rotation of eq. 26, sink of eq. 27; "Attention
@@ -28,7 +28,10 @@
 //    as the initial running max and once in the final sum;
 //  * epilogue: O^T / l and the -t de-rotation of the rope channels (partner channel via a
 //    lane shuffle), stored as bf16 pairs straight from registers while the next query's
-//    first tile loads and multiplies.
+//    first tile loads and multiplies;
+//  * decode-sized calls (few queries over a long cache) pack each query's rotated keys
+//    first; with few queries, each query's key tiles are split over two CTAs that write
+//    unnormalised partials, merged (sink, division, de-rotation) by attend_combine_kernel.
 #include <mutex>
 
 #include "attend.cuh"
