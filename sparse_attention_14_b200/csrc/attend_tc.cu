@@ -167,6 +167,15 @@ __global__ void __launch_bounds__(256) pack_rows_kernel(
     const int64_t qi = blockIdx.x;
     const int x0 = blockIdx.y * kPackRows;
     const int nk = n_keys[qi];
+    {
+        // rows [nk, kmax) hold no key but are read (with zero weight) by the last key tile
+        // of the query: zero them so that stale workspace bits cannot turn into NaN
+        const int z0 = nk > x0 ? nk : x0;
+        const int z1 = x0 + kPackRows < kmax ? x0 + kPackRows : kmax;
+        for (int v = threadIdx.x; v < (z1 - z0) * (kD / 8); v += blockDim.x)
+            *reinterpret_cast<uint4 *>(packed + (qi * kmax + z0 + v / (kD / 8)) * kD + (v % (kD / 8)) * 8) =
+                make_uint4(0u, 0u, 0u, 0u);
+    }
     if (x0 >= nk) return;
     const int64_t b = qi / S_q, t = q_pos0 + qi % S_q;
     int64_t lo = t - window + 1;

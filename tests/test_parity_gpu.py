@@ -33,6 +33,14 @@ MID = [
     LayerSpec(name="mid_decode_bf16", dtype="bf16", B=3, S_q=1, S_kv=128, q_pos0=4095,
               kv_pos0=3968, H=64, D=512, R=64, base=160000.0, W=128, m=4, P=1024, kind="csa",
               H_I=64, d_I=128, topk=64, decode=True, workload=94),
+    # decode-sized calls whose key tiles are split over two CTAs and merged by the combine
+    # kernel: HCA entries, and several queries per sequence over a window of 130 rows
+    LayerSpec(name="mid_hca_decode_bf16", dtype="bf16", B=2, S_q=1, S_kv=128, q_pos0=2047,
+              kv_pos0=1920, H=64, D=512, R=64, base=160000.0, W=128, m=128, P=16, kind="hca",
+              decode=True, workload=87),
+    LayerSpec(name="mid_decode_sq3_bf16", dtype="bf16", B=2, S_q=3, S_kv=130, q_pos0=4093,
+              kv_pos0=3966, H=64, D=512, R=64, base=160000.0, W=128, m=4, P=1024, kind="csa",
+              H_I=64, d_I=128, topk=64, decode=True, workload=86),
     # V4-Flash head shape on the tensor-core path: window-only layer, and a CSA layer
     # whose key count per query is not a multiple of the 128-key tile
     LayerSpec(name="mid_sliding_tc_bf16", dtype="bf16", B=2, S_q=333, S_kv=333, q_pos0=0,
@@ -124,6 +132,21 @@ def test_attend_stagewise_parity(spec):
     out = GpuLayer(spec, inp).attend(pool_in, idx_in)
     torch.cuda.synchronize()
     ref = oracle_attend(spec, inp, rows, None if pool_in is None else to_np(pool_in), o_idx)
+    assert rel_err(to_np(out), ref) <= TOL[spec.dtype]
+
+
+def test_decode_split_sink_minus_inf():
+    """The combine kernel adds the sink once: with a sink of -inf on half the heads (the
+    plain softmax over the keys) the split decode path still matches the oracle."""
+    spec = next(x for x in MID if x.name == "mid_decode_bf16")
+    inp = _inputs(spec)
+    inp["sink"][::2] = float("-inf")
+    rows = list(range(spec.S_q))
+    _, o_idx, _ = oracle_index(spec, inp, rows)
+    out = GpuLayer(spec, inp).attend(inp["pool"], torch.from_numpy(o_idx).to(DEV))
+    torch.cuda.synchronize()
+    ref = oracle_attend(spec, inp, rows, to_np(inp["pool"]), o_idx)
+    assert np.isfinite(to_np(out)).all()
     assert rel_err(to_np(out), ref) <= TOL[spec.dtype]
 
 
