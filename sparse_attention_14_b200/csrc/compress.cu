@@ -11,7 +11,9 @@
 // and each thread keeps a running (max, sum of weights, weighted sum) per channel --
 // an online softmax -- so the window is read exactly once, in one pass.
 //  * short windows (up to 8 tokens, e.g. CSA: 2m = 8): one thread per (entry, 8
-//    channels), the window loaded four tokens at a time into registers;
+//    channels); fp32 loads four tokens at a time into an online softmax, bf16 keeps the
+//    whole window's raw vectors in registers and takes the maximum first (one
+//    exponential per token and channel);
 //  * longer windows (HCA: 128 tokens): the window is split over `split` thread rows of
 //    one CTA, each row reads every split-th token (so a warp-row reads consecutive rows
 //    of HBM), and the partial softmax states are merged through shared memory.
@@ -92,6 +94,80 @@ __global__ void __launch_bounds__(256) compress_rows_kernel(const T *__restrict_
     store8(pool + (b * P + j) * D + g8 * 8, o);
 }
 
+// bf16, windows of up to 8 tokens (CSA): one thread per (b, j, 8-channel group) with the
+// whole window's raw 16-byte vectors in registers (all 16 loads in flight at once), then
+// two passes: the per-channel maximum, then one exponential per token and channel (the
+// online form above needs two).
+__device__ __forceinline__ void unpack8(const uint4 &u, float *v) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        v[2 * k] = __uint_as_float(w[k] << 16);
+        v[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+    }
+}
+
+__global__ void __launch_bounds__(256) compress_rows8_bf16_kernel(const __nv_bfloat16 *__restrict__ kv,
+                                                                   const __nv_bfloat16 *__restrict__ gate,
+                                                                   __nv_bfloat16 *__restrict__ pool, int64_t B,
+                                                                   int64_t S, int D, int ratio, int overlap,
+                                                                   int64_t P) {
+    const int groups = D / 8;
+    int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    int64_t total = B * P * groups;
+    if (gid >= total) return;
+    int g8 = (int)(gid % groups);
+    int64_t j = (gid / groups) % P;
+    int64_t b = gid / ((int64_t)groups * P);
+    int64_t lo = overlap ? (j - 1) * ratio : j * ratio;
+    if (lo < 0) lo = 0;
+    const int n = (int)((j + 1) * ratio - lo);   // <= 8
+    const uint4 *kv_p = reinterpret_cast<const uint4 *>(kv + (b * S + lo) * D + g8 * 8);
+    const uint4 *g_p = reinterpret_cast<const uint4 *>(gate + (b * S + lo) * D + g8 * 8);
+    const int stride = D / 8;   // uint4 per row
+    uint4 gr[8], vr[8];
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+        if (s < n) {
+            gr[s] = __ldg(g_p + (int64_t)s * stride);
+            vr[s] = __ldg(kv_p + (int64_t)s * stride);
+        }
+    }
+    float mx[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) mx[c] = -INFINITY;
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+        if (s < n) {
+            float gv[8];
+            unpack8(gr[s], gv);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) mx[c] = fmaxf(mx[c], gv[c]);
+        }
+    }
+    float den[8], num[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) den[c] = num[c] = 0.f;
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+        if (s < n) {
+            float gv[8], vv[8];
+            unpack8(gr[s], gv);
+            unpack8(vr[s], vv);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const float e = __expf(gv[c] - mx[c]);
+                den[c] += e;
+                num[c] = fmaf(e, vv[c], num[c]);
+            }
+        }
+    }
+    float o[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) o[c] = num[c] / den[c];
+    store8(pool + (b * P + j) * D + g8 * 8, o);
+}
+
 // CTA per (entry j, batch b, channel block); threadIdx.x = 8-channel group within the
 // block, threadIdx.y = token split.
 template <typename T>
@@ -152,8 +228,11 @@ csa_status_t launch_compress(const T *kv, const T *gate, T *pool, int64_t B, int
         int64_t total = B * P * (D / 8);
         int64_t blocks = ceil_div(total, 256);
         CSA_REQUIRE(blocks < (1ll << 31), CSA_ERR_UNSUPPORTED, "csa_compress: too many entries");
-        compress_rows_kernel<T, 8><<<(unsigned)blocks, 256, 0, st>>>(kv, gate, pool, B, S, D, ratio,
-                                                                     overlap, P);
+        if constexpr (sizeof(T) == 2)
+            compress_rows8_bf16_kernel<<<(unsigned)blocks, 256, 0, st>>>(kv, gate, pool, B, S, D, ratio, overlap, P);
+        else
+            compress_rows_kernel<T, 8><<<(unsigned)blocks, 256, 0, st>>>(kv, gate, pool, B, S, D, ratio,
+                                                                         overlap, P);
     } else {
         int split = 8;
         while (split > 1 && win / split < 4) split /= 2;
