@@ -321,7 +321,8 @@ __device__ __forceinline__ QueryGeom query_geom(int64_t qi, int64_t S_q, int64_t
 
 __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kv,
-    const __nv_bfloat16 *__restrict__ pool_rot, int64_t S_kv, int64_t kv_pos0, int64_t P,
+    const __grid_constant__ CUtensorMap map_pool, const __nv_bfloat16 *__restrict__ pool_rot, int64_t S_kv,
+    int64_t kv_pos0, int64_t P,
     const int32_t *__restrict__ idx, int topk, int mode, const float *__restrict__ sink,
     __nv_bfloat16 *__restrict__ out, int64_t B, int64_t S_q, int64_t q_pos0, int window, int ratio,
     float scale, RopeTable rope, const int32_t *__restrict__ packed_n, int kmax, int n_split,
@@ -470,15 +471,19 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 }
                 if (kt == kt1) break;
                 const bool win = kt < qg.n_wt;
-                if (win) {
-                    // window rows are contiguous: one 2-D TMA box of 128 rows per chunk
-                    const int y0 = packed_n ? (int)(qi * kmax + (int64_t)kt * kTile)
-                                            : (int)(qg.b * S_kv + (qg.lo_w - kv_pos0) + (int64_t)kt * kTile);
+                // HCA entries (every visible one, in order) are contiguous rows of the rotated
+                // pool, like window rows: both come as 2-D TMA boxes of 128 rows per chunk
+                const bool hca_ent = !win && mode == 1 && !packed_n;
+                if (win || hca_ent) {
+                    const CUtensorMap *map = win ? &map_kv : &map_pool;
+                    const int y0 = hca_ent ? (int)(qg.b * P + (int64_t)(kt - qg.n_wt) * kTile)
+                                   : packed_n ? (int)(qi * kmax + (int64_t)kt * kTile)
+                                              : (int)(qg.b * S_kv + (qg.lo_w - kv_pos0) + (int64_t)kt * kTile);
                     for (int c = 0; c < 8 && ok; ++c) {
                         if ((c & 1) == 0 && g > 0) ok = mbar_wait(&sm.free_[c >> 1], (g - 1) & 1u, kWaitIter);
                         if (ok && lane == 0) {
                             mbar_expect_tx(&sm.full[c], 16384u);
-                            tma_load_2d(s_kv + (uint32_t)c * 16384u, &map_kv, 64 * c, y0, &sm.full[c]);
+                            tma_load_2d(s_kv + (uint32_t)c * 16384u, map, 64 * c, y0, &sm.full[c]);
                         }
                     }
                 } else {
@@ -958,10 +963,16 @@ csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st) {
             CSA_CHECK_LAUNCH("attend: rotate entries");
         }
     }
-    CUtensorMap map_q, map_kv;
+    CUtensorMap map_q, map_kv, map_pool;
     CSA_REQUIRE(encode_map_bf16_2d(&map_q, a.q, kD, (uint64_t)(a.B * a.S_q * kH), 64u, 64u) &&
                     encode_map_bf16_2d(&map_kv, kv_rot, kD, kv_rows, 64u, (uint32_t)kTile),
                 CSA_ERR_CUDA, "attend: cannot encode the TMA tensor maps");
+    // the rotated pool as TMA rows (HCA entry tiles); other calls never use it
+    if (!packed && a.mode == 1 && a.P > 0)
+        CSA_REQUIRE(encode_map_bf16_2d(&map_pool, pool_rot, kD, (uint64_t)(a.B * a.P), 64u, (uint32_t)kTile),
+                    CSA_ERR_CUDA, "attend: cannot encode the pool tensor map");
+    else
+        map_pool = map_kv;
     const size_t smem = tc_smem_bytes(a.mode == 0 && !packed ? a.topk : 1);
     CSA_REQUIRE(smem <= 232448, CSA_ERR_UNSUPPORTED, "attend: shared memory %zu B too large", smem);
     ensure_smem((const void *)attend_tc_kernel, smem);
@@ -978,7 +989,7 @@ csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st) {
     const int64_t nw = nq * n_split;
     const int grid = (int)(nw < sms ? nw : sms);
     attend_tc_kernel<<<grid, kThreads, smem, st>>>(
-        map_q, map_kv, pool_rot, a.S_kv, a.kv_pos0, a.P, a.idx, a.mode == 0 && !packed ? a.topk : 0, a.mode,
+        map_q, map_kv, map_pool, pool_rot, a.S_kv, a.kv_pos0, a.P, a.idx, a.mode == 0 && !packed ? a.topk : 0, a.mode,
         a.sink, (__nv_bfloat16 *)a.out, a.B, a.S_q, a.q_pos0, a.window, a.ratio, a.scale, a.rope, n_keys, kmax,
         n_split, part);
     CSA_CHECK_LAUNCH(a.mode == 0 ? "csa_attend" : "hca_attend");
