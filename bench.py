@@ -400,13 +400,9 @@ def gpu_arm(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "f32" if spec0.dtype == "f32" else "bf16",
         "data": "synthetic (seeded N(0,1) q/kv/gate/q_I/k_I, w/sqrt(H_I), RMS-normalised kv)",
-        "config": {"workload": workload_name(args.workload, specs), "B": spec0.B, "S": spec0.S_q,
-                   "H": spec0.H, "D": spec0.D, "rope_dim": spec0.R, "window": spec0.W,
-                   "layers": [s.kind for s in specs], "m": [s.m for s in specs],
-                   "P": [s.P for s in specs], "topk": spec0.topk, "H_I": spec0.H_I,
-                   "d_I": spec0.d_I, "parallelism": "independent layer instance per GPU",
-                   "l2": "inputs larger than L2 (q/out/q_I > 126 MB per step); no flush",
-                   "launch": launch_mode},
+        "config": dict(workload_config(args.workload, specs),
+                       l2="inputs larger than L2 (q/out/q_I > 126 MB per step); no flush",
+                       launch=launch_mode),
         "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
         "roofline": roof,
         "gpu_launches": int(launches),
@@ -420,6 +416,15 @@ def workload_name(w, specs):
     return {0: "tiny CSA layer fp32 (S=256)", 1: "CSA prefill bf16 S=8192 (V4-Flash layer shape)",
             2: "HCA prefill bf16 S=65536", 3: "CSA decode bf16 B=64 at 65536 cached tokens",
             4: "mixed 4-layer stack bf16 S=131072"}[w]
+
+
+def workload_config(w, specs):
+    """The workload part of the JSON line's config, shared by both arms."""
+    spec0 = specs[0]
+    return {"workload": workload_name(w, specs), "B": spec0.B, "S": spec0.S_q, "H": spec0.H,
+            "D": spec0.D, "rope_dim": spec0.R, "window": spec0.W, "layers": [s.kind for s in specs],
+            "m": [s.m for s in specs], "P": [s.P for s in specs], "topk": spec0.topk,
+            "H_I": spec0.H_I, "d_I": spec0.d_I, "parallelism": "independent layer instance per GPU"}
 
 
 def e2e_arm(args, runners, stage_names, stream, world, dev):
@@ -548,7 +553,7 @@ def reference_arm(args, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": workload_name(args.workload, None), "B": spec.B, "S": spec.S_q},
+            "config": workload_config(args.workload, workload_specs(args.workload)),
             "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s",
                              "cores": oracle_threads(), "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
