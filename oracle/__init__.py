@@ -7,6 +7,7 @@ float64 and calls it.  It shares no code with the CUDA library.
 
 Function map (each C function's comment cites the page passage it follows):
   compress      -> orc_compress       gated pooling, CSA/HCA windows
+  CompressorState.append -> orc_compress_step   stateful (decode) compressor
   n_visible     -> orc_n_visible      causal visibility of compressed entries
   index_scores  -> orc_index_scores   Lightning Indexer score
   topk          -> orc_topk           top-k with -1 marker
@@ -49,6 +50,8 @@ def _bind(path: str):
     lib = ctypes.CDLL(path)
     lib.orc_rope_rows.argtypes = [_dp, _dp, _i64, _i64, _i64, ctypes.c_double]
     lib.orc_compress.argtypes = [_dp, _dp, _dp, _i64, _i64, _i64, _i64, ctypes.c_int]
+    lib.orc_compress_step.argtypes = [_dp, _dp, _dp, _dp, _lp, _lp, _dp, _dp, _i64, _i64, _i64,
+                                      _i64, ctypes.c_int, _dp, _i64, _lp]
     lib.orc_n_visible.argtypes = [_i64, _i64, _i64]
     lib.orc_n_visible.restype = _i64
     lib.orc_index_scores.argtypes = [_dp, _dp, _dp, _lp, _i64, _i64, _i64, _i64, _i64, _i64, _dp]
@@ -125,6 +128,40 @@ def compress(kv, gate, m: int, overlap: int) -> np.ndarray:
     _check(_load().orc_compress(_ptr(kv, _dp), _ptr(gate, _dp), _ptr(pool, _dp), B, S, D, m,
                                 int(overlap)), "compress")
     return pool
+
+
+class CompressorState:
+    """Stateful compressor of B sequences for decode (orc_compress_step): a buffer of the
+    open window, the last closed block (overlap) and a token counter, all fp64."""
+
+    def __init__(self, B: int, D: int, m: int, overlap: int):
+        self.B, self.D, self.m, self.overlap = B, D, m, int(bool(overlap))
+        self.buf_kv = np.zeros((B, m, D))
+        self.buf_gate = np.zeros((B, m, D))
+        self.ovl_kv = np.zeros((B, m, D))
+        self.ovl_gate = np.zeros((B, m, D))
+        self.counter = np.zeros(B, dtype=np.int64)
+        self.n_ovl = np.zeros(B, dtype=np.int64)
+
+    def append(self, kv_new, gate_new) -> np.ndarray:
+        """kv_new, gate_new [B,n,D] (the next n tokens) -> the entries whose windows close
+        among them, [B, n_closed, D] in closing order (n_closed may be 0)."""
+        kv, gate = _f64(kv_new), _f64(gate_new)
+        B, n, D = kv.shape
+        if B != self.B or D != self.D or gate.shape != kv.shape:
+            raise ValueError("CompressorState.append: shape mismatch")
+        max_out = n // self.m + 1
+        out = np.zeros((B, max_out, D))
+        n_out = np.zeros(B, dtype=np.int64)
+        _check(_load().orc_compress_step(_ptr(self.buf_kv, _dp), _ptr(self.buf_gate, _dp),
+                                         _ptr(self.ovl_kv, _dp), _ptr(self.ovl_gate, _dp),
+                                         _ptr(self.counter, _lp), _ptr(self.n_ovl, _lp),
+                                         _ptr(kv, _dp), _ptr(gate, _dp), n, B, D, self.m,
+                                         self.overlap, _ptr(out, _dp), max_out,
+                                         _ptr(n_out, _lp)), "compress_step")
+        if B and not np.all(n_out == n_out[0]):
+            raise ValueError("CompressorState.append: sequences closed different counts")
+        return out[:, : int(n_out[0]) if B else 0]
 
 
 def n_visible(t: int, m: int, P: int) -> int:

@@ -107,6 +107,91 @@ int orc_compress(const double *kv, const double *gate, double *pool,
     return ORC_OK;
 }
 
+/* ---------------------------------------------------------------------------------
+ * Stateful compressor for decode, [HF-PR] "Compressor/Indexer statefulness ... state
+ * lives on a new DeepseekV4Cache ... per-layer compressor_state and indexer_state dicts
+ * (buffer_kv, buffer_gate, pooled_kv)" and "_accumulate_windows and _update_pool ...
+ * single cache update per call"; [HF-DOC] "Cache layers": the HCA cache keeps a
+ * compressor buffer / pool / counter, the CSA cache the same plus its overlap state.
+ *
+ * State of sequence b (the layout is this oracle's own):
+ *   buf_kv, buf_gate [B, m, D]  tokens of the window that has not closed yet; the first
+ *                               counter[b] mod m rows are live
+ *   ovl_kv, ovl_gate [B, m, D]  the last closed block of m tokens (overlap=1 only);
+ *                               n_ovl[b] rows are live (0 before the first close)
+ *   counter [B]                 tokens seen so far
+ * Each new token goes into the buffer.  When the buffer holds m tokens the window
+ * closes: its entry pools the overlap block followed by the buffer (overlap=1), or the
+ * buffer alone (overlap=0), by the per-channel gate softmax of orc_compress; then, with
+ * overlap, the buffer becomes the overlap block; the buffer starts empty again.
+ * Entries are written in closing order to out[b, 0 .. n_out[b]).
+ * ------------------------------------------------------------------------------- */
+static void pool_window(const double *kv, const double *gate, int64_t n, int64_t D,
+                        double *entry)
+{
+    for (int64_t d = 0; d < D; ++d) {
+        double gmax = -INFINITY;
+        for (int64_t s = 0; s < n; ++s)
+            if (gate[s * D + d] > gmax) gmax = gate[s * D + d];
+        double acc = 0.0, z = 0.0;
+        for (int64_t s = 0; s < n; ++s) {
+            double wgt = exp(gate[s * D + d] - gmax);
+            acc += wgt * kv[s * D + d];
+            z += wgt;
+        }
+        entry[d] = acc / z;
+    }
+}
+
+int orc_compress_step(double *buf_kv, double *buf_gate, double *ovl_kv, double *ovl_gate,
+                      int64_t *counter, int64_t *n_ovl, const double *kv_new,
+                      const double *gate_new, int64_t n_new, int64_t B, int64_t D, int64_t m,
+                      int overlap, double *out, int64_t max_out, int64_t *n_out)
+{
+    if (B < 0 || n_new < 0 || D <= 0 || m <= 0 || max_out < 0) return ORC_BAD_ARG;
+    double *win_kv = (double *)malloc(sizeof(double) * (size_t)(2 * m * D));
+    double *win_gate = (double *)malloc(sizeof(double) * (size_t)(2 * m * D));
+    if (!win_kv || !win_gate) {
+        free(win_kv);
+        free(win_gate);
+        return ORC_NO_MEM;
+    }
+    int rc = ORC_OK;
+    for (int64_t b = 0; b < B && rc == ORC_OK; ++b) {
+        n_out[b] = 0;
+        for (int64_t i = 0; i < n_new; ++i) {
+            int64_t fill = counter[b] % m;   /* live rows in the buffer */
+            memcpy(buf_kv + (b * m + fill) * D, kv_new + (b * n_new + i) * D, sizeof(double) * (size_t)D);
+            memcpy(buf_gate + (b * m + fill) * D, gate_new + (b * n_new + i) * D, sizeof(double) * (size_t)D);
+            counter[b] += 1;
+            if (fill + 1 < m) continue;      /* the window is still open */
+            int64_t n = 0;
+            if (overlap) {
+                memcpy(win_kv, ovl_kv + b * m * D, sizeof(double) * (size_t)(n_ovl[b] * D));
+                memcpy(win_gate, ovl_gate + b * m * D, sizeof(double) * (size_t)(n_ovl[b] * D));
+                n = n_ovl[b];
+            }
+            memcpy(win_kv + n * D, buf_kv + b * m * D, sizeof(double) * (size_t)(m * D));
+            memcpy(win_gate + n * D, buf_gate + b * m * D, sizeof(double) * (size_t)(m * D));
+            n += m;
+            if (n_out[b] >= max_out) {
+                rc = ORC_BAD_ARG;
+                break;
+            }
+            pool_window(win_kv, win_gate, n, D, out + (b * max_out + n_out[b]) * D);
+            n_out[b] += 1;
+            if (overlap) {
+                memcpy(ovl_kv + b * m * D, buf_kv + b * m * D, sizeof(double) * (size_t)(m * D));
+                memcpy(ovl_gate + b * m * D, buf_gate + b * m * D, sizeof(double) * (size_t)(m * D));
+                n_ovl[b] = m;
+            }
+        }
+    }
+    free(win_kv);
+    free(win_gate);
+    return rc;
+}
+
 /* Entry j is visible to the query at absolute position t iff (j+1)m-1 <= t, so the
  * visible entries are j < min(P, floor((t+1)/m)).  [HF-DOC] "Attention mask layout":
  * with m=8, entry 0 opens at t >= 7 and entry 1 at t >= 15. */

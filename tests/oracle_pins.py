@@ -108,6 +108,84 @@ def pin_compress_two_token_golden():
     np.testing.assert_allclose(pool, np.array(g["pool"]), rtol=1e-14, atol=1e-14)
 
 
+# ----------------------------------------------------------------------------- stateful compressor
+def _chunks(rng, S, m):
+    """A split of S tokens into calls: single tokens, a window's worth, runs across
+    several windows, in a seeded random order."""
+    sizes = [1, 1, 2, max(1, m - 1), m, m + 1, 2 * m + 1, 3, 5 * m]
+    out = []
+    while sum(out) < S:
+        out.append(min(int(rng.choice(sizes)), S - sum(out)))
+    return out
+
+
+def pin_stateful_compressor_equals_whole_sequence():
+    """HF PR #45616 (compressor state on the cache: buffer, pooled cache; one update per
+    call) and HF docs "Cache layers" (buffer / pool / counter, CSA overlap state): pooling
+    token by token through the state yields the entries the stateless compressor computes
+    over the whole sequence, for any split of the stream into calls, and each call emits
+    exactly the entries whose windows close inside it."""
+    for m, overlap, D in ((4, 1, 6), (8, 0, 5), (1, 1, 3), (3, 0, 4), (2, 1, 2)):
+        rng = _rng(300 + 10 * m + overlap)
+        B, S = 2, 61
+        kv = rng.standard_normal((B, S, D))
+        gate = 3.0 * rng.standard_normal((B, S, D))
+        ref = oracle.compress(kv, gate, m, overlap)
+        for chunks in ([1] * S, [S], _chunks(rng, S, m), _chunks(rng, S, m)):
+            st = oracle.CompressorState(B, D, m, overlap)
+            got, start = [], 0
+            for c in chunks:
+                e = st.append(kv[:, start:start + c], gate[:, start:start + c])
+                assert e.shape == (B, (start + c) // m - start // m, D), (m, overlap, start, c)
+                got.append(e)
+                start += c
+            np.testing.assert_allclose(np.concatenate(got, axis=1), ref, rtol=1e-13, atol=1e-13)
+
+
+def pin_stateful_compressor_closes_at_worked_example():
+    """HF docs "Attention mask layout", HCA paragraph (m=8): entry 0 (tokens 0..7) exists
+    once token 7 is in, entry 1 (tokens 8..15) once token 15 is in; HF PR #45616: before a
+    window closes the compressor returns an empty tensor, not nothing."""
+    g = _golden("hca_visibility_m8.json")
+    m, T = g["m"], g["tokens"]
+    close_at = {t0: int(j) for j, t0 in g["first_visible_query"].items()}
+    rng = _rng(7)
+    kv, gate = rng.standard_normal((1, T, 3)), rng.standard_normal((1, T, 3))
+    st = oracle.CompressorState(1, 3, m, 0)
+    for t in range(T):
+        e = st.append(kv[:, t:t + 1], gate[:, t:t + 1])
+        if t in close_at:
+            assert e.shape == (1, 1, 3), t
+            j = close_at[t]
+            w = np.exp(gate[0, j * m:(j + 1) * m] - gate[0, j * m:(j + 1) * m].max(axis=0))
+            np.testing.assert_allclose(e[0, 0], (w * kv[0, j * m:(j + 1) * m]).sum(0) / w.sum(0),
+                                       rtol=1e-13)
+        else:
+            assert e.shape == (1, 0, 3), t
+
+
+def pin_stateful_compressor_state_holds_open_window():
+    """The state after n tokens: the counter is n, the buffer holds the n mod m tokens of
+    the open window, and (CSA, overlap) the overlap block is the last closed block."""
+    m, D, B = 4, 3, 2
+    rng = _rng(11)
+    kv, gate = rng.standard_normal((B, 23, D)), rng.standard_normal((B, 23, D))
+    st = oracle.CompressorState(B, D, m, 1)
+    n = 0
+    for c in (3, 1, 6, 2, 11):
+        st.append(kv[:, n:n + c], gate[:, n:n + c])
+        n += c
+        assert list(st.counter) == [n] * B
+        r = n % m
+        np.testing.assert_array_equal(st.buf_kv[:, :r], kv[:, n - r:n])
+        np.testing.assert_array_equal(st.buf_gate[:, :r], gate[:, n - r:n])
+        if n >= m:
+            c0 = (n // m - 1) * m
+            assert list(st.n_ovl) == [m] * B
+            np.testing.assert_array_equal(st.ovl_kv, kv[:, c0:c0 + m])
+            np.testing.assert_array_equal(st.ovl_gate, gate[:, c0:c0 + m])
+
+
 # ----------------------------------------------------------------------------- visibility
 def pin_visibility_worked_example():
     g = _golden("hca_visibility_m8.json")

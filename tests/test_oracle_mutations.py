@@ -34,6 +34,10 @@ MUTATIONS = [
     ("hca_entry_position", "kpos[nk] = (double)j * (double)m;\n                        ++nk;\n                    }\n                }\n                attend_query",
      "kpos[nk] = (double)(j + 1) * (double)m - 1.0;\n                        ++nk;\n                    }\n                }\n                attend_query"),
     ("value_unrotated", "o[d] += p * krot[x * D + d];", "o[d] += p * keys[x][d];"),
+    ("step_closes_early", "if (fill + 1 < m) continue;", "if (fill + 2 < m) continue;"),
+    ("step_overlap_not_kept", "n_ovl[b] = m;", "n_ovl[b] = 0;"),
+    ("step_overlap_not_pooled", "n = n_ovl[b];\n", "n = 0;\n"),
+    ("step_unweighted_norm", "z += wgt;", "z += 1.0;"),
 ]
 
 # Entry-position readings are choices the pages do not fix; the pins cannot catch them.
