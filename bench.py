@@ -6,7 +6,7 @@ prefill workload: csa_compress, csa_index_topk, csa_attend).  Default workload: 
 prefill layer at V4-Flash head shape (B=1, S=8192, H=64, D=512, rope 64, window 128,
 m=4, 2048 entries, H_I=64, d_I=128, top-k 512).
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 1|2|3|4] [--impl reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 0..5] [--impl reference]
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs its own independent layer
 instance (its own seeded sequence), no data-path collective; value = all ranks' tokens
@@ -81,6 +81,14 @@ def algorithmic_work(spec):
     if spec.kind == "csa":
         w["index_bytes"] = spec.B * (spec.S_q * spec.H_I * (spec.d_I + 1) + spec.P * spec.d_I) * e \
             + spec.B * spec.S_q * spec.topk * 4
+    if spec.cache_update:
+        # per compressor (main at D, indexer keys at d_I): the new rows read and stored in the
+        # state (kv + gate), the state rows a closing window reaches back to read (kv + gate),
+        # each closed entry written
+        n_close = (spec.q_pos0 + spec.S_q) // spec.m - spec.q_pos0 // spec.m
+        back = spec.q_pos0 - max(0, (spec.q_pos0 // spec.m - spec.overlap) * spec.m) if n_close else 0
+        rows = 4 * spec.S_q + 2 * back + n_close
+        w["append_bytes"] = spec.B * rows * (spec.D + (spec.d_I if spec.kind == "csa" else 0)) * e
     return w
 
 
@@ -187,6 +195,8 @@ class LayerRunner:
         st = []
         if not s.decode and s.kind != "sliding":
             st.append("compress")
+        if s.cache_update:
+            st.append("append")
         if s.kind == "csa":
             st.append("index")
         st.append("attend")
@@ -196,6 +206,13 @@ class LayerRunner:
         s, i, csa = self.spec, self.inp, self.csa
         if name == "compress":
             csa.csa_compress(i["kv"], i["gate"], s.m, s.overlap, pool=self.pool)
+        elif name == "append":
+            import csa_synth as cs
+            csa.csa_compress_append(cs.kv_new(s, i), i["gate_new"], i["state"], s.q_pos0, s.m,
+                                    s.overlap, pool=self.pool)
+            if s.kind == "csa":
+                csa.csa_compress_append(i["kI_new"], i["gI_new"], i["state_I"], s.q_pos0, s.m,
+                                        s.overlap, pool=i["k_I"])
         elif name == "index":
             csa.csa_index_topk(i["q_I"], i["w"], i["k_I"], s.q_pos0, s.m, s.topk, idx=self.idx,
                                workspace=self.ws_i)
@@ -218,6 +235,7 @@ def src_hash(names):
 
 
 STAGE_SOURCES = {"compress": ["compress.cu", "common.cuh"],
+                 "append": ["compress.cu", "common.cuh"],
                  "index": ["index_topk.cu", "topk.cuh", "index_tc.cu", "umma.cuh", "common.cuh"],
                  "attend": ["attend.cu", "attend_tc.cu", "umma.cuh", "common.cuh"]}
 
@@ -369,9 +387,11 @@ def gpu_arm(args, rank, world, local_rank):
                                          key=lambda x: x[1])
     wk = work[dom_layer]
     dom_spec = specs[dom_layer]
-    if dom_stage == "compress" or (dom_stage == "attend" and (dom_spec.kind == "sliding" or dom_spec.decode)) \
+    if dom_stage in ("compress", "append") \
+            or (dom_stage == "attend" and (dom_spec.kind == "sliding" or dom_spec.decode)) \
             or (dom_stage == "index" and dom_spec.decode):
-        key_b = {"compress": "compress_bytes", "attend": "attend_bytes", "index": "index_bytes"}[dom_stage]
+        key_b = {"compress": "compress_bytes", "attend": "attend_bytes", "index": "index_bytes",
+                 "append": "append_bytes"}[dom_stage]
         achieved = wk[key_b] / (dom_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
@@ -415,7 +435,8 @@ def gpu_arm(args, rank, world, local_rank):
 def workload_name(w, specs):
     return {0: "tiny CSA layer fp32 (S=256)", 1: "CSA prefill bf16 S=8192 (V4-Flash layer shape)",
             2: "HCA prefill bf16 S=65536", 3: "CSA decode bf16 B=64 at 65536 cached tokens",
-            4: "mixed 4-layer stack bf16 S=131072"}[w]
+            4: "mixed 4-layer stack bf16 S=131072",
+            5: "CSA decode step with compressor cache update, bf16 B=64 at 65536 tokens"}[w]
 
 
 def workload_config(w, specs):
@@ -484,15 +505,25 @@ def oracle_sample_run(spec, rows, inp_cpu=None):
     f64 = lambda t: None if t is None else t.double().numpy()
     t0 = time.perf_counter()
     pool = None
+    k_I = f64(inp["k_I"])
     if spec.decode:
         pool = f64(inp["pool"])
+        if spec.cache_update:
+            j0 = spec.q_pos0 // spec.m
+            comps = [(inp["state"], cs.kv_new(spec, inp), inp["gate_new"], pool)]
+            if spec.kind == "csa":
+                comps.append((inp["state_I"], inp["kI_new"], inp["gI_new"], k_I))
+            for state, new_kv, new_g, cache in comps:
+                kh, gh, s0 = cs.ring_history(state, spec.q_pos0, spec.m, spec.overlap)
+                st = oracle.CompressorState.resume(f64(kh), f64(gh), s0, spec.m, spec.overlap)
+                ent = st.append(f64(new_kv), f64(new_g))
+                cache[:, j0:j0 + ent.shape[1]] = ent
     elif spec.kind != "sliding":
         pool = oracle.compress(f64(inp["kv"]), f64(inp["gate"]), spec.m, spec.overlap)
     tpos = np.asarray(rows, dtype=np.int64) + spec.q_pos0
     idx = None
     if spec.kind == "csa":
-        sc = oracle.index_scores(f64(inp["q_I"][:, rows]), f64(inp["w"][:, rows]), f64(inp["k_I"]),
-                                 tpos, spec.m)
+        sc = oracle.index_scores(f64(inp["q_I"][:, rows]), f64(inp["w"][:, rows]), k_I, tpos, spec.m)
         idx, _ = oracle.topk(sc, tpos, spec.m, spec.topk)
     oracle.attend(f64(inp["q"][:, rows]), tpos, f64(inp["kv"]), spec.kv_pos0, pool, spec.m, idx,
                   f64(inp["sink"]), spec.R, spec.base, spec.W, spec.scale,
@@ -566,7 +597,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", type=int, default=1, choices=[0, 1, 2, 3, 4])
+    ap.add_argument("--workload", type=int, default=1, choices=[0, 1, 2, 3, 4, 5])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

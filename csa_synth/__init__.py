@@ -16,8 +16,15 @@ indexer head weights w ~ N(0,1)/sqrt(H_I); sink logits ~ N(0,1) in fp32; every k
 (and every directly generated pool row) RMS-normalised, x / sqrt(mean(x^2) + 1e-6),
 in fp64 before rounding to the storage dtype.
 
+Decode step with the cache update (workload 5): the main compressor's state is the ring of
+the last (1+overlap)*m raw rows before the new token, in the layout csa_compress_append
+documents (row of position p in slot p mod L); its kv rows are the window rows of those
+positions (the same tokens), its gates N(0,1).  The indexer's per-token keys and gates
+(state_I, kI_new, gI_new) and the new token's gate are N(0,1).  The new token's kv row is
+the last row of the window.
+
 Seeds: tensor seed = 1000*workload + 100*layer + tensor_id, tensor ids in the order
-q, kv, gate, q_I, k_I, w, sink, pool.
+q, kv, gate, q_I, k_I, w, sink, pool, gate_new, state, state_I, kI_new, gI_new.
 """
 from __future__ import annotations
 
@@ -27,7 +34,8 @@ from typing import Dict, List, Optional
 
 import torch
 
-TENSOR_IDS = {"q": 0, "kv": 1, "gate": 2, "q_I": 3, "k_I": 4, "w": 5, "sink": 6, "pool": 7}
+TENSOR_IDS = {"q": 0, "kv": 1, "gate": 2, "q_I": 3, "k_I": 4, "w": 5, "sink": 6, "pool": 7,
+              "gate_new": 8, "state": 9, "state_I": 10, "kI_new": 11, "gI_new": 12}
 RMS_EPS = 1e-6
 
 
@@ -39,6 +47,10 @@ class LayerSpec:
     visible entry) or "sliding" (window only, no pool).
     Query i sits at absolute position q_pos0 + i; raw kv row r at kv_pos0 + r.
     decode=True means the pool and k_I are a resident cache (no compressor run).
+    cache_update=True (decode only) adds the compressor cache update to the step: the S_q
+    new tokens (the last S_q window rows, at q_pos0..) go through the main compressor's
+    state and, with their per-token index keys, through the indexer's key compressor;
+    the entries that close are written into the pool and k_I before they are read.
     """
 
     name: str
@@ -60,12 +72,18 @@ class LayerSpec:
     d_I: int = 0
     topk: int = 0
     decode: bool = False
+    cache_update: bool = False
     workload: int = 0
     layer: int = 0
 
     @property
     def overlap(self) -> int:
         return 1 if self.kind == "csa" else 0
+
+    @property
+    def ring(self) -> int:
+        """Rows a compressor state keeps: (1+overlap)*m."""
+        return (1 + self.overlap) * self.m
 
     @property
     def scale(self) -> float:
@@ -104,6 +122,10 @@ CSA_DECODE = LayerSpec(name="csa_decode_b64_ctx65536", dtype="bf16", B=64, S_q=1
                        decode=True, workload=3)
 
 
+CSA_DECODE_STEP = dataclasses.replace(CSA_DECODE, name="csa_decode_step_b64_ctx65536",
+                                      cache_update=True, workload=5)
+
+
 def mixed_stack(S: int = 131072) -> List[LayerSpec]:
     """Four-layer long-context block: CSA, HCA, CSA, sliding-only."""
     return [
@@ -124,6 +146,7 @@ WORKLOADS: Dict[int, List[LayerSpec]] = {
     2: [HCA_PREFILL],
     3: [CSA_DECODE],
     4: mixed_stack(),
+    5: [CSA_DECODE_STEP],
 }
 
 
@@ -163,7 +186,46 @@ def make_inputs(spec: LayerSpec, device="cpu") -> Dict[str, Optional[torch.Tenso
     else:
         out["q_I"] = out["k_I"] = out["w"] = None
     out["sink"] = _randn((spec.H,), spec.seed("sink"), device)
+    if spec.cache_update:
+        assert spec.decode and spec.kind != "sliding" and spec.kv_pos0 + spec.S_kv == spec.q_pos0 + spec.S_q
+        L = spec.ring
+        st = _randn((spec.B, 2, L, spec.D), spec.seed("state"), device)
+        st[:, 0] = _rms_rows(st[:, 0]).float()
+        for p in range(spec.q_pos0 - L, spec.q_pos0):
+            r = p - spec.kv_pos0
+            if p >= 0 and 0 <= r < spec.S_kv:
+                st[:, 0, p % L] = out["kv"][:, r].float()
+        out["state"] = st.to(dt)
+        out["gate_new"] = _randn((spec.B, spec.S_q, spec.D), spec.seed("gate_new"), device).to(dt)
+        if spec.kind == "csa":
+            out["state_I"] = _randn((spec.B, 2, L, spec.d_I), spec.seed("state_I"), device).to(dt)
+            out["kI_new"] = _randn((spec.B, spec.S_q, spec.d_I), spec.seed("kI_new"), device).to(dt)
+            out["gI_new"] = _randn((spec.B, spec.S_q, spec.d_I), spec.seed("gI_new"), device).to(dt)
     return out
+
+
+def stream_rows(B: int, S: int, D: int, dtype: torch.dtype, seed: int, device="cpu"):
+    """Raw rows of S tokens fed to a compressor: kv RMS-normalised N(0,1), gate N(0,1)
+    (seeds `seed` and `seed + 1`)."""
+    kv = _rms_rows(_randn((B, S, D), seed, device)).to(dtype)
+    gate = _randn((B, S, D), seed + 1, device).to(dtype)
+    return kv, gate
+
+
+def kv_new(spec: LayerSpec, inp) -> torch.Tensor:
+    """The new tokens' raw rows in a cache-update step: a view of the window's last S_q rows."""
+    return inp["kv"][:, spec.S_kv - spec.S_q:]
+
+
+def ring_history(state: torch.Tensor, pos0: int, m: int, overlap: int):
+    """Rows of positions [s0, pos0) held by a compressor state [B, 2, L, D] (slot p mod L),
+    s0 the start of the last closed block (overlap) or of the open window (no overlap):
+    (kv rows [B, n, D], gate rows [B, n, D], s0).  Replaying them from s0 into a fresh
+    stateful compressor rebuilds its buffer and overlap block."""
+    L = state.shape[2]
+    s0 = max(0, (pos0 // m - overlap) * m)
+    slots = [p % L for p in range(s0, pos0)]
+    return state[:, 0, slots], state[:, 1, slots], s0
 
 
 def sample_rows(spec: LayerSpec, n_random: int = 256, seed: int = 12345) -> List[int]:

@@ -71,6 +71,44 @@ csa_status_t csa_compress(const void *kv, const void *gate, void *pool, int64_t 
                           void *stream);
 
 /*
+ * csa_compress_append -- decode-time compressor cache update (HF PR #45616 "Compressor/
+ * Indexer statefulness ... per-layer compressor_state and indexer_state (buffer_kv,
+ * buffer_gate, pooled_kv)", "_accumulate_windows and _update_pool ... single cache update
+ * per call"; HF docs model_doc/deepseek_v4 section "Cache layers": buffer / pool / counter,
+ * plus the overlap state for CSA).  The same call serves the main compressor (D = head_dim)
+ * and the indexer's key compressor (D = d_I), each with its own state.
+ *
+ * Appends the raw rows of positions pos0 .. pos0+n_new-1 of every sequence and writes each
+ * pool entry whose window closes among them -- entries j with pos0 <= (j+1)*ratio - 1 <
+ * pos0 + n_new -- with the value csa_compress gives over the whole sequence.  Other pool
+ * entries are not touched.
+ *
+ *   kv_new, gate_new : rows of sequence b at kv_new + b*kv_stride*D (gate: gate_stride),
+ *                      n_new consecutive rows of D elements each; strides are in rows and
+ *                      must be >= n_new when B > 1 (a view of a larger cache is fine)
+ *   state  : [B, 2, L, D], L = (1+overlap)*ratio, csa_compress_state_bytes() bytes, owned
+ *            by the caller: [b,0,p mod L,:] is the kv row of position p, [b,1,p mod L,:]
+ *            its gate.  The call reads the rows of positions [max(0, pos0-L+1), pos0),
+ *            which earlier calls must have stored (every call stores its newest
+ *            min(n_new, L) rows); its initial contents are never read at pos0 == 0.
+ *   pool   : [B, pool_cap, D], or NULL to store rows into the state only (e.g. to seed it
+ *            from the tail of a prefill that csa_compress pooled); requires
+ *            pool_cap >= floor((pos0+n_new)/ratio).
+ *   pos0   : tokens appended so far (the compressor's counter), the same for every
+ *            sequence.
+ * A call that closes more than ~500K entries returns CSA_ERR_UNSUPPORTED (csa_compress is
+ * the prefill path).
+ */
+csa_status_t csa_compress_append(const void *kv_new, const void *gate_new, int64_t kv_stride,
+                                 int64_t gate_stride, void *state, void *pool, int64_t pool_cap,
+                                 int64_t B, int64_t n_new, int64_t pos0, int32_t D,
+                                 int32_t ratio, int32_t overlap, csa_dtype_t dtype, void *stream);
+
+/* Bytes of the state csa_compress_append keeps for these sizes (0 for bad arguments). */
+size_t csa_compress_state_bytes(int64_t B, int32_t D, int32_t ratio, int32_t overlap,
+                                csa_dtype_t dtype);
+
+/*
  * csa_index_topk -- CSA Lightning Indexer and top-k (HF docs model_doc/deepseek_v4
  * section 2.3.1, eq. 13-17 named there; section "Attention mask layout": queries before
  * the first closed window get only the -1 marker).

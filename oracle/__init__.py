@@ -143,6 +143,20 @@ class CompressorState:
         self.counter = np.zeros(B, dtype=np.int64)
         self.n_ovl = np.zeros(B, dtype=np.int64)
 
+    @classmethod
+    def resume(cls, kv_hist, gate_hist, s0: int, m: int, overlap: int) -> "CompressorState":
+        """The state after the rows of positions [s0, s0+n) (kv_hist, gate_hist [B,n,D]),
+        rebuilt by replaying them from s0, a window start (s0 % m == 0) from which the
+        buffer and, with overlap, the last closed block are covered.  Entries that close
+        during the replay are dropped (the first one lacks its own overlap block)."""
+        if s0 % m:
+            raise ValueError("CompressorState.resume: s0 must be a multiple of m")
+        kv = _f64(kv_hist)
+        st = cls(kv.shape[0], kv.shape[2], m, overlap)
+        st.counter[:] = s0
+        st.append(kv, gate_hist)
+        return st
+
     def append(self, kv_new, gate_new) -> np.ndarray:
         """kv_new, gate_new [B,n,D] (the next n tokens) -> the entries whose windows close
         among them, [B, n_closed, D] in closing order (n_closed may be 0)."""

@@ -14,7 +14,8 @@ from typing import Optional
 
 import torch
 
-__all__ = ["csa_compress", "csa_index_topk", "csa_attend", "hca_attend",
+__all__ = ["csa_compress", "csa_compress_append", "csa_compress_state_bytes",
+           "csa_compress_state", "csa_index_topk", "csa_attend", "hca_attend",
            "csa_index_topk_workspace_bytes", "csa_attend_workspace_bytes", "library_path",
            "load_library", "launch_count", "device_status", "CsaError", "CSA_F32", "CSA_BF16"]
 
@@ -45,6 +46,10 @@ def load_library():
     lib = ctypes.CDLL(_LIB_PATH)
     vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
     lib.csa_compress.argtypes = [vp, vp, vp, i64, i64, i32, i32, i32, ctypes.c_int, vp]
+    lib.csa_compress_append.argtypes = [vp, vp, i64, i64, vp, vp, i64, i64, i64, i64, i32, i32,
+                                        i32, ctypes.c_int, vp]
+    lib.csa_compress_state_bytes.argtypes = [i64, i32, i32, i32, ctypes.c_int]
+    lib.csa_compress_state_bytes.restype = sz
     lib.csa_index_topk.argtypes = [vp, vp, vp, i64, i64, i64, i64, i32, i32, i32, i32, vp, vp, vp,
                                    sz, ctypes.c_int, vp]
     lib.csa_index_topk_workspace_bytes.argtypes = [i64, i64, i64, i64, i32, i32, i32, i32,
@@ -58,7 +63,7 @@ def load_library():
     lib.csa_attend_workspace_bytes.argtypes = [i32, i64, i64, i64, i64, i32, i32, i32,
                                                ctypes.c_int]
     lib.csa_attend_workspace_bytes.restype = sz
-    for f in ("csa_compress", "csa_index_topk", "csa_attend", "hca_attend"):
+    for f in ("csa_compress", "csa_compress_append", "csa_index_topk", "csa_attend", "hca_attend"):
         getattr(lib, f).restype = ctypes.c_int
     lib.csa_last_error.restype = ctypes.c_char_p
     lib.csa_version.restype = ctypes.c_char_p
@@ -127,6 +132,54 @@ def csa_compress(kv: torch.Tensor, gate: torch.Tensor, ratio: int, overlap: bool
         pool = torch.empty((B, P, D), dtype=kv.dtype, device=kv.device)
     _call("csa_compress", _ptr(kv), _ptr(gate), _ptr(pool), B, S, D, ratio, int(bool(overlap)),
           _dtype_code(kv), _stream(stream))
+    return pool
+
+
+def _rows_ptr(t: torch.Tensor, D: int):
+    """Pointer and sequence stride (in rows) of a [B, n, D] tensor whose rows are dense
+    (a slice of a larger cache along n is fine)."""
+    if not t.is_cuda:
+        raise ValueError("tensors must be on a CUDA device")
+    B, n, d = t.shape
+    if d != D or t.stride(2) != 1 or (n > 1 and t.stride(1) != D):
+        raise ValueError("rows must be dense [.., D] vectors with D=%d" % D)
+    if B > 1 and t.stride(0) % D != 0:
+        raise ValueError("sequence stride must be a whole number of rows")
+    return ctypes.c_void_p(t.data_ptr()), (t.stride(0) // D if B > 1 else n)
+
+
+def csa_compress_state_bytes(B: int, D: int, ratio: int, overlap: bool,
+                             dtype=torch.bfloat16) -> int:
+    code = CSA_F32 if dtype == torch.float32 else CSA_BF16
+    return int(load_library().csa_compress_state_bytes(B, D, ratio, int(bool(overlap)), code))
+
+
+def csa_compress_state(B: int, D: int, ratio: int, overlap: bool, dtype=torch.bfloat16,
+                       device="cuda") -> torch.Tensor:
+    """A zeroed state [B, 2, (1+overlap)*ratio, D] for csa_compress_append."""
+    L = (1 + int(bool(overlap))) * ratio
+    return torch.zeros((B, 2, L, D), dtype=dtype, device=device)
+
+
+def csa_compress_append(kv_new: torch.Tensor, gate_new: torch.Tensor, state: torch.Tensor,
+                        pos0: int, ratio: int, overlap: bool,
+                        pool: Optional[torch.Tensor] = None, stream=None) -> Optional[torch.Tensor]:
+    """Append rows kv_new, gate_new [B, n, D] at positions pos0.. to the compressor state
+    and write the entries that close among them into pool [B, cap, D] (see include/csa.h)."""
+    B, n, D = kv_new.shape
+    if gate_new.shape != kv_new.shape or gate_new.dtype != kv_new.dtype:
+        raise ValueError("gate_new must match kv_new in shape and dtype")
+    L = (1 + int(bool(overlap))) * ratio
+    if tuple(state.shape) != (B, 2, L, D) or state.dtype != kv_new.dtype:
+        raise ValueError("state must be [B, 2, %d, D] of the rows' dtype" % L)
+    if pool is not None and (pool.dim() != 3 or pool.shape[0] != B or pool.shape[2] != D
+                             or pool.dtype != kv_new.dtype):
+        raise ValueError("pool must be [B, cap, D] of the rows' dtype")
+    kp, ks = _rows_ptr(kv_new, D)
+    gp, gs = _rows_ptr(gate_new, D)
+    _call("csa_compress_append", kp, gp, ks, gs, _ptr(state), _ptr(pool),
+          0 if pool is None else pool.shape[1], B, n, pos0, D, ratio, int(bool(overlap)),
+          _dtype_code(kv_new), _stream(stream))
     return pool
 
 

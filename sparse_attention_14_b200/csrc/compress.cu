@@ -249,6 +249,99 @@ csa_status_t launch_compress(const T *kv, const T *gate, T *pool, int64_t B, int
     return CSA_OK;
 }
 
+// ---------------------------------------------------------------- decode-time cache update
+// HF PR #45616 "Compressor/Indexer statefulness ... per-layer compressor_state and
+// indexer_state (buffer_kv, buffer_gate, pooled_kv)" and "_accumulate_windows and
+// _update_pool ... single cache update per call"; HF docs "Cache layers" (buffer / pool /
+// counter, plus the CSA overlap state).
+//
+// The state of a sequence is a ring of its last L = (1+overlap)*ratio raw rows, kv and
+// gate, the row of position p in slot p mod L: exactly the rows that a window closing in
+// a later call can still reach (a window closing at t >= pos0 starts at or after
+// pos0 - L + 1).  The token counter is the caller's pos0.
+//
+// Grid (channel blocks, entry chunks, B); a thread owns 8 channels of one sequence.  Chunk
+// y pools entries j0 + [y*kAppendChunk, (y+1)*kAppendChunk), reading each window row from
+// the ring (positions before pos0) or from the new rows; then chunk 0 stores the newest
+// min(n_new, L) rows into the ring.  Only the first two entries of a call can reach back
+// before pos0 (from the third on, lo = (j - overlap)*ratio >= pos0); they belong to chunk
+// 0, whose threads read their own channels of the ring before overwriting them, so no
+// other block ever touches the ring.
+constexpr int kAppendChunk = 8;
+
+template <typename T>
+__global__ void __launch_bounds__(128) compress_append_kernel(
+    const T *__restrict__ kv_new, const T *__restrict__ gate_new, int64_t kv_stride,
+    int64_t gate_stride, T *__restrict__ state, T *__restrict__ pool, int64_t pool_cap,
+    int64_t n_new, int64_t pos0, int D, int ratio, int overlap, int64_t j0, int64_t n_close) {
+    const int g8 = blockIdx.x * blockDim.x + threadIdx.x;
+    if (g8 >= D / 8) return;
+    const int64_t b = blockIdx.z;
+    const int64_t L = (int64_t)(1 + overlap) * ratio;
+    T *ring_kv = state + (b * 2) * L * D + g8 * 8;
+    T *ring_g = state + (b * 2 + 1) * L * D + g8 * 8;
+    const T *nkv = kv_new + b * kv_stride * D + g8 * 8;
+    const T *ng = gate_new + b * gate_stride * D + g8 * 8;
+    const int64_t c0 = (int64_t)blockIdx.y * kAppendChunk;
+    const int64_t c1 = c0 + kAppendChunk < n_close ? c0 + kAppendChunk : n_close;
+    for (int64_t c = c0; c < c1; ++c) {
+        const int64_t j = j0 + c;
+        int64_t lo = (j - overlap) * ratio;
+        if (lo < 0) lo = 0;
+        const int64_t hi = (j + 1) * ratio;   // <= pos0 + n_new
+        SoftPool8 st;
+        st.init();
+        for (int64_t s = lo; s < hi; ++s) {
+            float gv[8], vv[8];
+            if (s >= pos0) {
+                load8(ng + (s - pos0) * D, gv);
+                load8(nkv + (s - pos0) * D, vv);
+            } else {
+                const int64_t slot = s % L;
+                load8(ring_g + slot * D, gv);
+                load8(ring_kv + slot * D, vv);
+            }
+            st.add(gv, vv);
+        }
+        float o[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) o[k] = st.num[k] / st.den[k];
+        store8(pool + (b * pool_cap + j) * D + g8 * 8, o);
+    }
+    if (blockIdx.y != 0) return;
+    int64_t q0 = pos0 + n_new - L;
+    if (q0 < pos0) q0 = pos0;
+    for (int64_t q = q0; q < pos0 + n_new; ++q) {
+        const int64_t slot = q % L;
+        float v[8];
+        load8(nkv + (q - pos0) * D, v);
+        store8(ring_kv + slot * D, v);   // exact: the values came from T
+        load8(ng + (q - pos0) * D, v);
+        store8(ring_g + slot * D, v);
+    }
+}
+
+template <typename T>
+csa_status_t launch_append(const T *kv_new, const T *gate_new, int64_t kv_stride,
+                           int64_t gate_stride, T *state, T *pool, int64_t pool_cap, int64_t B,
+                           int64_t n_new, int64_t pos0, int D, int ratio, int overlap,
+                           cudaStream_t st) {
+    const int64_t j0 = pos0 / ratio;
+    const int64_t n_close = pool ? (pos0 + n_new) / ratio - j0 : 0;
+    const int groups = D / 8;
+    const int bx = groups < 128 ? groups : 128;
+    const int64_t gy = n_close > 0 ? ceil_div(n_close, kAppendChunk) : 1;
+    CSA_REQUIRE(gy < 65536 && B < 65536, CSA_ERR_UNSUPPORTED,
+                "csa_compress_append: grid too large (%lld entries, B=%lld); use csa_compress "
+                "for long prefixes", (long long)n_close, (long long)B);
+    dim3 grid((unsigned)ceil_div(groups, bx), (unsigned)gy, (unsigned)B);
+    compress_append_kernel<T><<<grid, bx, 0, st>>>(kv_new, gate_new, kv_stride, gate_stride,
+                                                   state, pool, pool_cap, n_new, pos0, D, ratio,
+                                                   overlap, j0, n_close);
+    CSA_CHECK_LAUNCH("csa_compress_append");
+    return CSA_OK;
+}
+
 }  // namespace
 }  // namespace csa
 
@@ -274,4 +367,58 @@ extern "C" csa_status_t csa_compress(const void *kv, const void *gate, void *poo
                                       D, ratio, overlap, P, st);
     return launch_compress<__nv_bfloat16>((const __nv_bfloat16 *)kv, (const __nv_bfloat16 *)gate,
                                           (__nv_bfloat16 *)pool, B, S, D, ratio, overlap, P, st);
+}
+
+extern "C" size_t csa_compress_state_bytes(int64_t B, int32_t D, int32_t ratio, int32_t overlap,
+                                           csa_dtype_t dtype) {
+    if (B < 0 || D < 8 || D > 1024 || D % 8 != 0 || ratio < 1 || (overlap != 0 && overlap != 1) ||
+        (dtype != CSA_F32 && dtype != CSA_BF16))
+        return 0;
+    const size_t e = dtype == CSA_F32 ? 4 : 2;
+    return (size_t)B * 2 * (size_t)(1 + overlap) * (size_t)ratio * (size_t)D * e;
+}
+
+extern "C" csa_status_t csa_compress_append(const void *kv_new, const void *gate_new,
+                                            int64_t kv_stride, int64_t gate_stride, void *state,
+                                            void *pool, int64_t pool_cap, int64_t B,
+                                            int64_t n_new, int64_t pos0, int32_t D, int32_t ratio,
+                                            int32_t overlap, csa_dtype_t dtype, void *stream) {
+    using namespace csa;
+    clear_error();
+    CSA_REQUIRE(B >= 0 && n_new >= 0 && pos0 >= 0, CSA_ERR_INVALID_ARG,
+                "csa_compress_append: negative B, n_new or pos0");
+    CSA_REQUIRE(D >= 8 && D <= 1024 && D % 8 == 0, CSA_ERR_INVALID_ARG,
+                "csa_compress_append: D=%d must be a multiple of 8 in [8, 1024]", D);
+    CSA_REQUIRE(ratio >= 1, CSA_ERR_INVALID_ARG, "csa_compress_append: ratio=%d must be >= 1", ratio);
+    CSA_REQUIRE(overlap == 0 || overlap == 1, CSA_ERR_INVALID_ARG,
+                "csa_compress_append: overlap must be 0 or 1");
+    CSA_REQUIRE(dtype == CSA_F32 || dtype == CSA_BF16, CSA_ERR_INVALID_ARG,
+                "csa_compress_append: bad dtype");
+    CSA_REQUIRE(pos0 <= (int64_t)1 << 40 && n_new <= (int64_t)1 << 40, CSA_ERR_INVALID_ARG,
+                "csa_compress_append: pos0 or n_new out of range");
+    if (B == 0 || n_new == 0) return CSA_OK;
+    CSA_REQUIRE(B == 1 || (kv_stride >= n_new && gate_stride >= n_new), CSA_ERR_INVALID_ARG,
+                "csa_compress_append: sequence strides (%lld, %lld rows) must be >= n_new=%lld",
+                (long long)kv_stride, (long long)gate_stride, (long long)n_new);
+    CSA_REQUIRE(kv_stride >= 0 && gate_stride >= 0, CSA_ERR_INVALID_ARG,
+                "csa_compress_append: negative stride");
+    CSA_REQUIRE(kv_new && gate_new && state, CSA_ERR_INVALID_ARG, "csa_compress_append: null pointer");
+    if (pool) {
+        const int64_t need = (pos0 + n_new) / ratio;
+        CSA_REQUIRE(pool_cap >= need, CSA_ERR_INVALID_ARG,
+                    "csa_compress_append: pool_cap=%lld < %lld entries closed by position %lld",
+                    (long long)pool_cap, (long long)need, (long long)(pos0 + n_new - 1));
+    }
+    CSA_REQUIRE(aligned(kv_new, 16) && aligned(gate_new, 16) && aligned(state, 16) &&
+                    (!pool || aligned(pool, 16)),
+                CSA_ERR_INVALID_ARG, "csa_compress_append: tensors must be 16-byte aligned");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (dtype == CSA_F32)
+        return launch_append<float>((const float *)kv_new, (const float *)gate_new, kv_stride,
+                                    gate_stride, (float *)state, (float *)pool, pool_cap, B, n_new,
+                                    pos0, D, ratio, overlap, st);
+    return launch_append<__nv_bfloat16>((const __nv_bfloat16 *)kv_new,
+                                        (const __nv_bfloat16 *)gate_new, kv_stride, gate_stride,
+                                        (__nv_bfloat16 *)state, (__nv_bfloat16 *)pool, pool_cap, B,
+                                        n_new, pos0, D, ratio, overlap, st);
 }

@@ -13,6 +13,7 @@ from __future__ import annotations
 import numpy as np
 import torch
 
+import csa_synth as cs
 import oracle
 import sparse_attention_14_b200 as csa
 
@@ -69,6 +70,16 @@ class GpuLayer:
         s, i = self.spec, self.inp
         return csa.csa_compress(i["kv"], i["gate"], s.m, s.overlap)
 
+    def append(self):
+        """Decode-time cache update: the new tokens into the main compressor state (closed
+        entries into the pool) and their index keys into the indexer's (into k_I)."""
+        s, i = self.spec, self.inp
+        csa.csa_compress_append(cs.kv_new(s, i), i["gate_new"], i["state"], s.q_pos0, s.m,
+                                s.overlap, pool=i["pool"])
+        if s.kind == "csa":
+            csa.csa_compress_append(i["kI_new"], i["gI_new"], i["state_I"], s.q_pos0, s.m,
+                                    s.overlap, pool=i["k_I"])
+
     def index(self, want_scores=True):
         s, i = self.spec, self.inp
         return csa.csa_index_topk(i["q_I"], i["w"], i["k_I"], s.q_pos0, s.m, s.topk,
@@ -81,6 +92,53 @@ class GpuLayer:
                                   s.base, s.W, s.m, s.scale)
         return csa.hca_attend(i["q"], i["kv"], s.kv_pos0, pool if s.kind == "hca" else None,
                               i["sink"], s.q_pos0, s.R, s.base, s.W, s.m, s.scale)
+
+
+def oracle_cache_update(spec, inp):
+    """The oracle's stateful compressors, rebuilt from the step's input states, fed the
+    new tokens: [(cache key, first entry j0, entries [B, n, D]), ...] for the main
+    compressor ("pool") and, for CSA, the indexer's key compressor ("k_I")."""
+    comps = [("state", cs.kv_new(spec, inp), "gate_new", "pool")]
+    if spec.kind == "csa":
+        comps.append(("state_I", inp["kI_new"], "gI_new", "k_I"))
+    out = []
+    for st_key, new, g_key, cache in comps:
+        kh, gh, s0 = cs.ring_history(inp[st_key], spec.q_pos0, spec.m, spec.overlap)
+        st = oracle.CompressorState.resume(to_np(kh), to_np(gh), s0, spec.m, spec.overlap)
+        out.append((cache, spec.q_pos0 // spec.m, st.append(to_np(new), to_np(inp[g_key]))))
+    return out
+
+
+def gpu_cache_update_checked(spec, inp):
+    """Run the step's cache update on the GPU (csa_compress_append on the main and the
+    indexer state) and check it: the closed entries against the oracle, every other cache
+    row near them unchanged, the new rows stored in their state slots bit for bit."""
+    expected = oracle_cache_update(spec, inp)
+    L = spec.ring
+    keep = {}
+    for cache, j0, ent in expected:
+        lo, hi = max(0, j0 - 3), min(inp[cache].shape[1], j0 + ent.shape[1] + 3)
+        keep[cache] = (lo, hi, inp[cache][:, lo:hi].clone())
+    GpuLayer(spec, inp).append()
+    torch.cuda.synchronize()
+    for cache, j0, ent in expected:
+        n = ent.shape[1]
+        assert n == (spec.q_pos0 + spec.S_q) // spec.m - spec.q_pos0 // spec.m
+        if n:
+            assert rel_err(to_np(inp[cache][:, j0:j0 + n]), ent) <= TOL[spec.dtype], cache
+        lo, hi, before = keep[cache]
+        after = inp[cache][:, lo:hi]
+        for r in range(hi - lo):
+            if not (j0 <= lo + r < j0 + n):
+                assert torch.equal(after[:, r], before[:, r]), (cache, lo + r)
+    news = [("state", cs.kv_new(spec, inp), inp["gate_new"])]
+    if spec.kind == "csa":
+        news.append(("state_I", inp["kI_new"], inp["gI_new"]))
+    for st_key, kv_rows, g_rows in news:
+        for i in range(max(0, spec.S_q - L), spec.S_q):
+            slot = (spec.q_pos0 + i) % L
+            assert torch.equal(inp[st_key][:, 0, slot], kv_rows[:, i]), (st_key, i)
+            assert torch.equal(inp[st_key][:, 1, slot], g_rows[:, i]), (st_key, i)
 
 
 def oracle_pool(spec, inp):

@@ -60,6 +60,30 @@ def test_compress_rejects(lib):
     assert lib.csa_compress(None, None, None, 0, 64, 64, 4, 1, 1, None) == 0
 
 
+def test_compress_append_rejects(lib):
+    args = lambda **kw: [kw.get("kv", FAKE), kw.get("g", FAKE), kw.get("ks", 4), kw.get("gs", 4),
+                         kw.get("state", FAKE), kw.get("pool", FAKE), kw.get("cap", 64),
+                         kw.get("B", 2), kw.get("n", 4), kw.get("pos", 8), kw.get("D", 64),
+                         kw.get("ratio", 4), kw.get("overlap", 1), kw.get("dtype", 1), None]
+    assert lib.csa_compress_append(*args(D=60)) == -1
+    assert lib.csa_compress_append(*args(ratio=0)) == -1
+    assert lib.csa_compress_append(*args(overlap=2)) == -1
+    assert lib.csa_compress_append(*args(pos=-1)) == -1
+    assert lib.csa_compress_append(*args(n=-1)) == -1
+    assert lib.csa_compress_append(*args(dtype=5)) == -1
+    assert lib.csa_compress_append(*args(ks=3)) == -1          # sequences would overlap
+    assert lib.csa_compress_append(*args(state=None)) == -1
+    assert lib.csa_compress_append(*args(kv=MIS)) == -1
+    # entries up to position 11 close 3 entries: a 2-entry pool is too short
+    assert lib.csa_compress_append(*args(cap=2)) == -1
+    assert "pool_cap" in _err(lib)
+    assert lib.csa_compress_append(*args(n=0)) == 0
+    assert lib.csa_compress_append(*args(B=0)) == 0
+    assert lib.csa_compress_state_bytes(3, 64, 4, 1, 1) == 3 * 2 * 8 * 64 * 2
+    assert lib.csa_compress_state_bytes(3, 512, 128, 0, 0) == 3 * 2 * 128 * 512 * 4
+    assert lib.csa_compress_state_bytes(3, 60, 4, 1, 1) == 0
+
+
 def test_index_topk_rejects(lib):
     args = lambda **kw: [kw.get("q", FAKE), kw.get("w", FAKE), kw.get("k", FAKE), kw.get("B", 1),
                          kw.get("S", 8), kw.get("pos", 0), kw.get("P", 2), kw.get("HI", 4),

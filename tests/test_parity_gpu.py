@@ -4,14 +4,18 @@ tail); the five full workloads are checked end to end on sampled rows, in the la
 configuration the benchmark times.  Tolerances are in parity_util."""
 from __future__ import annotations
 
+import random
+
 import numpy as np
 import pytest
 import torch
 
 import csa_synth as cs
+import oracle
+import sparse_attention_14_b200 as csa
 from csa_synth import LayerSpec
-from parity_util import (TOL, GpuLayer, check_topk, kk_rows, oracle_attend, oracle_index,
-                         oracle_pool, rel_err, to_np)
+from parity_util import (TOL, GpuLayer, check_topk, gpu_cache_update_checked, kk_rows,
+                         oracle_attend, oracle_index, oracle_pool, rel_err, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -58,6 +62,15 @@ MID = [
     LayerSpec(name="mid_csa_cut_bf16", dtype="bf16", B=1, S_q=4801, S_kv=4801, q_pos0=0,
               kv_pos0=0, H=64, D=512, R=64, base=160000.0, W=128, m=4, P=1200, kind="csa",
               H_I=64, d_I=128, topk=200, workload=89),
+    # decode steps that first run the compressor cache update: three new tokens closing the
+    # last CSA entry (main and indexer keys), and one HCA token closing a 128-token window
+    # whose state reaches back before the attention window
+    LayerSpec(name="mid_decode_step_bf16", dtype="bf16", B=2, S_q=3, S_kv=130, q_pos0=4093,
+              kv_pos0=3966, H=64, D=512, R=64, base=160000.0, W=128, m=4, P=1024, kind="csa",
+              H_I=64, d_I=128, topk=64, decode=True, cache_update=True, workload=85),
+    LayerSpec(name="mid_hca_decode_step_bf16", dtype="bf16", B=2, S_q=1, S_kv=128,
+              q_pos0=2047, kv_pos0=1920, H=64, D=512, R=64, base=160000.0, W=128, m=128, P=16,
+              kind="hca", decode=True, cache_update=True, workload=84),
     # odd shapes: general path
     LayerSpec(name="odd_csa_bf16", dtype="bf16", B=1, S_q=77, S_kv=77, q_pos0=0, kv_pos0=0, H=5,
               D=40, R=8, base=10000.0, W=9, m=3, P=25, kind="csa", H_I=3, d_I=24, topk=7,
@@ -191,6 +204,8 @@ def test_no_kernel_gave_up():
 def _end_to_end(spec, rows, inp=None):
     inp = _inputs(spec) if inp is None else inp
     layer = GpuLayer(spec, inp)
+    if spec.cache_update:
+        gpu_cache_update_checked(spec, inp)
     pool = None
     if spec.decode:
         pool = inp["pool"]
@@ -225,7 +240,7 @@ def test_end_to_end_parity(spec):
     _end_to_end(spec, list(range(spec.S_q)))
 
 
-@pytest.mark.parametrize("workload", [0, 1, 2, 3])
+@pytest.mark.parametrize("workload", [0, 1, 2, 3, 5])
 def test_workload_end_to_end(workload):
     for spec in cs.WORKLOADS[workload]:
         rows = list(range(spec.S_q)) if spec.S_q <= 512 else cs.sample_rows(spec, n_random=96)
@@ -239,3 +254,81 @@ def test_mixed_stack_layer_end_to_end(layer):
     rows = cs.sample_rows(spec, n_random=48)
     _end_to_end(spec, rows)
     torch.cuda.empty_cache()
+
+
+# ----------------------------------------------------------------------------- cache update
+def _chunks(seed, S, m, L):
+    r = random.Random(seed)
+    sizes = [1, 1, 1, 2, max(1, m - 1), m, L, L + 1, 3 * L + 2, 40]
+    out = []
+    while sum(out) < S:
+        out.append(min(r.choice(sizes), S - sum(out)))
+    return out
+
+
+APPEND_CASES = [  # name, dtype, B, S, D, ratio, overlap
+    ("csa_kv_bf16", torch.bfloat16, 3, 203, 512, 4, 1),
+    ("csa_index_keys_bf16", torch.bfloat16, 2, 157, 128, 4, 1),
+    ("hca_kv_bf16", torch.bfloat16, 2, 421, 512, 128, 0),
+    ("csa_kv_f32", torch.float32, 2, 99, 64, 4, 1),
+    ("odd_ratio_f32", torch.float32, 3, 50, 24, 3, 0),
+    ("wide_ratio2_bf16", torch.bfloat16, 1, 37, 1024, 2, 1),
+]
+
+
+@pytest.mark.parametrize("name,dt,B,S,D,ratio,overlap", APPEND_CASES,
+                         ids=[c[0] for c in APPEND_CASES])
+def test_append_stream_parity(name, dt, B, S, D, ratio, overlap):
+    """A token stream fed in calls of 1 .. 3L+2 rows, each a strided view of one buffer:
+    after every call the entries that closed match the oracle's stateful compressor and
+    the rest of the pool is untouched; at the end the whole pool matches the stateless
+    oracle and the state holds the last L rows bit for bit."""
+    seed = 600 + [c[0] for c in APPEND_CASES].index(name)
+    kv, gate = cs.stream_rows(B, S, D, dt, seed, device=DEV)
+    L = (1 + overlap) * ratio
+    tol = TOL["f32" if dt == torch.float32 else "bf16"]
+    state = csa.csa_compress_state(B, D, ratio, overlap, dtype=dt)
+    pool = torch.zeros((B, S // ratio + 2, D), dtype=dt, device=DEV)
+    ora = oracle.CompressorState(B, D, ratio, overlap)
+    kv_h, gate_h = to_np(kv), to_np(gate)
+    pos = 0
+    for n in _chunks(seed, S, ratio, L):
+        csa.csa_compress_append(kv[:, pos:pos + n], gate[:, pos:pos + n], state, pos, ratio,
+                                overlap, pool=pool)
+        ent = ora.append(kv_h[:, pos:pos + n], gate_h[:, pos:pos + n])
+        torch.cuda.synchronize()
+        j0 = pos // ratio
+        if ent.shape[1]:
+            assert rel_err(to_np(pool[:, j0:j0 + ent.shape[1]]), ent) <= tol, (pos, n)
+        assert (pool[:, j0 + ent.shape[1]:] == 0).all(), (pos, n)
+        pos += n
+    assert rel_err(to_np(pool[:, :S // ratio]), oracle.compress(kv_h, gate_h, ratio, overlap)) <= tol
+    for p in range(max(0, S - L), S):
+        assert torch.equal(state[:, 0, p % L], kv[:, p]) and torch.equal(state[:, 1, p % L], gate[:, p])
+
+
+@pytest.mark.parametrize("ratio,overlap,S0,S", [(4, 1, 61, 90), (128, 0, 300, 530), (4, 1, 5, 20)])
+def test_append_resumes_after_prefill(ratio, overlap, S0, S):
+    """Prefill pooled by csa_compress, its tail stored into a state that starts as NaN
+    (a state-only call, no pool), then decode one token per call: every entry matches the
+    stateless oracle over the whole sequence, so the state's initial contents were never
+    read."""
+    B, D, dt = 2, 512, torch.bfloat16
+    kv, gate = cs.stream_rows(B, S, D, dt, 700 + ratio, device=DEV)
+    L = (1 + overlap) * ratio
+    pool = torch.zeros((B, S // ratio, D), dtype=dt, device=DEV)
+    P0 = S0 // ratio
+    if P0:
+        pool[:, :P0] = csa.csa_compress(kv[:, :S0].contiguous(), gate[:, :S0].contiguous(), ratio,
+                                        overlap)
+    state = torch.full((B, 2, L, D), float("nan"), dtype=dt, device=DEV)
+    t = max(0, S0 - L)
+    csa.csa_compress_append(kv[:, t:S0], gate[:, t:S0], state, t, ratio, overlap)
+    for p in range(S0, S):
+        csa.csa_compress_append(kv[:, p:p + 1], gate[:, p:p + 1], state, p, ratio, overlap,
+                                pool=pool)
+    torch.cuda.synchronize()
+    ref = oracle.compress(to_np(kv), to_np(gate), ratio, overlap)
+    got = to_np(pool)
+    assert np.isfinite(got).all()
+    assert rel_err(got, ref) <= TOL["bf16"]
