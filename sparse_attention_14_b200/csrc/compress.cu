@@ -269,6 +269,28 @@ csa_status_t launch_compress(const T *kv, const T *gate, T *pool, int64_t B, int
 // other block ever touches the ring.
 constexpr int kAppendChunk = 8;
 
+// Eight channels of one row kept as raw 16-byte vectors until they are used; kBatch rows
+// of kv and gate per batch hold 64 registers either way.
+template <typename T> struct Raw8;
+template <> struct Raw8<__nv_bfloat16> {
+    static constexpr int kBatch = 8;
+    uint4 u;
+    __device__ __forceinline__ void load(const __nv_bfloat16 *p) { u = *reinterpret_cast<const uint4 *>(p); }
+    __device__ __forceinline__ void get(float *v) const { unpack8(u, v); }
+};
+template <> struct Raw8<float> {
+    static constexpr int kBatch = 4;
+    float4 a, b;
+    __device__ __forceinline__ void load(const float *p) {
+        a = *reinterpret_cast<const float4 *>(p);
+        b = *reinterpret_cast<const float4 *>(p + 4);
+    }
+    __device__ __forceinline__ void get(float *v) const {
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+};
+
 template <typename T>
 __global__ void __launch_bounds__(128) compress_append_kernel(
     const T *__restrict__ kv_new, const T *__restrict__ gate_new, int64_t kv_stride,
@@ -289,23 +311,60 @@ __global__ void __launch_bounds__(128) compress_append_kernel(
         int64_t lo = (j - overlap) * ratio;
         if (lo < 0) lo = 0;
         const int64_t hi = (j + 1) * ratio;   // <= pos0 + n_new
-        SoftPool8 st;
-        st.init();
-        for (int64_t s = lo; s < hi; ++s) {
-            float gv[8], vv[8];
-            if (s >= pos0) {
-                load8(ng + (s - pos0) * D, gv);
-                load8(nkv + (s - pos0) * D, vv);
-            } else {
-                const int64_t slot = s % L;
-                load8(ring_g + slot * D, gv);
-                load8(ring_kv + slot * D, vv);
+        float mx[8], den[8], num[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) { mx[k] = -INFINITY; den[k] = 0.f; num[k] = 0.f; }
+        // the window in batches of kB rows: all loads of a batch in flight together, then one
+        // rescale of the running state and one exponential per row and channel
+        constexpr int kB = Raw8<T>::kBatch;
+        for (int64_t s0 = lo; s0 < hi; s0 += kB) {
+            Raw8<T> rg[kB], rv[kB];
+#pragma unroll
+            for (int k = 0; k < kB; ++k) {
+                const int64_t s = s0 + k;
+                if (s < hi) {
+                    const int64_t off = s >= pos0 ? -1 : (s % L) * D;
+                    rg[k].load(off < 0 ? ng + (s - pos0) * D : ring_g + off);
+                    rv[k].load(off < 0 ? nkv + (s - pos0) * D : ring_kv + off);
+                }
             }
-            st.add(gv, vv);
+            float bm[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) bm[k] = mx[k];
+#pragma unroll
+            for (int k = 0; k < kB; ++k) {
+                if (s0 + k < hi) {
+                    float g[8];
+                    rg[k].get(g);
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) bm[ch] = fmaxf(bm[ch], g[ch]);
+                }
+            }
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                const float a = __expf(mx[ch] - bm[ch]);   // 0 on the first batch (mx = -inf)
+                den[ch] *= a;
+                num[ch] *= a;
+                mx[ch] = bm[ch];
+            }
+#pragma unroll
+            for (int k = 0; k < kB; ++k) {
+                if (s0 + k < hi) {
+                    float g[8], v[8];
+                    rg[k].get(g);
+                    rv[k].get(v);
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        const float e = __expf(g[ch] - mx[ch]);
+                        den[ch] += e;
+                        num[ch] = fmaf(e, v[ch], num[ch]);
+                    }
+                }
+            }
         }
         float o[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) o[k] = st.num[k] / st.den[k];
+        for (int k = 0; k < 8; ++k) o[k] = num[k] / den[k];
         store8(pool + (b * pool_cap + j) * D + g8 * 8, o);
     }
     if (blockIdx.y != 0) return;
