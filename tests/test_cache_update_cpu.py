@@ -81,3 +81,30 @@ def test_oracle_sample_run_includes_the_update():
     spec = _small_step("csa")
     dt = bench.oracle_sample_run(spec, [0])
     assert dt > 0
+
+
+def test_append_window_reach_invariants():
+    """The facts the cache-update kernel's layout rests on, over many calls: entries that
+    close in a call at pos0 are j0 = pos0 // m onwards; each window ends inside the call's
+    rows and starts no earlier than pos0 - L + 1 (so a ring of L rows holds every earlier
+    row it needs); and from the third closing entry on a window starts at or after pos0
+    (so only the first chunk of entries reads the ring)."""
+    rng = np.random.default_rng(5)
+    for _ in range(20000):
+        m = int(rng.integers(1, 160))
+        overlap = int(rng.integers(0, 2))
+        L = (1 + overlap) * m
+        pos0 = int(rng.integers(0, 10 * m + 50))
+        n_new = int(rng.integers(1, 4 * L + 3))
+        j0 = pos0 // m
+        n_close = (pos0 + n_new) // m - j0
+        closing = [j for j in range(j0 - 2, (pos0 + n_new) // m + 2)
+                   if pos0 <= (j + 1) * m - 1 < pos0 + n_new]
+        assert closing == list(range(j0, j0 + n_close))
+        for c, j in enumerate(closing):
+            lo = max(0, (j - overlap) * m)
+            hi = (j + 1) * m
+            assert hi <= pos0 + n_new
+            assert lo >= pos0 - L + 1
+            if c >= 2:
+                assert lo >= pos0
