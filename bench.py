@@ -531,6 +531,13 @@ def oracle_sample_run(spec, rows, inp_cpu=None):
     return time.perf_counter() - t0
 
 
+def compressor_note(spec):
+    """How the sampled oracle run treats the compressor, for the sample description."""
+    if spec.decode:
+        return "cache update in full" if spec.cache_update else "resident pool (no compressor)"
+    return "no compressor" if spec.kind == "sliding" else "compressor in full"
+
+
 def oracle_rows(spec, n):
     # evenly spaced query rows: the same causal mix of window/entry counts as the workload
     S = spec.S_q
@@ -558,8 +565,8 @@ def cpu_baseline(args):
     units = spec.B * len(rows)
     return {"value": round(units / dt, 3), "unit": "tokens/s", "cores": oracle_threads(),
             "kind": "oracle",
-            "sample": "%d of %d query rows (evenly spaced) x B=%d of %s; compressor in full; %.1f s"
-                      % (len(rows), spec.S_q, spec.B, spec.name, dt)}
+            "sample": "%d of %d query rows (evenly spaced) x B=%d of %s; %s; %.1f s"
+                      % (len(rows), spec.S_q, spec.B, spec.name, compressor_note(spec), dt)}
 
 
 def reference_arm(args, rank, world):
@@ -578,8 +585,8 @@ def reference_arm(args, rank, world):
     ms = 1e3 * sum(t) / len(t)
     units = spec.B * len(rows)
     value = units / (ms * 1e-3)
-    sample = "%d of %d query rows (evenly spaced) x B=%d of %s per step; compressor in full" % (
-        len(rows), spec.S_q, spec.B, spec.name)
+    sample = "%d of %d query rows (evenly spaced) x B=%d of %s per step; %s" % (
+        len(rows), spec.S_q, spec.B, spec.name, compressor_note(spec))
     return {"metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
