@@ -10,6 +10,7 @@ Function map (each C function's comment cites the page passage it follows):
   CompressorState.append -> orc_compress_step   stateful (decode) compressor
   n_visible     -> orc_n_visible      causal visibility of compressed entries
   index_scores  -> orc_index_scores   Lightning Indexer score
+  index_scores_rope -> orc_rope_rows + orc_index_scores   the same with indexer RoPE
   topk          -> orc_topk           top-k with -1 marker
   attend        -> orc_attend         sink MQA over window + entries, RoPE, de-rotation
   attend_keys   -> orc_attend_keys    the same for one query over explicit keys
@@ -192,6 +193,20 @@ def index_scores(q_I, w, k_I, tpos, m: int) -> np.ndarray:
     _check(_load().orc_index_scores(_ptr(q_I, _dp), _ptr(w, _dp), _ptr(k_I, _dp), _ptr(tp, _lp),
                                     B, n, P, HI, dI, m, _ptr(out, _dp)), "index_scores")
     return out
+
+
+def index_scores_rope(q_I, w, k_I, tpos, m: int, R: int, base: float) -> np.ndarray:
+    """The Lightning Indexer score with the indexer's own rotary embedding: every head of
+    q_I[t] is rotated at t and every pooled key k_I[j] at j*m (interleaved pairs on the
+    last R channels, orc_rope_rows), then scored as index_scores does."""
+    q = _f64(q_I)
+    k = _f64(k_I)
+    B, n, HI, dI = q.shape
+    P = k.shape[1]
+    tp = np.asarray(tpos, dtype=np.float64)
+    q_rot = rope(q, np.broadcast_to(tp[None, :, None], (B, n, HI)), R, base)
+    k_rot = rope(k, np.broadcast_to((np.arange(P, dtype=np.float64) * m)[None, :], (B, P)), R, base)
+    return index_scores(q_rot, w, k_rot, tpos, m)
 
 
 def topk(scores, tpos, m: int, k: int):

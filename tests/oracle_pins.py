@@ -269,6 +269,45 @@ def pin_indexer_unit_keys_golden():
     assert idx[0, 0].tolist() == g["top2"]
 
 
+def pin_indexer_rope_zero_width_is_plain_indexer():
+    """No rotated channels: the indexer with RoPE is the plain indexer."""
+    rng = _rng(40)
+    q, w, k = rng.standard_normal((2, 5, 3, 8)), rng.standard_normal((2, 5, 3)), rng.standard_normal((2, 6, 8))
+    tpos = [3, 8, 11, 20, 23]
+    np.testing.assert_array_equal(oracle.index_scores_rope(q, w, k, tpos, 4, 0, 10000.0),
+                                  oracle.index_scores(q, w, k, tpos, 4))
+
+
+def pin_indexer_rope_relative_position():
+    """RoPE makes the score a function of t - j*m: moving the query by c*m positions and
+    the keys by c entries (c new entries in front) leaves every score unchanged."""
+    rng = _rng(41)
+    m, c, R, base = 4, 5, 8, 160000.0
+    q, w = rng.standard_normal((1, 3, 2, 16)), rng.standard_normal((1, 3, 2))
+    k = rng.standard_normal((1, 9, 16))
+    tpos = np.array([35, 36, 39])
+    k2 = np.concatenate([rng.standard_normal((1, c, 16)), k], axis=1)
+    s1 = oracle.index_scores_rope(q, w, k, tpos, m, R, base)
+    s2 = oracle.index_scores_rope(q, w, k2, tpos + c * m, m, R, base)
+    np.testing.assert_allclose(s2[:, :, c:], s1, rtol=1e-12, atol=1e-12)
+    # and it is not the plain indexer: the rotation does change the scores
+    assert np.nanmax(np.abs(s1 - oracle.index_scores(q, w, k, tpos, m))) > 1e-3
+
+
+def pin_indexer_rope_two_dim_closed_form():
+    """d_I = R = 2, one head, w = 1 (pair 0 turns by the position itself): q at angle a
+    rotated by t, key j at angle b_j rotated by j*m, so the score is
+    max(0, |q| |k_j| cos(a + t - b_j - j*m))."""
+    m, t, a, qn = 3, 14, 0.3, 1.7
+    b = np.array([0.2, -1.1, 2.5, 0.9])
+    kn = np.array([1.0, 0.5, 2.0, 1.3])
+    q = np.array([qn * math.cos(a), qn * math.sin(a)])[None, None, None]
+    k = np.stack([kn * np.cos(b), kn * np.sin(b)], axis=-1)[None]
+    sc = oracle.index_scores_rope(q, np.ones((1, 1, 1)), k, [t], m, 2, 10000.0)[0, 0]
+    want = [max(0.0, qn * kn[j] * math.cos(a + t - b[j] - j * m)) for j in range(4)]
+    np.testing.assert_allclose(sc, want, rtol=1e-12, atol=1e-12)
+
+
 def pin_indexer_single_head_ranking():
     """H_I=1, w=1: the ranking is that of ReLU(q.k) (dot products from numpy matmul)."""
     r = _rng(7)
