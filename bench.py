@@ -6,7 +6,7 @@ prefill workload: csa_compress, csa_index_topk, csa_attend).  Default workload: 
 prefill layer at V4-Flash head shape (B=1, S=8192, H=64, D=512, rope 64, window 128,
 m=4, 2048 entries, H_I=64, d_I=128, top-k 512).
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 0..5] [--impl reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 0..6] [--impl reference]
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs its own independent layer
 instance (its own seeded sequence), no data-path collective; value = all ranks' tokens
@@ -81,6 +81,11 @@ def algorithmic_work(spec):
     if spec.kind == "csa":
         w["index_bytes"] = spec.B * (spec.S_q * spec.H_I * (spec.d_I + 1) + spec.P * spec.d_I) * e \
             + spec.B * spec.S_q * spec.topk * 4
+    if spec.pool_index_keys:
+        w["compress_I_bytes"] = spec.B * (2 * spec.S_kv * spec.d_I + spec.P * spec.d_I) * e
+    if spec.index_rope:
+        # every indexer query head and every pooled key read and written once
+        w["rope_I_bytes"] = 2 * spec.B * (spec.S_q * spec.H_I + spec.P) * spec.d_I * e
     if spec.cache_update:
         # per compressor (main at D, indexer keys at d_I): the new rows read and stored in the
         # state (kv + gate), the state rows a closing window reaches back to read (kv + gate),
@@ -182,6 +187,10 @@ class LayerRunner:
         self.idx = torch.empty((s.B, s.S_q, s.topk), dtype=torch.int32, device=device) \
             if s.kind == "csa" else None
         self.out = torch.empty_like(self.inp["q"])
+        self.k_I = torch.empty((s.B, s.P, s.d_I), dtype=dt, device=device) \
+            if s.pool_index_keys else self.inp["k_I"]
+        self.q_I = torch.empty_like(self.inp["q_I"]) if s.index_rope else self.inp["q_I"]
+        self.k_I_rot = torch.empty_like(self.k_I) if s.index_rope else self.k_I
         wsi = csa.csa_index_topk_workspace_bytes(s.B, s.S_q, s.q_pos0, s.P, s.H_I, s.d_I, s.m,
                                                  s.topk, dt) \
             if s.kind == "csa" else 0
@@ -195,6 +204,10 @@ class LayerRunner:
         st = []
         if not s.decode and s.kind != "sliding":
             st.append("compress")
+        if s.pool_index_keys:
+            st.append("compress_I")
+        if s.index_rope:
+            st.append("rope_I")
         if s.cache_update:
             st.append("append")
         if s.kind == "csa":
@@ -206,6 +219,11 @@ class LayerRunner:
         s, i, csa = self.spec, self.inp, self.csa
         if name == "compress":
             csa.csa_compress(i["kv"], i["gate"], s.m, s.overlap, pool=self.pool)
+        elif name == "compress_I":
+            csa.csa_compress(i["kI_tok"], i["gI_tok"], s.m, s.overlap, pool=self.k_I)
+        elif name == "rope_I":
+            csa.csa_rope_rows(i["q_I"], s.q_pos0, s.H_I, s.S_q, 1, s.index_rope, s.base, out=self.q_I)
+            csa.csa_rope_rows(self.k_I, 0, 1, s.P, s.m, s.index_rope, s.base, out=self.k_I_rot)
         elif name == "append":
             import csa_synth as cs
             csa.csa_compress_append(cs.kv_new(s, i), i["gate_new"], i["state"], s.q_pos0, s.m,
@@ -214,7 +232,7 @@ class LayerRunner:
                 csa.csa_compress_append(i["kI_new"], i["gI_new"], i["state_I"], s.q_pos0, s.m,
                                         s.overlap, pool=i["k_I"])
         elif name == "index":
-            csa.csa_index_topk(i["q_I"], i["w"], i["k_I"], s.q_pos0, s.m, s.topk, idx=self.idx,
+            csa.csa_index_topk(self.q_I, i["w"], self.k_I_rot, s.q_pos0, s.m, s.topk, idx=self.idx,
                                workspace=self.ws_i)
         elif s.kind == "csa":
             csa.csa_attend(i["q"], i["kv"], s.kv_pos0, self.pool, self.idx, i["sink"], s.q_pos0, s.R,
@@ -236,6 +254,8 @@ def src_hash(names):
 
 STAGE_SOURCES = {"compress": ["compress.cu", "common.cuh"],
                  "append": ["compress.cu", "common.cuh"],
+                 "compress_I": ["compress.cu", "common.cuh"],
+                 "rope_I": ["rope.cu", "common.cuh"],
                  "index": ["index_topk.cu", "topk.cuh", "index_tc.cu", "umma.cuh", "common.cuh"],
                  "attend": ["attend.cu", "attend_tc.cu", "umma.cuh", "common.cuh"]}
 
@@ -387,11 +407,12 @@ def gpu_arm(args, rank, world, local_rank):
                                          key=lambda x: x[1])
     wk = work[dom_layer]
     dom_spec = specs[dom_layer]
-    if dom_stage in ("compress", "append") \
+    if dom_stage in ("compress", "append", "compress_I", "rope_I") \
             or (dom_stage == "attend" and (dom_spec.kind == "sliding" or dom_spec.decode)) \
             or (dom_stage == "index" and dom_spec.decode):
         key_b = {"compress": "compress_bytes", "attend": "attend_bytes", "index": "index_bytes",
-                 "append": "append_bytes"}[dom_stage]
+                 "append": "append_bytes", "compress_I": "compress_I_bytes",
+                 "rope_I": "rope_I_bytes"}[dom_stage]
         achieved = wk[key_b] / (dom_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
@@ -436,7 +457,8 @@ def workload_name(w, specs):
     return {0: "tiny CSA layer fp32 (S=256)", 1: "CSA prefill bf16 S=8192 (V4-Flash layer shape)",
             2: "HCA prefill bf16 S=65536", 3: "CSA decode bf16 B=64 at 65536 cached tokens",
             4: "mixed 4-layer stack bf16 S=131072",
-            5: "CSA decode step with compressor cache update, bf16 B=64 at 65536 tokens"}[w]
+            5: "CSA decode step with compressor cache update, bf16 B=64 at 65536 tokens",
+            6: "CSA prefill bf16 S=8192 with the indexer key path (pooled index keys, indexer RoPE 64)"}[w]
 
 
 def workload_config(w, specs):
@@ -445,7 +467,8 @@ def workload_config(w, specs):
     return {"workload": workload_name(w, specs), "B": spec0.B, "S": spec0.S_q, "H": spec0.H,
             "D": spec0.D, "rope_dim": spec0.R, "window": spec0.W, "layers": [s.kind for s in specs],
             "m": [s.m for s in specs], "P": [s.P for s in specs], "topk": spec0.topk,
-            "H_I": spec0.H_I, "d_I": spec0.d_I, "parallelism": "independent layer instance per GPU"}
+            "H_I": spec0.H_I, "d_I": spec0.d_I, "index_rope": spec0.index_rope,
+            "parallelism": "independent layer instance per GPU"}
 
 
 def e2e_arm(args, runners, stage_names, stream, world, dev):
@@ -505,7 +528,8 @@ def oracle_sample_run(spec, rows, inp_cpu=None):
     f64 = lambda t: None if t is None else t.double().numpy()
     t0 = time.perf_counter()
     pool = None
-    k_I = f64(inp["k_I"])
+    k_I = oracle.compress(f64(inp["kI_tok"]), f64(inp["gI_tok"]), spec.m, spec.overlap) \
+        if spec.pool_index_keys else f64(inp["k_I"])
     if spec.decode:
         pool = f64(inp["pool"])
         if spec.cache_update:
@@ -523,7 +547,11 @@ def oracle_sample_run(spec, rows, inp_cpu=None):
     tpos = np.asarray(rows, dtype=np.int64) + spec.q_pos0
     idx = None
     if spec.kind == "csa":
-        sc = oracle.index_scores(f64(inp["q_I"][:, rows]), f64(inp["w"][:, rows]), k_I, tpos, spec.m)
+        if spec.index_rope:
+            sc = oracle.index_scores_rope(f64(inp["q_I"][:, rows]), f64(inp["w"][:, rows]), k_I, tpos,
+                                          spec.m, spec.index_rope, spec.base)
+        else:
+            sc = oracle.index_scores(f64(inp["q_I"][:, rows]), f64(inp["w"][:, rows]), k_I, tpos, spec.m)
         idx, _ = oracle.topk(sc, tpos, spec.m, spec.topk)
     oracle.attend(f64(inp["q"][:, rows]), tpos, f64(inp["kv"]), spec.kv_pos0, pool, spec.m, idx,
                   f64(inp["sink"]), spec.R, spec.base, spec.W, spec.scale,
@@ -604,7 +632,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", type=int, default=1, choices=[0, 1, 2, 3, 4, 5])
+    ap.add_argument("--workload", type=int, default=1, choices=[0, 1, 2, 3, 4, 5, 6])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

@@ -24,7 +24,12 @@ positions (the same tokens), its gates N(0,1).  The indexer's per-token keys and
 the last row of the window.
 
 Seeds: tensor seed = 1000*workload + 100*layer + tensor_id, tensor ids in the order
-q, kv, gate, q_I, k_I, w, sink, pool, gate_new, state, state_I, kI_new, gI_new.
+q, kv, gate, q_I, k_I, w, sink, pool, gate_new, state, state_I, kI_new, gI_new, kI_tok,
+gI_tok.
+
+Prefill with the indexer's key path (workload 6): instead of pooled k_I, per-token index
+keys kI_tok (RMS-normalised N(0,1) rows, as the indexer's kv_norm leaves them) and their
+gate logits gI_tok (N(0,1)), both [B,S,d_I].
 """
 from __future__ import annotations
 
@@ -35,7 +40,8 @@ from typing import Dict, List, Optional
 import torch
 
 TENSOR_IDS = {"q": 0, "kv": 1, "gate": 2, "q_I": 3, "k_I": 4, "w": 5, "sink": 6, "pool": 7,
-              "gate_new": 8, "state": 9, "state_I": 10, "kI_new": 11, "gI_new": 12}
+              "gate_new": 8, "state": 9, "state_I": 10, "kI_new": 11, "gI_new": 12,
+              "kI_tok": 13, "gI_tok": 14}
 RMS_EPS = 1e-6
 
 
@@ -51,6 +57,9 @@ class LayerSpec:
     new tokens (the last S_q window rows, at q_pos0..) go through the main compressor's
     state and, with their per-token index keys, through the indexer's key compressor;
     the entries that close are written into the pool and k_I before they are read.
+    pool_index_keys=True (prefill CSA) pools k_I in the step from per-token index keys
+    by the same gated compressor; index_rope > 0 rotates that many trailing channels of
+    every indexer query head (at t) and pooled key (at j*m) before scoring.
     """
 
     name: str
@@ -73,6 +82,8 @@ class LayerSpec:
     topk: int = 0
     decode: bool = False
     cache_update: bool = False
+    pool_index_keys: bool = False
+    index_rope: int = 0
     workload: int = 0
     layer: int = 0
 
@@ -122,6 +133,8 @@ CSA_DECODE = LayerSpec(name="csa_decode_b64_ctx65536", dtype="bf16", B=64, S_q=1
                        decode=True, workload=3)
 
 
+CSA_PREFILL_INDEX_KEYS = dataclasses.replace(CSA_PREFILL, name="csa_prefill_s8192_index_keys",
+                                             pool_index_keys=True, index_rope=64, workload=6)
 CSA_DECODE_STEP = dataclasses.replace(CSA_DECODE, name="csa_decode_step_b64_ctx65536",
                                       cache_update=True, workload=5)
 
@@ -147,6 +160,7 @@ WORKLOADS: Dict[int, List[LayerSpec]] = {
     3: [CSA_DECODE],
     4: mixed_stack(),
     5: [CSA_DECODE_STEP],
+    6: [CSA_PREFILL_INDEX_KEYS],
 }
 
 
@@ -186,6 +200,12 @@ def make_inputs(spec: LayerSpec, device="cpu") -> Dict[str, Optional[torch.Tenso
     else:
         out["q_I"] = out["k_I"] = out["w"] = None
     out["sink"] = _randn((spec.H,), spec.seed("sink"), device)
+    if spec.pool_index_keys:
+        assert spec.kind == "csa" and not spec.decode
+        out["k_I"] = None
+        out["kI_tok"] = _rms_rows(_randn((spec.B, spec.S_kv, spec.d_I), spec.seed("kI_tok"),
+                                         device)).to(dt)
+        out["gI_tok"] = _randn((spec.B, spec.S_kv, spec.d_I), spec.seed("gI_tok"), device).to(dt)
     if spec.cache_update:
         assert spec.decode and spec.kind != "sliding" and spec.kv_pos0 + spec.S_kv == spec.q_pos0 + spec.S_q
         L = spec.ring
@@ -202,6 +222,11 @@ def make_inputs(spec: LayerSpec, device="cpu") -> Dict[str, Optional[torch.Tenso
             out["kI_new"] = _randn((spec.B, spec.S_q, spec.d_I), spec.seed("kI_new"), device).to(dt)
             out["gI_new"] = _randn((spec.B, spec.S_q, spec.d_I), spec.seed("gI_new"), device).to(dt)
     return out
+
+
+def normal_rows(shape, dtype: torch.dtype, seed: int, device="cpu") -> torch.Tensor:
+    """N(0,1) values of any shape (rows to rotate, and the like)."""
+    return _randn(tuple(shape), seed, device).to(dtype)
 
 
 def stream_rows(B: int, S: int, D: int, dtype: torch.dtype, seed: int, device="cpu"):

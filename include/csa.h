@@ -131,6 +131,29 @@ csa_status_t csa_index_topk(const void *q_I, const void *w, const void *k_I, int
                             void *workspace, size_t workspace_bytes, csa_dtype_t dtype,
                             void *stream);
 
+/*
+ * csa_rope_rows -- interleaved-pair partial RoPE over rows, for the Lightning Indexer's
+ * own rotary embedding (TransformerLens deepseek_v4 bridge: the indexer carries a
+ * rotary_emb; HF PR #45616 "RoPE apply: interleaved-pair rotation"; HF docs
+ * model_doc/deepseek_v4 section 2.3.3).  With it the indexer scores rotated queries
+ * against rotated pooled keys, so a score depends on t - j*ratio:
+ *
+ *   out[r] = Rot(x[r], pos0 + ((r / group) mod period) * step),  r in [0, rows)
+ *   Rot: pairs (D-R+2i, D-R+2i+1) turned by pos * rope_base^(-2i/R), R = rope_dim; the
+ *        first D-R channels are copied unchanged.
+ *
+ * Rows are taken in memory order.  Indexer queries q_I [B,S_q,H_I,d_I]: rows =
+ * B*S_q*H_I, group = H_I, period = S_q, step = 1, pos0 = q_pos0.  Pooled index keys
+ * k_I [B,P,d_I]: rows = B*P, group = 1, period = P, step = ratio, pos0 = 0 (entry j at
+ * j*ratio, as the attention rotates entries).  Call it on both before csa_index_topk.
+ *   x, out : [rows, D] device buffers; out may be x (in place) but must not otherwise
+ *            overlap it.  D % 8 == 0, rope_dim even and <= min(D, 256); every position
+ *            must stay within +-2^31.
+ */
+csa_status_t csa_rope_rows(const void *x, void *out, int64_t rows, int32_t D, int32_t rope_dim,
+                           double rope_base, int64_t pos0, int64_t group, int64_t period,
+                           int64_t step, csa_dtype_t dtype, void *stream);
+
 /* Scratch bytes csa_index_topk needs for these sizes (0 when the call needs none; a
  * decode-sized call is split over entry ranges and merges through the workspace). */
 size_t csa_index_topk_workspace_bytes(int64_t B, int64_t S_q, int64_t q_pos0, int64_t P,

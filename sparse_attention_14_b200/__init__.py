@@ -15,7 +15,7 @@ from typing import Optional
 import torch
 
 __all__ = ["csa_compress", "csa_compress_append", "csa_compress_state_bytes",
-           "csa_compress_state", "csa_index_topk", "csa_attend", "hca_attend",
+           "csa_compress_state", "csa_rope_rows", "csa_index_topk", "csa_attend", "hca_attend",
            "csa_index_topk_workspace_bytes", "csa_attend_workspace_bytes", "library_path",
            "load_library", "launch_count", "device_status", "CsaError", "CSA_F32", "CSA_BF16"]
 
@@ -50,6 +50,8 @@ def load_library():
                                         i32, ctypes.c_int, vp]
     lib.csa_compress_state_bytes.argtypes = [i64, i32, i32, i32, ctypes.c_int]
     lib.csa_compress_state_bytes.restype = sz
+    lib.csa_rope_rows.argtypes = [vp, vp, i64, i32, i32, ctypes.c_double, i64, i64, i64, i64,
+                                  ctypes.c_int, vp]
     lib.csa_index_topk.argtypes = [vp, vp, vp, i64, i64, i64, i64, i32, i32, i32, i32, vp, vp, vp,
                                    sz, ctypes.c_int, vp]
     lib.csa_index_topk_workspace_bytes.argtypes = [i64, i64, i64, i64, i32, i32, i32, i32,
@@ -63,7 +65,8 @@ def load_library():
     lib.csa_attend_workspace_bytes.argtypes = [i32, i64, i64, i64, i64, i32, i32, i32,
                                                ctypes.c_int]
     lib.csa_attend_workspace_bytes.restype = sz
-    for f in ("csa_compress", "csa_compress_append", "csa_index_topk", "csa_attend", "hca_attend"):
+    for f in ("csa_compress", "csa_compress_append", "csa_rope_rows", "csa_index_topk", "csa_attend",
+              "hca_attend"):
         getattr(lib, f).restype = ctypes.c_int
     lib.csa_last_error.restype = ctypes.c_char_p
     lib.csa_version.restype = ctypes.c_char_p
@@ -181,6 +184,23 @@ def csa_compress_append(kv_new: torch.Tensor, gate_new: torch.Tensor, state: tor
           0 if pool is None else pool.shape[1], B, n, pos0, D, ratio, int(bool(overlap)),
           _dtype_code(kv_new), _stream(stream))
     return pool
+
+
+def csa_rope_rows(x: torch.Tensor, pos0: int, group: int, period: int, step: int, rope_dim: int,
+                  rope_base: float, out: Optional[torch.Tensor] = None,
+                  stream=None) -> torch.Tensor:
+    """Rotate the last rope_dim channels of every row of x [..., D] (rows in memory order)
+    at position pos0 + ((r // group) % period) * step (see include/csa.h).  For indexer
+    queries q_I [B,S_q,H_I,d_I]: group=H_I, period=S_q, step=1, pos0=q_pos0; for pooled
+    index keys k_I [B,P,d_I]: group=1, period=P, step=ratio, pos0=0."""
+    D = x.shape[-1]
+    if out is None:
+        out = torch.empty_like(x)
+    if out.shape != x.shape or out.dtype != x.dtype:
+        raise ValueError("out must match x in shape and dtype")
+    _call("csa_rope_rows", _ptr(x), _ptr(out), x.numel() // D if D else 0, D, rope_dim,
+          float(rope_base), pos0, group, period, step, _dtype_code(x), _stream(stream))
+    return out
 
 
 def csa_index_topk_workspace_bytes(B, S_q, q_pos0, P, H_I, d_I, ratio, topk,

@@ -84,6 +84,30 @@ def test_compress_append_rejects(lib):
     assert lib.csa_compress_state_bytes(3, 60, 4, 1, 1) == 0
 
 
+def test_rope_rows_rejects(lib):
+    args = lambda **kw: [kw.get("x", FAKE), kw.get("out", FAKE), kw.get("rows", 10),
+                         kw.get("D", 128), kw.get("R", 64), kw.get("base", 160000.0),
+                         kw.get("pos0", 0), kw.get("group", 1), kw.get("period", 10),
+                         kw.get("step", 4), kw.get("dtype", 1), None]
+    assert lib.csa_rope_rows(*args(D=60)) == -1
+    assert lib.csa_rope_rows(*args(R=63)) == -1
+    assert lib.csa_rope_rows(*args(R=136)) == -1          # wider than the row
+    assert lib.csa_rope_rows(*args(D=1024, R=512)) == -1  # more than 128 pairs
+    assert lib.csa_rope_rows(*args(base=0.0)) == -1
+    assert lib.csa_rope_rows(*args(group=0)) == -1
+    assert lib.csa_rope_rows(*args(period=0)) == -1
+    assert lib.csa_rope_rows(*args(pos0=2 ** 31)) == -1
+    assert lib.csa_rope_rows(*args(period=2 ** 29, step=8)) == -1
+    assert lib.csa_rope_rows(*args(rows=-1)) == -1
+    assert lib.csa_rope_rows(*args(x=None)) == -1
+    assert lib.csa_rope_rows(*args(out=MIS)) == -1
+    assert lib.csa_rope_rows(*args(dtype=3)) == -1
+    # out overlapping x without being x
+    assert lib.csa_rope_rows(*args(out=ctypes.c_void_p(0x10000 + 256))) == -1
+    assert "overlap" in _err(lib)
+    assert lib.csa_rope_rows(*args(rows=0)) == 0
+
+
 def test_index_topk_rejects(lib):
     args = lambda **kw: [kw.get("q", FAKE), kw.get("w", FAKE), kw.get("k", FAKE), kw.get("B", 1),
                          kw.get("S", 8), kw.get("pos", 0), kw.get("P", 2), kw.get("HI", 4),

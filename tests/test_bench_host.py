@@ -149,3 +149,19 @@ def test_workload_config_is_plain_json(w):
     assert len(cfg["m"]) == len(cfg["P"]) == len(specs)
     # no model keys: the config names a workload, not a checkpoint
     assert "model" not in cfg
+
+
+def test_index_key_path_work_and_oracle_sample():
+    """Workload 6 (prefill with the indexer's key path): the extra stages' bytes, the stage
+    order, and the sampled oracle run that pools the index keys and rotates both sides."""
+    s = cs.WORKLOADS[6][0]
+    w = bench.algorithmic_work(s)
+    assert w["compress_I_bytes"] == (2 * 8192 + 2048) * 128 * 2
+    assert w["rope_I_bytes"] == 2 * (8192 * 64 + 2048) * 128 * 2
+    base = bench.algorithmic_work(cs.CSA_PREFILL)
+    assert {k: v for k, v in w.items() if k not in ("compress_I_bytes", "rope_I_bytes")} == base
+    assert bench.LayerRunner.stages(type("R", (), {"spec": s})()) == \
+        ["compress", "compress_I", "rope_I", "index", "attend"]
+    small = dataclasses.replace(s, S_q=96, S_kv=96, P=24, topk=8, H=4, D=64, R=16, H_I=4, d_I=32,
+                                index_rope=16, workload=72)
+    assert bench.oracle_sample_run(small, [0, 50, 95]) > 0

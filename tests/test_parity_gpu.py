@@ -332,3 +332,126 @@ def test_append_resumes_after_prefill(ratio, overlap, S0, S):
     got = to_np(pool)
     assert np.isfinite(got).all()
     assert rel_err(got, ref) <= TOL["bf16"]
+
+
+# ----------------------------------------------------------------------------- indexer RoPE
+ROPE_CASES = [  # name, dtype, shape, group, period, step, pos0, rope_dim, base
+    ("q_I_bf16", torch.bfloat16, (2, 37, 5, 128), 5, 37, 1, 4000, 64, 160000.0),
+    ("k_I_bf16", torch.bfloat16, (2, 50, 128), 1, 50, 4, 0, 64, 160000.0),
+    ("odd_f32", torch.float32, (3, 11, 40), 1, 33, 3, 7, 8, 10000.0),
+    ("full_width_far_f32", torch.float32, (4, 16), 2, 2, 5, 2 ** 30, 16, 10000.0),
+]
+
+
+@pytest.mark.parametrize("name,dt,shape,group,period,step,pos0,R,base", ROPE_CASES,
+                         ids=[c[0] for c in ROPE_CASES])
+def test_rope_rows_parity(name, dt, shape, group, period, step, pos0, R, base):
+    """csa_rope_rows against the oracle's rotation row by row, out of place and in place;
+    the channels before the rotated ones are copied bit for bit."""
+    x = cs.normal_rows(shape, dt, 800 + [c[0] for c in ROPE_CASES].index(name), device=DEV)
+    D = shape[-1]
+    rows = x.numel() // D
+    out = csa.csa_rope_rows(x, pos0, group, period, step, R, base)
+    xi = x.clone()
+    csa.csa_rope_rows(xi, pos0, group, period, step, R, base, out=xi)
+    torch.cuda.synchronize()
+    pos = pos0 + ((np.arange(rows) // group) % period) * step
+    ref = oracle.rope(to_np(x).reshape(rows, D), pos, R, base)
+    tol = TOL["f32" if dt == torch.float32 else "bf16"]
+    assert rel_err(to_np(out).reshape(rows, D), ref) <= tol
+    assert torch.equal(out, xi)
+    assert torch.equal(out[..., :D - R], x[..., :D - R])
+
+
+def _pooled_index_keys(spec, dt):
+    """Per-token index keys and their gates (seeded), pooled like the main compressor."""
+    kI_tok, gI_tok = cs.stream_rows(spec.B, spec.S_kv, spec.d_I, dt, 900 + spec.workload, device=DEV)
+    return kI_tok, gI_tok, csa.csa_compress(kI_tok, gI_tok, spec.m, spec.overlap)
+
+
+def test_indexer_key_pooling_and_rope_end_to_end_f32():
+    """The indexer's key path in full (fp32, so top-k sets are compared directly):
+    per-token index keys pooled by the gated compressor, queries and pooled keys rotated,
+    then scored and selected, against the oracle's compressor, indexer RoPE and top-k."""
+    spec = next(x for x in MID if x.name == "mid_csa_f32")
+    inp = _inputs(spec)
+    R = 16
+    kI_tok, gI_tok, k_I = _pooled_index_keys(spec, torch.float32)
+    q_rot = csa.csa_rope_rows(inp["q_I"], spec.q_pos0, spec.H_I, spec.S_q, 1, R, spec.base)
+    k_rot = csa.csa_rope_rows(k_I, 0, 1, spec.P, spec.m, R, spec.base)
+    idx = csa.csa_index_topk(q_rot, inp["w"], k_rot, spec.q_pos0, spec.m, spec.topk)
+    torch.cuda.synchronize()
+    rows = list(range(spec.S_q))
+    tpos = np.asarray(rows, dtype=np.int64) + spec.q_pos0
+    o_kI = oracle.compress(to_np(kI_tok), to_np(gI_tok), spec.m, spec.overlap)
+    assert rel_err(to_np(k_I), o_kI) <= TOL["f32"]
+    sc = oracle.index_scores_rope(to_np(inp["q_I"]), to_np(inp["w"]), o_kI, tpos, spec.m, R,
+                                  spec.base)
+    o_idx, _ = oracle.topk(sc, tpos, spec.m, spec.topk)
+    g_idx = idx.cpu().numpy()
+    n_diff = 0
+    for b in range(spec.B):
+        n_diff += check_topk(g_idx[b], o_idx[b], sc[b], kk_rows(spec, rows))
+    assert n_diff <= 0.02 * spec.B * spec.S_q
+
+
+def test_indexer_key_pooling_and_rope_stagewise_bf16():
+    """The same chain at the V4-Flash indexer shape (d_I = 128, rope 64, bf16), stage by
+    stage so that bf16 rounding between stages cannot move a top-k boundary: pooled keys
+    and both rotations against the oracle, then the indexer on the rotated tensors against
+    the oracle indexer on the same tensors."""
+    spec = next(x for x in MID if x.name == "mid_csa_bf16")
+    inp = _inputs(spec)
+    R = 64
+    kI_tok, gI_tok, k_I = _pooled_index_keys(spec, torch.bfloat16)
+    q_rot = csa.csa_rope_rows(inp["q_I"], spec.q_pos0, spec.H_I, spec.S_q, 1, R, spec.base)
+    k_rot = csa.csa_rope_rows(k_I, 0, 1, spec.P, spec.m, R, spec.base)
+    idx = csa.csa_index_topk(q_rot, inp["w"], k_rot, spec.q_pos0, spec.m, spec.topk)
+    torch.cuda.synchronize()
+    rows = list(range(spec.S_q))
+    tpos = np.asarray(rows, dtype=np.int64) + spec.q_pos0
+    assert rel_err(to_np(k_I), oracle.compress(to_np(kI_tok), to_np(gI_tok), spec.m,
+                                               spec.overlap)) <= TOL["bf16"]
+    q_ref = oracle.rope(to_np(inp["q_I"]), np.broadcast_to(tpos[None, :, None], q_rot.shape[:3]),
+                        R, spec.base)
+    k_ref = oracle.rope(to_np(k_I), np.broadcast_to((np.arange(spec.P) * spec.m)[None, :],
+                                                    k_rot.shape[:2]), R, spec.base)
+    assert rel_err(to_np(q_rot), q_ref) <= TOL["bf16"]
+    assert rel_err(to_np(k_rot), k_ref) <= TOL["bf16"]
+    sc = oracle.index_scores(to_np(q_rot), to_np(inp["w"]), to_np(k_rot), tpos, spec.m)
+    o_idx, _ = oracle.topk(sc, tpos, spec.m, spec.topk)
+    g_idx = idx.cpu().numpy()
+    for b in range(spec.B):
+        check_topk(g_idx[b], o_idx[b], sc[b], kk_rows(spec, rows))
+
+
+def test_workload6_index_key_path_sampled():
+    """Workload 6 at full size, in the benchmark's call sequence, checked stage by stage:
+    every pooled index key and every rotated key against the oracle, then the rotated
+    queries and the top-k on sampled query rows (the oracle indexer on the same rotated
+    tensors).  The attention after it is the one workload 1 checks."""
+    spec = cs.WORKLOADS[6][0]
+    inp = _inputs(spec)
+    R = spec.index_rope
+    k_I = csa.csa_compress(inp["kI_tok"], inp["gI_tok"], spec.m, spec.overlap)
+    q_rot = csa.csa_rope_rows(inp["q_I"], spec.q_pos0, spec.H_I, spec.S_q, 1, R, spec.base)
+    k_rot = csa.csa_rope_rows(k_I, 0, 1, spec.P, spec.m, R, spec.base)
+    idx = csa.csa_index_topk(q_rot, inp["w"], k_rot, spec.q_pos0, spec.m, spec.topk)
+    torch.cuda.synchronize()
+    assert rel_err(to_np(k_I), oracle.compress(to_np(inp["kI_tok"]), to_np(inp["gI_tok"]),
+                                               spec.m, spec.overlap)) <= TOL["bf16"]
+    k_ref = oracle.rope(to_np(k_I), np.broadcast_to((np.arange(spec.P) * spec.m)[None, :],
+                                                    k_rot.shape[:2]), R, spec.base)
+    assert rel_err(to_np(k_rot), k_ref) <= TOL["bf16"]
+    rows = cs.sample_rows(spec, n_random=64)
+    rows_t = torch.tensor(rows, device=DEV)
+    tpos = np.asarray(rows, dtype=np.int64) + spec.q_pos0
+    q_s = q_rot[:, rows_t]
+    q_ref = oracle.rope(to_np(inp["q_I"][:, rows_t]),
+                        np.broadcast_to(tpos[None, :, None], q_s.shape[:3]), R, spec.base)
+    assert rel_err(to_np(q_s), q_ref) <= TOL["bf16"]
+    sc = oracle.index_scores(to_np(q_s), to_np(inp["w"][:, rows_t]), to_np(k_rot), tpos, spec.m)
+    o_idx, _ = oracle.topk(sc, tpos, spec.m, spec.topk)
+    g_idx = idx[:, rows_t].cpu().numpy()
+    for b in range(spec.B):
+        check_topk(g_idx[b], o_idx[b], sc[b], kk_rows(spec, rows))
