@@ -15,6 +15,7 @@ Function map (each C function's comment cites the page passage it follows):
   attend        -> orc_attend         sink MQA over window + entries, RoPE, de-rotation
   attend_keys   -> orc_attend_keys    the same for one query over explicit keys
   rope          -> orc_rope_rows      interleaved-pair partial RoPE
+  grouped_out_proj -> numpy matmuls   grouped low-rank output projection (after attention)
 """
 from __future__ import annotations
 
@@ -259,3 +260,29 @@ def attend(q, tpos, kv, kv_pos0: int, pool, m: int, idx, sink, R: int, base: flo
                               _ptr(sink, _dp), B, H, D, R, base, W, scale, _ptr(out, _dp)),
            "attend")
     return out
+
+
+def grouped_out_proj(o, w_a, w_b, return_groups: bool = False):
+    """Grouped low-rank output projection after the attention (HF docs model_doc/
+    deepseek_v4, section 2.3 "Grouped Output Projection": o_groups head groups ->
+    o_lora_rank per group -> hidden_size, computed by DeepseekV4GroupedLinear (o_a_proj)
+    and then o_b_proj; HF PR #45616: the grouped linear's forward is a per-group batched
+    matmul, and the output's rope slice is un-rotated before this projection).
+
+    o    [B,S,H,D]          de-rotated attention output
+    w_a  [G, r, (H/G)*D]    o_a_proj: group g projects heads [g*H/G, (g+1)*H/G), flattened
+                            head-major, to r features
+    w_b  [hidden, G*r]      o_b_proj over the G groups' features, group-major
+    -> y [B,S,hidden] (and z [B,S,G,r] when return_groups).
+    Plain fp64 matmuls per group, in the order the definition states."""
+    o, w_a, w_b = _f64(o), _f64(w_a), _f64(w_b)
+    B, S, H, D = o.shape
+    G, r, per = w_a.shape
+    if H % G or per != (H // G) * D or w_b.shape[1] != G * r:
+        raise ValueError("grouped_out_proj: shapes do not match")
+    x = o.reshape(B, S, G, per)
+    z = np.zeros((B, S, G, r))
+    for g in range(G):
+        z[:, :, g] = x[:, :, g] @ w_a[g].T
+    y = z.reshape(B, S, G * r) @ w_b.T
+    return (y, z) if return_groups else y

@@ -494,4 +494,51 @@ def pin_entry_position_and_duplicates():
     assert not np.allclose(dup, want)
 
 
+# ----------------------------------------------------------------------------- output projection
+def _proj_weights(rng, G, r, H, D, hidden):
+    return rng.standard_normal((G, r, (H // G) * D)), rng.standard_normal((hidden, G * r))
+
+
+def pin_grouped_out_proj_one_group_is_two_linears():
+    """With one group the projection is o_b_proj(o_a_proj(flattened heads)): checked with
+    torch.nn.functional.linear in float64."""
+    rng = _rng(50)
+    B, S, H, D, r, hidden = 2, 3, 4, 6, 5, 7
+    o = rng.standard_normal((B, S, H, D))
+    w_a, w_b = _proj_weights(rng, 1, r, H, D, hidden)
+    t = torch.from_numpy
+    want = torch.nn.functional.linear(torch.nn.functional.linear(t(o).reshape(B, S, H * D),
+                                                                 t(w_a[0])), t(w_b)).numpy()
+    np.testing.assert_allclose(oracle.grouped_out_proj(o, w_a, w_b), want, rtol=1e-12, atol=1e-12)
+
+
+def pin_grouped_out_proj_block_diagonal():
+    """G groups equal one dense o_a_proj whose weight is block-diagonal in the groups
+    (scipy's block_diag), followed by o_b_proj."""
+    from scipy.linalg import block_diag
+    rng = _rng(51)
+    B, S, H, D, G, r, hidden = 1, 4, 8, 3, 4, 2, 5
+    o = rng.standard_normal((B, S, H, D))
+    w_a, w_b = _proj_weights(rng, G, r, H, D, hidden)
+    dense = block_diag(*[w_a[g] for g in range(G)])          # [G*r, H*D]
+    want = (o.reshape(B, S, H * D) @ dense.T) @ w_b.T
+    np.testing.assert_allclose(oracle.grouped_out_proj(o, w_a, w_b), want, rtol=1e-12, atol=1e-12)
+
+
+def pin_grouped_out_proj_head_groups():
+    """Group g sees exactly heads [g*H/G, (g+1)*H/G): changing one head moves only its
+    group's low-rank features."""
+    rng = _rng(52)
+    B, S, H, D, G, r, hidden = 1, 2, 8, 4, 4, 3, 6
+    o = rng.standard_normal((B, S, H, D))
+    w_a, w_b = _proj_weights(rng, G, r, H, D, hidden)
+    _, z0 = oracle.grouped_out_proj(o, w_a, w_b, return_groups=True)
+    for h in range(H):
+        o2 = o.copy()
+        o2[:, :, h] += 1.0
+        _, z1 = oracle.grouped_out_proj(o2, w_a, w_b, return_groups=True)
+        moved = np.abs(z1 - z0).max(axis=(0, 1, 3)) > 1e-9
+        assert moved.tolist() == [g == h // (H // G) for g in range(G)], h
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
