@@ -113,7 +113,7 @@ class ClockSampler:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu),
                                           "--query-gpu=" + self.FIELDS, "--format=csv,noheader",
-                                          "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+                                          "-lms", "20"], stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
@@ -441,9 +441,9 @@ def gpu_arm(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "f32" if spec0.dtype == "f32" else "bf16",
         "data": "synthetic (seeded N(0,1) q/kv/gate/q_I/k_I, w/sqrt(H_I), RMS-normalised kv)",
-        "config": dict(workload_config(args.workload, specs),
-                       l2="inputs larger than L2 (q/out/q_I > 126 MB per step); no flush",
-                       launch=launch_mode),
+        "config": workload_config(args.workload, specs),
+        "l2": "inputs larger than L2 (q/out/q_I > 126 MB per step); no flush",
+        "launch": launch_mode,
         "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
         "roofline": roof,
         "gpu_launches": int(launches),
@@ -627,6 +627,25 @@ def reference_arm(args, rank, world):
 
 
 # ----------------------------------------------------------------------------- main
+def _free_port() -> int:
+    import socket
+    sk = socket.socket()
+    sk.bind(("127.0.0.1", 0))
+    port = sk.getsockname()[1]
+    sk.close()
+    return port
+
+
+def launch_ranks(n: int, limit_s: int = 1800) -> int:
+    """`bench.py --gpus N` run without a launcher: re-run this command under
+    torch.distributed.run with one rank per GPU (rendezvous on 127.0.0.1), bounded by
+    `timeout`.  Returns the launcher's exit code; rank 0 prints the JSON line."""
+    cmd = ["timeout", "-k", "60", str(limit_s), sys.executable, "-m", "torch.distributed.run",
+           "--nnodes=1", "--nproc-per-node=%d" % n, "--master-addr", "127.0.0.1",
+           "--master-port", str(_free_port()), os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -641,6 +660,8 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(launch_ranks(args.gpus))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -250,6 +250,19 @@ const char *csa_last_error(void);
  * clears the flags.  For tests and diagnostics. */
 uint32_t csa_device_status(void);
 
+/*
+ * csa_debug_withhold_attention_loads -- test hook for the bounded-wait error path of the
+ * tensor-core attention; not part of the layer (the pages have no counterpart).
+ * on != 0: from the next launch on, the attention kernel's loader publishes nothing, so
+ * every wait on it gives up after a short bound (well under a millisecond); the kernel
+ * then skips its work (out is left unwritten or holds partial values), frees its tensor
+ * memory, returns and sets bit 0 of csa_device_status().  Nothing faults or hangs and the
+ * context stays usable.  on == 0 restores normal operation.  Synchronous (a copy to a
+ * device variable on the current device); call it only while no attention work is in
+ * flight.  Returns CSA_ERR_CUDA if the copy fails.
+ */
+csa_status_t csa_debug_withhold_attention_loads(int32_t on);
+
 /* Number of kernels this library has enqueued in this process (all devices, all
  * threads); for accounting launches in a timed region. */
 uint64_t csa_launch_count(void);

@@ -17,7 +17,7 @@ import torch
 __all__ = ["csa_compress", "csa_compress_append", "csa_compress_state_bytes",
            "csa_compress_state", "csa_rope_rows", "csa_index_topk", "csa_attend", "hca_attend",
            "csa_index_topk_workspace_bytes", "csa_attend_workspace_bytes", "library_path",
-           "load_library", "launch_count", "device_status", "CsaError", "CSA_F32", "CSA_BF16"]
+           "load_library", "launch_count", "device_status", "debug_withhold_attention_loads", "CsaError", "CSA_F32", "CSA_BF16"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libcsa_b200.so")
@@ -72,6 +72,8 @@ def load_library():
     lib.csa_version.restype = ctypes.c_char_p
     lib.csa_launch_count.restype = ctypes.c_uint64
     lib.csa_device_status.restype = ctypes.c_uint32
+    lib.csa_debug_withhold_attention_loads.argtypes = [ctypes.c_int32]
+    lib.csa_debug_withhold_attention_loads.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -84,6 +86,11 @@ def launch_count() -> int:
 def device_status() -> int:
     """Nonzero if a kernel gave up on a bounded wait since the last call (synchronises)."""
     return int(load_library().csa_device_status())
+
+
+def debug_withhold_attention_loads(on: bool) -> None:
+    """Test hook: make the tensor-core attention's bounded waits run out (see csa.h)."""
+    _call("csa_debug_withhold_attention_loads", int(bool(on)))
 
 
 def _dtype_code(t: torch.Tensor) -> int:

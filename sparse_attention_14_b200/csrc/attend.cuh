@@ -46,6 +46,8 @@ int attend_tc_kmax(const AttendArgs &a);
 size_t attend_tc_workspace(const AttendArgs &a);
 csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st);
 unsigned int read_attend_tc_status();
+// Test hook behind csa_debug_withhold_attention_loads.
+csa_status_t set_attend_tc_withhold(int on);
 // Same kernel with its scratch in a fixed device array (csa_attend_noalloc).
 csa_status_t attend_tc_noalloc(AttendArgs &a, cudaStream_t st);
 

@@ -40,6 +40,10 @@
 namespace csa {
 
 __device__ unsigned int g_attend_tc_status;
+// Test hook (csa_debug_withhold_attention_loads): when nonzero the loader publishes
+// nothing, so every bounded wait on it runs out after a short bound and the kernel takes
+// its error path (status bit, skipped work) without any fault or hang.
+__device__ unsigned int g_attend_tc_withhold;
 
 namespace {
 
@@ -57,7 +61,7 @@ constexpr float kRescaleThreshold = 8.0f;        // log2 units
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 64, 0, 0);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 64, 1, 1);
 constexpr uint32_t kColO = 0, kColS = 256;
-constexpr uint32_t kWaitIter = 1u << 25;         // bounded waits (~seconds)
+constexpr uint32_t kWaitIterMax = 1u << 25;      // bounded waits (~seconds)
 
 struct Meta {
     int n_ent;
@@ -253,20 +257,6 @@ __device__ __forceinline__ void warp_reduce32(float *v) {
     }
 }
 
-// Named barrier over `count` threads that also ORs a predicate across them.
-__device__ __forceinline__ bool named_sync_any(uint32_t id, uint32_t count, bool v) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred pi, po;\n\t"
-        "setp.ne.u32 pi, %1, 0;\n\t"
-        "bar.red.or.pred po, %2, %3, pi;\n\t"
-        "selp.u32 %0, 1, 0, po;\n\t}\n"
-        : "=r"(r)
-        : "r"((uint32_t)v), "r"(id), "r"(count)
-        : "memory");
-    return r != 0;
-}
-
 // 2^x by the hardware approximation (relative error about 2^-22, flushes subnormal
 // results to zero): P is rounded to bf16 right after, so this is exact enough.
 __device__ __forceinline__ float ex2_fast(float x) {
@@ -337,6 +327,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     Small &sm = *reinterpret_cast<Small *>(smem + kOffEnt + ent_bytes);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const bool withhold = *reinterpret_cast<volatile unsigned int *>(&g_attend_tc_withhold) != 0u;
+    const uint32_t kWaitIter = withhold ? (1u << 12) : kWaitIterMax;
     // work item w = query w / n_split, key-tile range w % n_split of it (n_split > 1 only for
     // decode-sized calls, whose partial results the combine kernel merges)
     const int64_t nw = B * S_q * n_split;
@@ -364,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     if (warp == 0) {
         // ===================================================== loader
         uint32_t g = 0, qc = 0;
-        for (int64_t w = blockIdx.x; w < nw && !sm.abort_; w += gridDim.x, ++qc) {
+        for (int64_t w = blockIdx.x; w < nw && !sm.abort_ && !withhold; w += gridDim.x, ++qc) {
             const int64_t qi = w / n_split;
             const int64_t qn = (w + gridDim.x) / n_split;   // query of the next work item
             const QueryGeom qg = query_geom(qi, S_q, q_pos0, kv_pos0, S_kv, window, packed_n);
@@ -1045,6 +1037,13 @@ csa_status_t attend_tc_noalloc(AttendArgs &a, cudaStream_t st) {
     a.workspace = ptr;
     a.workspace_bytes = kNoAllocScratchBytes;
     return attend_tc(a, st);
+}
+
+csa_status_t set_attend_tc_withhold(int on) {
+    const unsigned int v = on ? 1u : 0u;
+    cudaError_t e = cudaMemcpyToSymbol(g_attend_tc_withhold, &v, sizeof(v));
+    CSA_REQUIRE(e == cudaSuccess, CSA_ERR_CUDA, "csa_debug_withhold_attention_loads: %s", cudaGetErrorString(e));
+    return CSA_OK;
 }
 
 unsigned int read_attend_tc_status() {

@@ -135,6 +135,11 @@ extern "C" uint32_t csa_device_status(void) {
     return s;
 }
 
+extern "C" csa_status_t csa_debug_withhold_attention_loads(int32_t on) {
+    csa::clear_error();
+    return csa::set_attend_tc_withhold(on);
+}
+
 extern "C" uint64_t csa_launch_count(void) { return csa::g_launches.load(); }
 
 extern "C" const char *csa_version(void) { return "csa_b200 0.1 (sm_100a)"; }

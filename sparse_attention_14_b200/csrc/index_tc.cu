@@ -13,7 +13,7 @@
 //    MMAs (one thread), the epilogue warps read D from TMEM (thread = entry row) and
 //    form sum_h w[q,h] ReLU(D) for their queries, while the next tile's MMA runs;
 //  * top-k without writing scores to HBM: each query keeps a candidate buffer of
-//    1024 64-bit keys (order-preserving score bits, then the complemented entry index,
+//    kCap = 2048 64-bit keys (order-preserving score bits, then the complemented entry index,
 //    so that equal scores rank the lower index first) and a threshold; a tile inserts
 //    only keys above the threshold, and whenever the buffer could overflow it is cut
 //    back to exactly k by an exact radix select over the 64-bit keys (which then becomes
@@ -493,8 +493,9 @@ __global__ void __launch_bounds__(Cfg<QB>::kThreads, Cfg<QB>::kMinBlocks) index_
                 if (ms.cnt[q] > (unsigned)(kCap - kTileE) && grp == q)
                     group_cut<C::GS>(cand_all + q * kCap, topk, gt, 2 + q, hist_all + q * 256, ms, q, q);
             }
-            named_sync(1, C::NE * 32);
-            if (!ok) break;
+            // leave the loop together: a thread whose wait ran out must not leave the others
+            // waiting for it at the next barrier
+            if (named_sync_any(1, C::NE * 32, !ok)) break;
         }
         // final: this group's query
         if (grp < nq_valid) {

@@ -203,5 +203,21 @@ __device__ __forceinline__ void named_sync(uint32_t id, uint32_t count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Named barrier over `count` threads that also ORs a predicate across them: every thread
+// gets the same answer, so a decision taken on it (such as leaving a loop after a bounded
+// wait ran out in some thread) is uniform and no thread is left waiting at a later barrier.
+__device__ __forceinline__ bool named_sync_any(uint32_t id, uint32_t count, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\t"
+        "setp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.or.pred po, %2, %3, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}\n"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
+}
+
 }  // namespace umma
 }  // namespace csa

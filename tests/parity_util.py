@@ -24,6 +24,9 @@ TIE_BAND = 1e-3
 def rel_err(gpu, ref) -> float:
     gpu = np.asarray(gpu, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
+    assert gpu.shape == ref.shape, (gpu.shape, ref.shape)
+    if ref.size == 0:
+        return 0.0
     den = np.max(np.abs(ref))
     if den == 0:
         return float(np.max(np.abs(gpu)))
