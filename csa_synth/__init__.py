@@ -275,3 +275,24 @@ def sample_rows(spec: LayerSpec, n_random: int = 256, seed: int = 12345) -> List
     if S > 0:
         rows.update(torch.randint(0, S, (n_random,), generator=g).tolist())
     return sorted(rows)
+
+
+# Projection sizes around the layer.  The pages name o_groups, o_lora_rank and hidden_size
+# but give no values; these are readings at the V4-Flash head shape: 64 heads of 512 in 8
+# groups of 8 heads, 1024 low-rank features per group, a 4096-wide hidden state.
+PROJ_HIDDEN, PROJ_GROUPS, PROJ_RANK = 4096, 8, 1024
+
+
+def proj_weights(H: int, D: int, G: int, r: int, hidden: int, dtype: torch.dtype, seed: int,
+                 device="cpu"):
+    """Seeded weights of the projections, scaled like a linear layer's default init
+    (N(0,1) / sqrt(fan_in)): w_a [G, r, (H/G)*D], w_b [hidden, G*r] (output projection);
+    w_kv, w_gate [D, hidden] and kv_norm_w [D] ~ 1 + N(0,1)/10 (compressor inputs);
+    seeds seed .. seed+4."""
+    per = (H // G) * D
+    w_a = (_randn((G, r, per), seed, device) / math.sqrt(per)).to(dtype)
+    w_b = (_randn((hidden, G * r), seed + 1, device) / math.sqrt(G * r)).to(dtype)
+    w_kv = (_randn((D, hidden), seed + 2, device) / math.sqrt(hidden)).to(dtype)
+    w_gate = (_randn((D, hidden), seed + 3, device) / math.sqrt(hidden)).to(dtype)
+    kv_norm_w = (1.0 + 0.1 * _randn((D,), seed + 4, device)).to(dtype)
+    return {"w_a": w_a, "w_b": w_b, "w_kv": w_kv, "w_gate": w_gate, "kv_norm_w": kv_norm_w}

@@ -237,6 +237,50 @@ csa_status_t csa_attend_noalloc(const void *q, const void *kv, int64_t S_kv, int
                                 double rope_base, int32_t window, int32_t ratio, float scale,
                                 csa_dtype_t dtype, void *stream);
 
+/*
+ * csa_out_proj -- grouped low-rank output projection after the attention (HF docs
+ * model_doc/deepseek_v4, section 2.3 "Grouped Output Projection": o_groups head groups,
+ * o_lora_rank features per group by DeepseekV4GroupedLinear (o_a_proj), then o_b_proj to
+ * hidden_size; HF PR #45616 on DeepseekV4GroupedLinear as a per-group batched matmul).
+ *
+ *   z[m, g*r + i] = sum_c o[m, g*(H/G)*D + c] * w_a[g, i, c]      (group g: heads
+ *                   [g*H/G, (g+1)*H/G), flattened head-major, c < (H/G)*D)
+ *   y[m, n]       = sum_k z[m, k] * w_b[n, k]
+ *
+ *   o   : [M, H, D]  the de-rotated attention output (M = B*S rows)
+ *   w_a : [G, r, (H/G)*D]   w_b : [hidden, G*r]   y : [M, hidden] output
+ *   workspace : at least csa_out_proj_workspace_bytes(M, G, r) bytes; it receives z in
+ *               bf16 [M, G*r] (rounded there, fp32 accumulation in both products).
+ * bf16 only.  Shape limits: (H/G)*D and G*r multiples of 64; r and hidden multiples of
+ * 256 (CSA_ERR_UNSUPPORTED otherwise).
+ */
+csa_status_t csa_out_proj(const void *o, const void *w_a, const void *w_b, void *y, int64_t M,
+                          int32_t H, int32_t D, int32_t G, int32_t r, int32_t hidden,
+                          void *workspace, size_t workspace_bytes, csa_dtype_t dtype,
+                          void *stream);
+
+/* Scratch bytes csa_out_proj needs (the bf16 group features z). */
+size_t csa_out_proj_workspace_bytes(int64_t M, int32_t G, int32_t r);
+
+/*
+ * csa_kv_gate_proj -- the compressor's input projections (TransformerLens deepseek_v4
+ * bridge: the compressor carries kv_proj, gate_proj and kv_norm): per token row m,
+ *
+ *   kv[m, :]   = RMSNorm(x[m, :] . w_kv^T) * kv_norm_w,  RMSNorm(v) = v / sqrt(mean(v^2) + eps)
+ *   gate[m, :] = x[m, :] . w_gate^T
+ *
+ * i.e. the raw K=V rows and gate logits csa_compress pools (the synthetic workloads feed
+ * csa_compress RMS-normalised rows, which is what this produces with kv_norm_w = 1).
+ *
+ *   x : [M, hidden]   w_kv, w_gate : [D, hidden]   kv_norm_w : [D]
+ *   kv, gate : [M, D] outputs
+ * bf16 only (fp32 accumulation and normalisation).  Shape limits: hidden % 64 == 0,
+ * D in {256, 512} (CSA_ERR_UNSUPPORTED otherwise).
+ */
+csa_status_t csa_kv_gate_proj(const void *x, const void *w_kv, const void *w_gate,
+                              const void *kv_norm_w, float eps, void *kv, void *gate, int64_t M,
+                              int32_t hidden, int32_t D, csa_dtype_t dtype, void *stream);
+
 /* Scratch bytes csa_attend (mode 0) or hca_attend (mode 1) needs for these sizes. */
 size_t csa_attend_workspace_bytes(int32_t mode, int64_t B, int64_t S_q, int64_t S_kv,
                                   int64_t P, int32_t H, int32_t D, int32_t topk,
@@ -246,7 +290,7 @@ size_t csa_attend_workspace_bytes(int32_t mode, int64_t B, int64_t S_q, int64_t 
 const char *csa_last_error(void);
 
 /* Nonzero if a kernel of this library gave up on a bounded wait (and skipped the rest
- * of its work) since the last call; bit 0: attention, bit 1: indexer.  Synchronises the device and
+ * of its work) since the last call; bit 0: attention, bit 1: indexer, bit 2: projections.  Synchronises the device and
  * clears the flags.  For tests and diagnostics. */
 uint32_t csa_device_status(void);
 

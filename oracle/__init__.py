@@ -16,6 +16,7 @@ Function map (each C function's comment cites the page passage it follows):
   attend_keys   -> orc_attend_keys    the same for one query over explicit keys
   rope          -> orc_rope_rows      interleaved-pair partial RoPE
   grouped_out_proj -> numpy matmuls   grouped low-rank output projection (after attention)
+  kv_gate_proj  -> numpy matmuls      kv_proj + kv_norm and gate_proj (before the compressor)
 """
 from __future__ import annotations
 
@@ -286,3 +287,23 @@ def grouped_out_proj(o, w_a, w_b, return_groups: bool = False):
         z[:, :, g] = x[:, :, g] @ w_a[g].T
     y = z.reshape(B, S, G * r) @ w_b.T
     return (y, z) if return_groups else y
+
+
+def kv_gate_proj(x, w_kv, w_gate, kv_norm_w, eps: float):
+    """The compressor's input projections (TransformerLens deepseek_v4 bridge: the
+    compressor's kv_proj, gate_proj and kv_norm submodules, an RMSNormalizationBridge).
+    Reading taken (the pages name the modules, not their order): per token the K=V row is
+    kv_proj of the token, RMS-normalised over its D channels and scaled by the norm's
+    weight; the gate logits are gate_proj of the token.
+
+    x [..., hidden]; w_kv, w_gate [D, hidden]; kv_norm_w [D]
+    -> kv [..., D] = u / sqrt(mean(u^2) + eps) * kv_norm_w with u = x . w_kv^T,
+       gate [..., D] = x . w_gate^T.
+    Plain fp64 matmuls and the norm in the order the definition states."""
+    x, w_kv, w_gate, g = _f64(x), _f64(w_kv), _f64(w_gate), _f64(kv_norm_w)
+    if w_kv.shape != w_gate.shape or w_kv.shape[1] != x.shape[-1] or g.shape != (w_kv.shape[0],):
+        raise ValueError("kv_gate_proj: shapes do not match")
+    u = x @ w_kv.T
+    kv = u / np.sqrt((u * u).mean(axis=-1, keepdims=True) + eps) * g
+    gate = x @ w_gate.T
+    return kv, gate

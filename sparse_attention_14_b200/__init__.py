@@ -16,7 +16,8 @@ import torch
 
 __all__ = ["csa_compress", "csa_compress_append", "csa_compress_state_bytes",
            "csa_compress_state", "csa_rope_rows", "csa_index_topk", "csa_attend", "hca_attend",
-           "csa_index_topk_workspace_bytes", "csa_attend_workspace_bytes", "library_path",
+           "csa_index_topk_workspace_bytes", "csa_attend_workspace_bytes", "csa_out_proj",
+           "csa_out_proj_workspace_bytes", "csa_kv_gate_proj", "library_path",
            "load_library", "launch_count", "device_status", "debug_withhold_attention_loads", "CsaError", "CSA_F32", "CSA_BF16"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -72,6 +73,12 @@ def load_library():
     lib.csa_version.restype = ctypes.c_char_p
     lib.csa_launch_count.restype = ctypes.c_uint64
     lib.csa_device_status.restype = ctypes.c_uint32
+    lib.csa_out_proj.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, i32, i32, vp, sz, ctypes.c_int, vp]
+    lib.csa_out_proj.restype = ctypes.c_int
+    lib.csa_out_proj_workspace_bytes.argtypes = [i64, i32, i32]
+    lib.csa_out_proj_workspace_bytes.restype = sz
+    lib.csa_kv_gate_proj.argtypes = [vp, vp, vp, vp, ctypes.c_float, vp, vp, i64, i32, i32, ctypes.c_int, vp]
+    lib.csa_kv_gate_proj.restype = ctypes.c_int
     lib.csa_debug_withhold_attention_loads.argtypes = [ctypes.c_int32]
     lib.csa_debug_withhold_attention_loads.restype = ctypes.c_int
     _lib = lib
@@ -273,3 +280,47 @@ def hca_attend(q, kv, kv_pos0: int, pool, sink, q_pos0: int, rope_dim: int, rope
           _ptr(out), B, S_q, q_pos0, H, D, rope_dim, rope_base, window, ratio, scale, _ptr(ws), wsb,
           _dtype_code(q), _stream(stream))
     return out
+
+
+def csa_out_proj_workspace_bytes(M: int, G: int, r: int) -> int:
+    return int(load_library().csa_out_proj_workspace_bytes(M, G, r))
+
+
+def csa_out_proj(o: torch.Tensor, w_a: torch.Tensor, w_b: torch.Tensor, y=None, workspace=None,
+                 stream=None) -> torch.Tensor:
+    """Grouped low-rank output projection: o [..., H, D] (bf16), w_a [G, r, (H/G)*D],
+    w_b [hidden, G*r] -> y [..., hidden] (see include/csa.h)."""
+    H, D = o.shape[-2], o.shape[-1]
+    G, r, per = w_a.shape
+    hidden = w_b.shape[0]
+    M = o.numel() // (H * D) if H * D else 0
+    if per != (H // G) * D or w_b.shape[1] != G * r:
+        raise ValueError("w_a must be [G, r, (H/G)*D] and w_b [hidden, G*r]")
+    if not (o.dtype == w_a.dtype == w_b.dtype):
+        raise ValueError("o, w_a and w_b must share a dtype")
+    if y is None:
+        y = torch.empty(o.shape[:-2] + (hidden,), dtype=o.dtype, device=o.device)
+    ws, wsb = _ws(csa_out_proj_workspace_bytes(M, G, r), o.device, workspace)
+    _call("csa_out_proj", _ptr(o), _ptr(w_a), _ptr(w_b), _ptr(y), M, H, D, G, r, hidden, _ptr(ws),
+          wsb, _dtype_code(o), _stream(stream))
+    return y
+
+
+def csa_kv_gate_proj(x: torch.Tensor, w_kv: torch.Tensor, w_gate: torch.Tensor,
+                     kv_norm_w: torch.Tensor, eps: float = 1e-6, kv=None, gate=None, stream=None):
+    """The compressor's input projections: x [..., hidden] (bf16), w_kv / w_gate [D, hidden],
+    kv_norm_w [D] -> (kv, gate) [..., D] with kv RMS-normalised (see include/csa.h)."""
+    hidden = x.shape[-1]
+    D = w_kv.shape[0]
+    M = x.numel() // hidden if hidden else 0
+    if w_kv.shape != (D, hidden) or w_gate.shape != (D, hidden) or kv_norm_w.shape != (D,):
+        raise ValueError("w_kv, w_gate must be [D, hidden] and kv_norm_w [D]")
+    if not (x.dtype == w_kv.dtype == w_gate.dtype == kv_norm_w.dtype):
+        raise ValueError("x, weights and kv_norm_w must share a dtype")
+    if kv is None:
+        kv = torch.empty(x.shape[:-1] + (D,), dtype=x.dtype, device=x.device)
+    if gate is None:
+        gate = torch.empty(x.shape[:-1] + (D,), dtype=x.dtype, device=x.device)
+    _call("csa_kv_gate_proj", _ptr(x), _ptr(w_kv), _ptr(w_gate), _ptr(kv_norm_w), float(eps),
+          _ptr(kv), _ptr(gate), M, hidden, D, _dtype_code(x), _stream(stream))
+    return kv, gate

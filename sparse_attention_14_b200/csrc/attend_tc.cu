@@ -68,9 +68,10 @@ struct Meta {
 };
 
 struct Small {
-    uint64_t full[8], free_[4], s_full, p_full, o_full, q_tma, q_full, q_free, meta_full[2];
+    uint64_t full[8], free_[4], s_full, p_full, o_full, q_tma, q_full, q_free, meta_full[2], drain;
     uint32_t tmem_base;
     int abort_;
+    int last_tma[8];   // per key slot: tile counter of its last TMA load, -1 if its last load was not one
     Meta meta[2];
     int32_t rows[kTile];
     float qcs[2][32];
@@ -344,8 +345,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         mbar_init(&sm.q_free, 1);
         mbar_init(&sm.meta_full[0], 1);
         mbar_init(&sm.meta_full[1], 1);
+        mbar_init(&sm.drain, 1);
         fence_mbar_init();
         sm.abort_ = 0;
+        for (int c = 0; c < 8; ++c) sm.last_tma[c] = -1;
     }
     if (warp == 1) tmem_alloc(&sm.tmem_base, 512);
     tc_fence_before();
@@ -356,6 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     if (warp == 0) {
         // ===================================================== loader
         uint32_t g = 0, qc = 0;
+        int q_pending = -1;   // work item whose Q TMA has not been waited for yet
         for (int64_t w = blockIdx.x; w < nw && !sm.abort_ && !withhold; w += gridDim.x, ++qc) {
             const int64_t qi = w / n_split;
             const int64_t qn = (w + gridDim.x) / n_split;   // query of the next work item
@@ -399,11 +403,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 mbar_arrive(&sm.meta_full[qc & 1]);
             }
             // Q of this query: start its TMA now, rotate it once the first tile is issued
-            if (qc > 0 && !mbar_wait(&sm.q_free, (qc - 1) & 1u, kWaitIter)) {
+            if (qc > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(&sm.q_free, (qc - 1) & 1u, kWaitIter))) {
                 atomicOr(&g_attend_tc_status, 1u);
                 sm.abort_ = 1;
                 break;
             }
+            q_pending = (int)qc;
             if (lane == 0) {
                 mbar_expect_tx(&sm.q_tma, kQBytes);
                 for (int c = 0; c < 8; ++c)
@@ -429,8 +434,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             for (int kt = kt0; kt <= kt1 && ok; ++kt) {
                 if (kt == kt0 + 1 || (kt == kt1 && !q_done)) {
                     // rotate the rope channels of Q in place and publish it
-                    ok = mbar_wait(&sm.q_tma, qc & 1u, kWaitIter);
+                    ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.q_tma, qc & 1u, kWaitIter));
                     if (!ok) break;
+                    q_pending = -1;
                     __syncwarp();
                     for (int v = lane; v < kH * 8; v += 32) {
                         const int h = v >> 3, pc = v & 7;
@@ -472,10 +478,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                                    : packed_n ? (int)(qi * kmax + (int64_t)kt * kTile)
                                               : (int)(qg.b * S_kv + (qg.lo_w - kv_pos0) + (int64_t)kt * kTile);
                     for (int c = 0; c < 8 && ok; ++c) {
-                        if ((c & 1) == 0 && g > 0) ok = mbar_wait(&sm.free_[c >> 1], (g - 1) & 1u, kWaitIter);
+                        if ((c & 1) == 0 && g > 0)
+                            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.free_[c >> 1], (g - 1) & 1u, kWaitIter));
                         if (ok && lane == 0) {
                             mbar_expect_tx(&sm.full[c], 16384u);
                             tma_load_2d(s_kv + (uint32_t)c * 16384u, map, 64 * c, y0, &sm.full[c]);
+                            sm.last_tma[c] = (int)g;
                         }
                     }
                 } else {
@@ -498,9 +506,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                         dsto[k] = sw128((uint32_t)xr, (uint32_t)pc);
                     }
                     for (int c = 0; c < 8 && ok; ++c) {
-                        if ((c & 1) == 0 && g > 0) ok = mbar_wait(&sm.free_[c >> 1], (g - 1) & 1u, kWaitIter);
+                        if ((c & 1) == 0 && g > 0)
+                            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.free_[c >> 1], (g - 1) & 1u, kWaitIter));
                         if (!ok) break;
                         const uint32_t dst = s_kv + (uint32_t)c * 16384u;
+                        if (lane == 0) sm.last_tma[c] = -1;
 #pragma unroll
                         for (int k = 0; k < 32; ++k) cp_async16(dst + dsto[k], src[k] + c * 64, 16u);
                         cp_async_commit();
@@ -534,6 +544,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 sm.abort_ = 1;
                 break;
             }
+        }
+        // nothing of this warp may still be landing in shared memory when the CTA exits
+        // (only possible with loads outstanding after an abort): its async copies, and
+        // (bounded) the last TMA of every slot whose last load was one (a completed phase
+        // returns at once) and Q
+        cp_async_wait_all();
+        __syncwarp();
+        if (lane == 0) {
+            for (int c = 0; c < 8; ++c)
+                if (sm.last_tma[c] >= 0) (void)mbar_wait(&sm.full[c], (uint32_t)sm.last_tma[c] & 1u, kWaitIter);
+            if (q_pending >= 0) (void)mbar_wait(&sm.q_tma, (uint32_t)q_pending & 1u, kWaitIter);
         }
     } else if (warp == 1) {
         // ===================================================== MMA issuer
@@ -592,6 +613,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             if (!ok) {
                 atomicOr(&g_attend_tc_status, 1u);
                 sm.abort_ = 1;
+                // let the MMAs already issued finish before the tensor memory is freed
+                mma_commit(&sm.drain);
+                (void)mbar_wait(&sm.drain, 0u, kWaitIter);
             }
         }
     } else {
@@ -608,7 +632,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         for (int64_t w = blockIdx.x; ok && w < nw; w += gridDim.x, ++qc) {
             const int64_t qi = w / n_split;
             const QueryGeom qg = query_geom(qi, S_q, q_pos0, kv_pos0, S_kv, window, packed_n);
-            ok = mbar_wait(&sm.meta_full[qc & 1], (qc >> 1) & 1u, kWaitIter);
+            // every exit after a wait that ran out is decided together (vote at the named
+            // barrier), so no thread is left waiting for the others at a later barrier
+            ok = !named_sync_any(1, kSoftThreads, !mbar_wait(&sm.meta_full[qc & 1], (qc >> 1) & 1u, kWaitIter));
             if (!ok) break;
             const int n_ent = sm.meta[qc & 1].n_ent;
             int kt0, kt1;
@@ -624,7 +650,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             // the running maxima of this thread's 32 heads, read as broadcast 16-byte loads
             const float4 *m4 = reinterpret_cast<const float4 *>(&sm.m_used[hb]);
             for (int kt = kt0; kt < kt1; ++kt, ++g) {
-                ok = mbar_wait(&sm.s_full, g & 1u, kWaitIter);
+                ok = !named_sync_any(1, kSoftThreads, !mbar_wait(&sm.s_full, g & 1u, kWaitIter));
                 if (!ok) break;
                 tc_fence_after();
                 const bool valid = kt < qg.n_wt ? (kt * kTile + x < qg.n_win)
@@ -712,8 +738,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                     pml[st] = sm.m_used[st];
                     pml[kH + st] = sm.red[0][st] + sm.red[1][st] + sm.red[2][st] + sm.red[3][st];
                 }
-                ok = mbar_wait(&sm.o_full, qc & 1u, kWaitIter);
-                named_sync(1, kSoftThreads);
+                ok = !named_sync_any(1, kSoftThreads, !mbar_wait(&sm.o_full, qc & 1u, kWaitIter));
                 if (!ok) break;
                 tc_fence_after();
                 float *po = part + w * (int64_t)(kH * kD);
@@ -739,8 +764,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 if (sk != -INFINITY) l += exp2f(sk * kLog2e - sm.m_used[st]);
                 sm.inv_l[st] = l > 0.f ? 1.f / l : 0.f;
             }
-            ok = mbar_wait(&sm.o_full, qc & 1u, kWaitIter);
-            named_sync(1, kSoftThreads);
+            ok = !named_sync_any(1, kSoftThreads, !mbar_wait(&sm.o_full, qc & 1u, kWaitIter));
             if (!ok) break;
             tc_fence_after();
             __nv_bfloat16 *orow = out + qi * (int64_t)kH * kD;

@@ -9,6 +9,7 @@
 #include "attend.cuh"
 #include "common.cuh"
 #include "index_topk.cuh"
+#include "proj.cuh"
 
 namespace csa {
 
@@ -132,6 +133,7 @@ extern "C" uint32_t csa_device_status(void) {
     uint32_t s = 0;
     if (csa::read_attend_tc_status()) s |= 1u;
     if (csa::read_index_tc_status()) s |= 2u;
+    if (csa::read_proj_tc_status()) s |= 4u;
     return s;
 }
 

@@ -541,4 +541,56 @@ def pin_grouped_out_proj_head_groups():
         assert moved.tolist() == [g == h // (H // G) for g in range(G)], h
 
 
+# ----------------------------------------------------------------------------- input projections
+def pin_kv_gate_proj_one_hot_weights_select_channels():
+    """One-hot weight rows make both projections pick token channels: gate channel d is
+    x[..., perm[d]] (a transposed weight would pick a different channel), and kv is that
+    selection divided by its own RMS, times the norm weight (closed form)."""
+    rng = _rng(60)
+    hidden, D = 9, 5
+    x = rng.standard_normal((2, 3, hidden))
+    perm = rng.permutation(hidden)[:D]
+    w = np.zeros((D, hidden))
+    w[np.arange(D), perm] = 1.0
+    gam = rng.uniform(0.5, 2.0, D)
+    eps = 1e-6
+    kv, gate = oracle.kv_gate_proj(x, w, w, gam, eps)
+    sel = x[..., perm]
+    np.testing.assert_allclose(gate, sel, rtol=0, atol=0)
+    want = sel / np.sqrt((sel ** 2).sum(axis=-1, keepdims=True) / D + eps) * gam
+    np.testing.assert_allclose(kv, want, rtol=1e-13, atol=1e-13)
+
+
+def pin_kv_gate_proj_norm_invariants():
+    """With a unit norm weight and eps = 0 every K=V row has mean square exactly 1 and is
+    unchanged by scaling the token; the gate logits scale with the token; the norm
+    weight multiplies channel by channel after the normalisation."""
+    rng = _rng(61)
+    hidden, D = 16, 8
+    x = rng.standard_normal((4, hidden))
+    wk, wg = rng.standard_normal((D, hidden)), rng.standard_normal((D, hidden))
+    ones = np.ones(D)
+    kv, gate = oracle.kv_gate_proj(x, wk, wg, ones, 0.0)
+    np.testing.assert_allclose((kv ** 2).mean(axis=-1), 1.0, rtol=1e-13)
+    kv3, gate3 = oracle.kv_gate_proj(3.0 * x, wk, wg, ones, 0.0)
+    np.testing.assert_allclose(kv3, kv, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(gate3, 3.0 * gate, rtol=1e-12, atol=1e-12)
+    gam = rng.uniform(0.5, 2.0, D)
+    kvg, _ = oracle.kv_gate_proj(x, wk, wg, gam, 0.0)
+    np.testing.assert_allclose(kvg, kv * gam, rtol=1e-12, atol=1e-12)
+
+
+def pin_kv_gate_proj_epsilon():
+    """eps enters under the square root with the mean square: for a token whose projection
+    is the constant c on every channel, kv = c / sqrt(c^2 + eps) (closed form)."""
+    hidden, D = 4, 6
+    x = np.array([[1.0, 0.0, 0.0, 0.0]])
+    c = 0.01
+    w = np.zeros((D, hidden))
+    w[:, 0] = c
+    kv, gate = oracle.kv_gate_proj(x, w, w, np.ones(D), 1e-4)
+    np.testing.assert_allclose(kv, c / math.sqrt(c * c + 1e-4), rtol=1e-13)
+    np.testing.assert_allclose(gate, c, rtol=0)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
