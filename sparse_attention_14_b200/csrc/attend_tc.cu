@@ -50,7 +50,8 @@ namespace {
 using namespace umma;
 
 constexpr int kD = 512, kH = 64, kTile = 128;
-constexpr int kThreads = 320;                    // warp 0 loads, warp 1 MMA, warps 2-9 softmax
+constexpr int kThreads = 352;                    // warps 0 and 10 load, warp 1 MMA, warps 2-9 softmax
+constexpr int kLoaders = 2;                      // loader li fills the chunk pairs p with p % 2 == li
 constexpr int kSoftThreads = 256;                // two warps per TMEM lane group, 32 heads each
 constexpr uint32_t kKvBytes = kTile * kD * 2;    // 8 chunks x 16 KB
 constexpr uint32_t kQBytes = kH * kD * 2;        // 8 chunks x 8 KB
@@ -81,10 +82,11 @@ struct Small {
     float inv_l[kH];
 };
 
-size_t tc_smem_bytes(int topk) {
-    size_t ent = ((size_t)(topk > 0 ? topk : 1) * 4 + 15) & ~(size_t)15;
-    return 1024 + kOffEnt + ent + sizeof(Small);
+__host__ __device__ __forceinline__ size_t tc_ent_bytes(int topk) {
+    return ((size_t)(topk > 0 ? topk : 1) * 4 + 15) & ~(size_t)15;
 }
+
+size_t tc_smem_bytes(int topk) { return 1024 + kOffEnt + kLoaders * tc_ent_bytes(topk) + sizeof(Small); }
 
 __global__ void rope_rows_kernel(const __nv_bfloat16 *__restrict__ src, __nv_bfloat16 *__restrict__ dst,
                                  int64_t rows, int64_t pos0, int64_t pos_step, int D, RopeTable rope) {
@@ -323,9 +325,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     unsigned char *smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
     const uint32_t base = smem_u32(smem);
     const uint32_t s_kv = base + kOffKv, s_q = base + kOffQ, s_p = base + kOffP;
-    int32_t *ent = reinterpret_cast<int32_t *>(smem + kOffEnt);
-    const size_t ent_bytes = ((size_t)(topk > 0 ? topk : 1) * 4 + 15) & ~(size_t)15;
-    Small &sm = *reinterpret_cast<Small *>(smem + kOffEnt + ent_bytes);
+    const size_t ent_bytes = tc_ent_bytes(topk);
+    Small &sm = *reinterpret_cast<Small *>(smem + kOffEnt + kLoaders * ent_bytes);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const bool withhold = *reinterpret_cast<volatile unsigned int *>(&g_attend_tc_withhold) != 0u;
@@ -356,8 +357,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
 
-    if (warp == 0) {
-        // ===================================================== loader
+    if (warp == 0 || warp == 10) {
+        // ===================================================== loaders
+        // Both loader warps walk every work item; loader li fills the chunk pairs p of each
+        // key tile with p % 2 == li (its own entry list, so neither waits for the other).
+        // Loader 0 also publishes the entry count and brings in and rotates Q.
+        const int li = warp == 0 ? 0 : 1;
+        int32_t *ent = reinterpret_cast<int32_t *>(smem + kOffEnt + li * ent_bytes);
         uint32_t g = 0, qc = 0;
         int q_pending = -1;   // work item whose Q TMA has not been waited for yet
         for (int64_t w = blockIdx.x; w < nw && !sm.abort_ && !withhold; w += gridDim.x, ++qc) {
@@ -398,18 +404,18 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 n_ent = (int)nv;
             }
             __syncwarp();
-            if (lane == 0) {
+            if (li == 0 && lane == 0) {
                 sm.meta[qc & 1].n_ent = n_ent;
                 mbar_arrive(&sm.meta_full[qc & 1]);
             }
             // Q of this query: start its TMA now, rotate it once the first tile is issued
-            if (qc > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(&sm.q_free, (qc - 1) & 1u, kWaitIter))) {
+            if (li == 0 && qc > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(&sm.q_free, (qc - 1) & 1u, kWaitIter))) {
                 atomicOr(&g_attend_tc_status, 1u);
                 sm.abort_ = 1;
                 break;
             }
-            q_pending = (int)qc;
-            if (lane == 0) {
+            if (li == 0) q_pending = (int)qc;
+            if (li == 0 && lane == 0) {
                 mbar_expect_tx(&sm.q_tma, kQBytes);
                 for (int c = 0; c < 8; ++c)
                     tma_load_2d(s_q + (uint32_t)c * 8192u, &map_q, 64 * c, (int)(qi * kH), &sm.q_tma);
@@ -421,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                                      "r"(64 * c), "r"((int)(qn * kH))
                                      : "memory");
             }
-            if (lane < rope.n_pairs) {
+            if (li == 0 && lane < rope.n_pairs) {
                 float cs, sn;
                 rope_cs((double)qg.t, rope.inv_freq[lane], &cs, &sn);
                 sm.qcs[0][lane] = cs;
@@ -432,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             bool q_done = false;
             bool ok = true;
             for (int kt = kt0; kt <= kt1 && ok; ++kt) {
-                if (kt == kt0 + 1 || (kt == kt1 && !q_done)) {
+                if (li == 0 && (kt == kt0 + 1 || (kt == kt1 && !q_done))) {
                     // rotate the rope channels of Q in place and publish it
                     ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.q_tma, qc & 1u, kWaitIter));
                     if (!ok) break;
@@ -478,6 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                                    : packed_n ? (int)(qi * kmax + (int64_t)kt * kTile)
                                               : (int)(qg.b * S_kv + (qg.lo_w - kv_pos0) + (int64_t)kt * kTile);
                     for (int c = 0; c < 8 && ok; ++c) {
+                        if (((c >> 1) & 1) != li) continue;
                         if ((c & 1) == 0 && g > 0)
                             ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.free_[c >> 1], (g - 1) & 1u, kWaitIter));
                         if (ok && lane == 0) {
@@ -505,36 +512,55 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                         src[k] = pool_rot + (qg.b * P + j) * kD + pc * 8;
                         dsto[k] = sw128((uint32_t)xr, (uint32_t)pc);
                     }
-                    for (int c = 0; c < 8 && ok; ++c) {
-                        if ((c & 1) == 0 && g > 0)
-                            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.free_[c >> 1], (g - 1) & 1u, kWaitIter));
-                        if (!ok) break;
-                        const uint32_t dst = s_kv + (uint32_t)c * 16384u;
-                        if (lane == 0) sm.last_tma[c] = -1;
-#pragma unroll
-                        for (int k = 0; k < 32; ++k) cp_async16(dst + dsto[k], src[k] + c * 64, 16u);
-                        cp_async_commit();
-                        if (c >= 3) {
-                            asm volatile("cp.async.wait_group 3;" ::: "memory");
-                            fence_async_smem();
-                            __syncwarp();
-                            if (lane == 0) mbar_arrive(&sm.full[c - 3]);
-                        }
-                    }
-                    if (ok) {
-                        asm volatile("cp.async.wait_group 2;" ::: "memory");
-                        fence_async_smem();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&sm.full[5]);
-                        asm volatile("cp.async.wait_group 1;" ::: "memory");
-                        fence_async_smem();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&sm.full[6]);
+                    // this loader's two pairs: both chunks of a pair in flight, published
+                    // (own copies complete, proxy fence, warp sync, one arrive per chunk) as
+                    // soon as the next pair would have to wait for its slots, else after the
+                    // next pair is issued
+                    int pend = -1;   // first chunk of the pair issued but not yet published
+                    auto publish_pair = [&](int c0) {
                         asm volatile("cp.async.wait_group 0;" ::: "memory");
                         fence_async_smem();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(&sm.full[7]);
+                        if (lane == 0) {
+                            mbar_arrive(&sm.full[c0]);
+                            mbar_arrive(&sm.full[c0 + 1]);
+                        }
+                    };
+                    for (int p = li; p < 4 && ok; p += kLoaders) {
+                        if (g > 0) {
+                            bool fr = __all_sync(0xFFFFFFFFu, mbar_test_wait(&sm.free_[p], (g - 1) & 1u));
+                            if (!fr) {
+                                if (pend >= 0) {
+                                    publish_pair(pend);
+                                    pend = -1;
+                                }
+                                fr = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.free_[p], (g - 1) & 1u, kWaitIter));
+                            }
+                            ok = fr;
+                        }
+                        if (!ok) break;
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int c = 2 * p + h;
+                            const uint32_t dst = s_kv + (uint32_t)c * 16384u;
+                            if (lane == 0) sm.last_tma[c] = -1;
+#pragma unroll
+                            for (int k = 0; k < 32; ++k) cp_async16(dst + dsto[k], src[k] + c * 64, 16u);
+                        }
+                        cp_async_commit();
+                        if (pend >= 0) {
+                            // the previous pair completes before the one just issued
+                            asm volatile("cp.async.wait_group 1;" ::: "memory");
+                            fence_async_smem();
+                            __syncwarp();
+                            if (lane == 0) {
+                                mbar_arrive(&sm.full[pend]);
+                                mbar_arrive(&sm.full[pend + 1]);
+                            }
+                        }
+                        pend = 2 * p;
                     }
+                    if (ok && pend >= 0) publish_pair(pend);
                 }
                 __syncwarp();
                 ++g;
@@ -894,6 +920,8 @@ bool attend_tc_eligible(const AttendArgs &a) {
     if (a.dtype != CSA_BF16 || a.H != kH || a.D != kD) return false;
     if (a.rope_dim > 64) return false;               // rope channels inside the last chunk
     if (a.mode == 0 && a.topk > 2048) return false;
+    // both loaders' entry lists must fit next to the key tile, Q and P in shared memory
+    if (tc_smem_bytes(a.mode == 0 && !attend_tc_packed(a) ? a.topk : 1) > 232448) return false;
     // TMA row coordinates are 32-bit
     if (a.B * a.S_q * kH >= (1ll << 31) || a.B * a.S_kv + kTile >= (1ll << 31) ||
         a.B * a.P >= (1ll << 31))
