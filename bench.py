@@ -86,6 +86,12 @@ def algorithmic_work(spec):
     if spec.index_rope:
         # every indexer query head and every pooled key read and written once
         w["rope_I_bytes"] = 2 * spec.B * (spec.S_q * spec.H_I + spec.P) * spec.d_I * e
+    if spec.proj:
+        import csa_synth as cs
+        M = spec.B * spec.S_q
+        w["proj_in_flops"] = 2 * M * cs.PROJ_HIDDEN * 2 * spec.D
+        w["proj_out_flops"] = 2 * M * (spec.H * spec.D * cs.PROJ_RANK
+                                       + cs.PROJ_GROUPS * cs.PROJ_RANK * cs.PROJ_HIDDEN)
     if spec.cache_update:
         # per compressor (main at D, indexer keys at d_I): the new rows read and stored in the
         # state (kv + gate), the state rows a closing window reaches back to read (kv + gate),
@@ -198,10 +204,27 @@ class LayerRunner:
                                              s.H, s.D, s.topk, dt)
         self.ws_i = torch.empty(max(wsi, 1), dtype=torch.uint8, device=device) if wsi else None
         self.ws_a = torch.empty(max(wsa, 1), dtype=torch.uint8, device=device) if wsa else None
+        self.kv = self.inp["kv"]
+        self.gate = self.inp["gate"]
+        self.y = None
+        if s.proj:
+            import csa_synth as cs
+            self.kv = torch.empty((s.B, s.S_kv, s.D), dtype=dt, device=device)
+            self.gate = torch.empty_like(self.kv)
+            self.y = torch.empty((s.B, s.S_q, cs.PROJ_HIDDEN), dtype=dt, device=device)
+            wso = csa.csa_out_proj_workspace_bytes(s.B * s.S_q, cs.PROJ_GROUPS, cs.PROJ_RANK)
+            self.ws_o = torch.empty(wso, dtype=torch.uint8, device=device)
+
+    @property
+    def result(self):
+        """The step's output: y after the output projection, else the attention output."""
+        return self.y if self.y is not None else self.out
 
     def stages(self):
         s = self.spec
         st = []
+        if s.proj:
+            st.append("proj_in")
         if not s.decode and s.kind != "sliding":
             st.append("compress")
         if s.pool_index_keys:
@@ -213,12 +236,19 @@ class LayerRunner:
         if s.kind == "csa":
             st.append("index")
         st.append("attend")
+        if s.proj:
+            st.append("proj_out")
         return st
 
     def run_stage(self, name):
         s, i, csa = self.spec, self.inp, self.csa
-        if name == "compress":
-            csa.csa_compress(i["kv"], i["gate"], s.m, s.overlap, pool=self.pool)
+        if name == "proj_in":
+            csa.csa_kv_gate_proj(i["x"], i["w_kv"], i["w_gate"], i["kv_norm_w"], 1e-6, kv=self.kv,
+                                 gate=self.gate)
+        elif name == "proj_out":
+            csa.csa_out_proj(self.out, i["w_a"], i["w_b"], y=self.y, workspace=self.ws_o)
+        elif name == "compress":
+            csa.csa_compress(self.kv, self.gate, s.m, s.overlap, pool=self.pool)
         elif name == "compress_I":
             csa.csa_compress(i["kI_tok"], i["gI_tok"], s.m, s.overlap, pool=self.k_I)
         elif name == "rope_I":
@@ -235,10 +265,10 @@ class LayerRunner:
             csa.csa_index_topk(self.q_I, i["w"], self.k_I_rot, s.q_pos0, s.m, s.topk, idx=self.idx,
                                workspace=self.ws_i)
         elif s.kind == "csa":
-            csa.csa_attend(i["q"], i["kv"], s.kv_pos0, self.pool, self.idx, i["sink"], s.q_pos0, s.R,
+            csa.csa_attend(i["q"], self.kv, s.kv_pos0, self.pool, self.idx, i["sink"], s.q_pos0, s.R,
                            s.base, s.W, s.m, s.scale, out=self.out, workspace=self.ws_a)
         else:
-            csa.hca_attend(i["q"], i["kv"], s.kv_pos0, self.pool if s.kind == "hca" else None,
+            csa.hca_attend(i["q"], self.kv, s.kv_pos0, self.pool if s.kind == "hca" else None,
                            i["sink"], s.q_pos0, s.R, s.base, s.W, s.m, s.scale, out=self.out,
                            workspace=self.ws_a)
 
@@ -257,7 +287,9 @@ STAGE_SOURCES = {"compress": ["compress.cu", "common.cuh"],
                  "compress_I": ["compress.cu", "common.cuh"],
                  "rope_I": ["rope.cu", "common.cuh"],
                  "index": ["index_topk.cu", "topk.cuh", "index_tc.cu", "umma.cuh", "common.cuh"],
-                 "attend": ["attend.cu", "attend_tc.cu", "umma.cuh", "common.cuh"]}
+                 "attend": ["attend.cu", "attend_tc.cu", "umma.cuh", "common.cuh"],
+                 "proj_in": ["proj_tc.cu", "umma.cuh", "common.cuh"],
+                 "proj_out": ["proj_tc.cu", "umma.cuh", "common.cuh"]}
 
 
 def ncu_traffic(stage, workload):
@@ -418,7 +450,8 @@ def gpu_arm(args, rank, world, local_rank):
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "algorithmic_bytes_per_launch": wk[key_b]}
     else:
-        key_f = "attend_flops" if dom_stage == "attend" else "index_flops"
+        key_f = {"attend": "attend_flops", "index": "index_flops", "proj_in": "proj_in_flops",
+                 "proj_out": "proj_out_flops"}[dom_stage]
         achieved = wk[key_f] / (dom_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
@@ -458,7 +491,9 @@ def workload_name(w, specs):
             2: "HCA prefill bf16 S=65536", 3: "CSA decode bf16 B=64 at 65536 cached tokens",
             4: "mixed 4-layer stack bf16 S=131072",
             5: "CSA decode step with compressor cache update, bf16 B=64 at 65536 tokens",
-            6: "CSA prefill bf16 S=8192 with the indexer key path (pooled index keys, indexer RoPE 64)"}[w]
+            6: "CSA prefill bf16 S=8192 with the indexer key path (pooled index keys, indexer RoPE 64)",
+            7: "CSA prefill bf16 S=8192 with its projections (kv/gate from hidden 4096, grouped "
+               "output projection 8 groups x 1024 -> 4096)"}[w]
 
 
 def workload_config(w, specs):
@@ -485,8 +520,8 @@ def e2e_arm(args, runners, stage_names, stream, world, dev):
             hv.copy_(v)
             pairs.append((hv, v))
             h2d += v.numel() * v.element_size()
-        ho = torch.empty(r.out.shape, dtype=r.out.dtype, pin_memory=True)
-        d2h += r.out.numel() * r.out.element_size()
+        ho = torch.empty(r.result.shape, dtype=r.result.dtype, pin_memory=True)
+        d2h += r.result.numel() * r.result.element_size()
         host.append((pairs, ho))
     steps = max(1, min(args.steps, 5))
 
@@ -497,7 +532,7 @@ def e2e_arm(args, runners, stage_names, stream, world, dev):
         for li, st in stage_names:
             runners[li].run_stage(st)
         for (pairs, ho), r in zip(host, runners):
-            ho.copy_(r.out, non_blocking=True)
+            ho.copy_(r.result, non_blocking=True)
 
     one()
     torch.cuda.synchronize()
@@ -517,6 +552,60 @@ def e2e_arm(args, runners, stage_names, stream, world, dev):
             "steps": steps}
 
 
+# ----------------------------------------------------------------------------- sharded prefill
+def sharded_arm(args, rank, world, local_rank):
+    """One CSA prefill sequence split over the ranks by query rows (zig-zag chunks), each
+    rank pooling its share of the entries, one all-gather of the entries and one of the
+    index keys (NCCL), then the indexer and attention on its own rows.  Total work is fixed
+    (strong scaling); each step is timed on the device, max over ranks."""
+    import torch
+    import csa_synth as cs
+    import sparse_attention_14_b200 as csa
+    from sparse_attention_14_b200 import shard
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    spec = workload_specs(args.workload)[0]
+    if spec.kind != "csa" or spec.decode or spec.proj or spec.pool_index_keys or len(workload_specs(args.workload)) > 1:
+        raise SystemExit("--shard needs a single-layer CSA prefill workload (1)")
+    csa.load_library()
+    inp = cs.make_inputs(spec, device=dev)   # the same seeded sequence on every rank
+    be = shard.LibraryBackend()
+    for _ in range(args.warmup):
+        shard.prefill_sharded(be, world, rank, inp, spec)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    l0 = csa.launch_count()
+    clk = ClockSampler(local_rank)
+    clk.start()
+    time.sleep(0.3)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    t0.record()
+    for _ in range(args.steps):
+        shard.prefill_sharded(be, world, rank, inp, spec)
+    t1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = clk.stop()
+    launches = csa.launch_count() - l0
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev) / args.steps
+    if rank != 0:
+        return None
+    cfg = dict(workload_config(args.workload, [spec]),
+               parallelism="query-row shards (zig-zag) + NCCL all-gather of pool and k_I")
+    return {"metric": METRIC, "value": round(spec.B * spec.S_q / (ms * 1e-3), 1), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded, the same sequence on every rank)", "config": cfg,
+            "launch": "eager (collectives between the phases)", "gpu_launches": int(launches),
+            "clocks": clocks, "roofline": None, "e2e": None}
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 def oracle_sample_run(spec, rows, inp_cpu=None):
     """The fp64 oracle over the whole hot path for the given query rows (the compressor
@@ -528,6 +617,10 @@ def oracle_sample_run(spec, rows, inp_cpu=None):
     f64 = lambda t: None if t is None else t.double().numpy()
     t0 = time.perf_counter()
     pool = None
+    kv, gate = f64(inp["kv"]), f64(inp["gate"])
+    if spec.proj:
+        kv, gate = oracle.kv_gate_proj(f64(inp["x"]), f64(inp["w_kv"]), f64(inp["w_gate"]),
+                                       f64(inp["kv_norm_w"]), 1e-6)
     k_I = oracle.compress(f64(inp["kI_tok"]), f64(inp["gI_tok"]), spec.m, spec.overlap) \
         if spec.pool_index_keys else f64(inp["k_I"])
     if spec.decode:
@@ -543,7 +636,7 @@ def oracle_sample_run(spec, rows, inp_cpu=None):
                 ent = st.append(f64(new_kv), f64(new_g))
                 cache[:, j0:j0 + ent.shape[1]] = ent
     elif spec.kind != "sliding":
-        pool = oracle.compress(f64(inp["kv"]), f64(inp["gate"]), spec.m, spec.overlap)
+        pool = oracle.compress(kv, gate, spec.m, spec.overlap)
     tpos = np.asarray(rows, dtype=np.int64) + spec.q_pos0
     idx = None
     if spec.kind == "csa":
@@ -553,9 +646,11 @@ def oracle_sample_run(spec, rows, inp_cpu=None):
         else:
             sc = oracle.index_scores(f64(inp["q_I"][:, rows]), f64(inp["w"][:, rows]), k_I, tpos, spec.m)
         idx, _ = oracle.topk(sc, tpos, spec.m, spec.topk)
-    oracle.attend(f64(inp["q"][:, rows]), tpos, f64(inp["kv"]), spec.kv_pos0, pool, spec.m, idx,
-                  f64(inp["sink"]), spec.R, spec.base, spec.W, spec.scale,
-                  "csa" if spec.kind == "csa" else "hca")
+    o = oracle.attend(f64(inp["q"][:, rows]), tpos, kv, spec.kv_pos0, pool, spec.m, idx,
+                      f64(inp["sink"]), spec.R, spec.base, spec.W, spec.scale,
+                      "csa" if spec.kind == "csa" else "hca")
+    if spec.proj:
+        oracle.grouped_out_proj(o, f64(inp["w_a"]), f64(inp["w_b"]))
     return time.perf_counter() - t0
 
 
@@ -563,6 +658,8 @@ def compressor_note(spec):
     """How the sampled oracle run treats the compressor, for the sample description."""
     if spec.decode:
         return "cache update in full" if spec.cache_update else "resident pool (no compressor)"
+    if spec.proj:
+        return "kv/gate projections and compressor in full, output projection on the sampled rows"
     return "no compressor" if spec.kind == "sliding" else "compressor in full"
 
 
@@ -651,11 +748,13 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", type=int, default=1, choices=[0, 1, 2, 3, 4, 5, 6])
+    ap.add_argument("--workload", type=int, default=1, choices=[0, 1, 2, 3, 4, 5, 6, 7])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of CUDA graphs")
+    ap.add_argument("--shard", action="store_true",
+                    help="split one CSA prefill sequence over the ranks by query rows (strong scaling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -678,6 +777,11 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     try:
+        if args.shard:
+            line = sharded_arm(args, rank, world, local_rank)
+            if line is not None:
+                print(json.dumps(line), flush=True)
+            return
         line = gpu_arm(args, rank, world, local_rank)
         if line is not None:
             if world == 1 and not args.no_cpu_baseline:

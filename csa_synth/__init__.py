@@ -41,7 +41,7 @@ import torch
 
 TENSOR_IDS = {"q": 0, "kv": 1, "gate": 2, "q_I": 3, "k_I": 4, "w": 5, "sink": 6, "pool": 7,
               "gate_new": 8, "state": 9, "state_I": 10, "kI_new": 11, "gI_new": 12,
-              "kI_tok": 13, "gI_tok": 14}
+              "kI_tok": 13, "gI_tok": 14, "x": 15, "proj": 16}
 RMS_EPS = 1e-6
 
 
@@ -60,6 +60,10 @@ class LayerSpec:
     pool_index_keys=True (prefill CSA) pools k_I in the step from per-token index keys
     by the same gated compressor; index_rope > 0 rotates that many trailing channels of
     every indexer query head (at t) and pooled key (at j*m) before scoring.
+    proj=True (prefill) adds the projections around the layer to the step: the raw K=V
+    rows and gate logits come from the token states x [B,S,hidden] by the compressor's
+    kv_proj + kv_norm and gate_proj, and the attention output goes through the grouped
+    low-rank output projection to y [B,S,hidden].
     """
 
     name: str
@@ -84,6 +88,7 @@ class LayerSpec:
     cache_update: bool = False
     pool_index_keys: bool = False
     index_rope: int = 0
+    proj: bool = False
     workload: int = 0
     layer: int = 0
 
@@ -153,6 +158,9 @@ def mixed_stack(S: int = 131072) -> List[LayerSpec]:
     ]
 
 
+CSA_PREFILL_PROJ = dataclasses.replace(CSA_PREFILL, name="csa_prefill_s8192_proj", proj=True,
+                                       workload=7)
+
 WORKLOADS: Dict[int, List[LayerSpec]] = {
     0: [TINY_CSA],
     1: [CSA_PREFILL],
@@ -161,6 +169,7 @@ WORKLOADS: Dict[int, List[LayerSpec]] = {
     4: mixed_stack(),
     5: [CSA_DECODE_STEP],
     6: [CSA_PREFILL_INDEX_KEYS],
+    7: [CSA_PREFILL_PROJ],
 }
 
 
@@ -206,6 +215,13 @@ def make_inputs(spec: LayerSpec, device="cpu") -> Dict[str, Optional[torch.Tenso
         out["kI_tok"] = _rms_rows(_randn((spec.B, spec.S_kv, spec.d_I), spec.seed("kI_tok"),
                                          device)).to(dt)
         out["gI_tok"] = _randn((spec.B, spec.S_kv, spec.d_I), spec.seed("gI_tok"), device).to(dt)
+    if spec.proj:
+        assert not spec.decode and spec.kind != "sliding"
+        # the step makes the raw K=V rows and gates itself, from x
+        out["kv"] = out["gate"] = None
+        out["x"] = _randn((spec.B, spec.S_kv, PROJ_HIDDEN), spec.seed("x"), device).to(dt)
+        out.update(proj_weights(spec.H, spec.D, PROJ_GROUPS, PROJ_RANK, PROJ_HIDDEN, dt,
+                                spec.seed("proj"), device=device))
     if spec.cache_update:
         assert spec.decode and spec.kind != "sliding" and spec.kv_pos0 + spec.S_kv == spec.q_pos0 + spec.S_q
         L = spec.ring

@@ -81,3 +81,41 @@ def test_projections_reject_unsupported_shapes():
     w = torch.zeros((256, 100), dtype=torch.bfloat16, device=DEV)
     with pytest.raises(csa.CsaError):
         csa.csa_kv_gate_proj(x, w, w, torch.ones(256, dtype=torch.bfloat16, device=DEV))
+
+
+def test_workload7_layer_with_projections_sampled():
+    """The CSA prefill layer with its projections at full size (S = 8192, hidden 4096), in
+    the benchmark's call sequence, checked stage by stage on sampled rows: kv/gate against
+    the oracle's projections of the same token rows, the pool over the GPU's kv/gate, the
+    top-k sets (tie band), the attention over the GPU's pool, rows and validated top-k, and
+    the output projection of the GPU's attention output."""
+    from parity_util import check_topk, kk_rows
+    spec = cs.WORKLOADS[7][0]
+    inp = cs.make_inputs(spec, device=DEV)
+    kv, gate = csa.csa_kv_gate_proj(inp["x"], inp["w_kv"], inp["w_gate"], inp["kv_norm_w"], 1e-6)
+    pool = csa.csa_compress(kv, gate, spec.m, spec.overlap)
+    idx = csa.csa_index_topk(inp["q_I"], inp["w"], inp["k_I"], spec.q_pos0, spec.m, spec.topk)
+    out = csa.csa_attend(inp["q"], kv, spec.kv_pos0, pool, idx, inp["sink"], spec.q_pos0, spec.R,
+                         spec.base, spec.W, spec.m, spec.scale)
+    y = csa.csa_out_proj(out, inp["w_a"], inp["w_b"])
+    torch.cuda.synchronize()
+    assert csa.device_status() == 0
+    rows = cs.sample_rows(spec, n_random=48)
+    rt = torch.tensor(rows, device=DEV)
+    kv_ref, gate_ref = oracle.kv_gate_proj(to_np(inp["x"][0, rt]), to_np(inp["w_kv"]),
+                                           to_np(inp["w_gate"]), to_np(inp["kv_norm_w"]), 1e-6)
+    assert rel_err(to_np(kv[0, rt]), kv_ref) <= TOL["bf16"]
+    assert rel_err(to_np(gate[0, rt]), gate_ref) <= TOL["bf16"]
+    kv_h = to_np(kv)
+    assert rel_err(to_np(pool), oracle.compress(kv_h, to_np(gate), spec.m, spec.overlap)) <= TOL["bf16"]
+    tpos = np.asarray(rows, dtype=np.int64) + spec.q_pos0
+    sc = oracle.index_scores(to_np(inp["q_I"][:, rt]), to_np(inp["w"][:, rt]), to_np(inp["k_I"]), tpos,
+                             spec.m)
+    o_idx, _ = oracle.topk(sc, tpos, spec.m, spec.topk)
+    g_idx = idx[:, rt].cpu().numpy()
+    check_topk(g_idx[0], o_idx[0], sc[0], kk_rows(spec, rows))
+    ref = oracle.attend(to_np(inp["q"][:, rt]), tpos, kv_h, spec.kv_pos0, to_np(pool), spec.m, g_idx,
+                        to_np(inp["sink"]), spec.R, spec.base, spec.W, spec.scale, "csa")
+    assert rel_err(to_np(out[:, rt]), ref) <= TOL["bf16"]
+    y_ref = oracle.grouped_out_proj(to_np(out[:, rt]), to_np(inp["w_a"]), to_np(inp["w_b"]))
+    assert rel_err(to_np(y[:, rt]), y_ref) <= TOL["bf16"]
