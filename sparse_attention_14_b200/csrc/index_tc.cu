@@ -92,7 +92,7 @@ __device__ __forceinline__ float key_to_float(uint32_t key) {
 // ------------------------------------------------------------------ group selection
 // All GS threads of a group (named barrier `bar`) find a threshold T such that exactly k
 // of n unique 64-bit keys are >= T, by an MSB-first radix select, 8 bits per pass.  The
-// histogram is built with warp-aggregated atomics (lanes with the same bin add once), and
+// histogram is built with plain shared-memory atomics, four keys in flight per thread, and
 // the select stops at the first pass whose chosen bin is taken whole: T is then that
 // bin's prefix with the lower bits zero.
 template <int GS>
@@ -112,17 +112,20 @@ __device__ unsigned long long group_kth(const unsigned long long *a, int n, int 
         const unsigned long long prefix = ms.sel_prefix[g];
         const unsigned remaining = ms.sel_remaining[g];
         const unsigned long long mask = shift == 56 ? 0ull : (~0ull << (shift + 8));
-        for (int e0 = 0; e0 < n; e0 += GS) {
-            const int e = e0 + gt;
-            unsigned long long key = 0ull;
-            bool m = false;
-            if (e < n) {
-                key = a[e];
-                m = (key & mask) == prefix;
+        // plain shared-memory atomics, four keys in flight per thread (no warp-wide step
+        // between a key's load and its count)
+        for (int e0 = gt; e0 < n; e0 += 4 * GS) {
+            unsigned long long key[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = e0 + u * GS;
+                key[u] = e < n ? a[e] : 0ull;
             }
-            const unsigned bin = (unsigned)(key >> shift) & 255u;
-            const unsigned peers = __match_any_sync(0xFFFFFFFFu, m ? bin : 0xFFFFFFFFu);
-            if (m && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (unsigned)__popc(peers));
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = e0 + u * GS;
+                if (e < n && (key[u] & mask) == prefix) atomicAdd(&hist[(unsigned)(key[u] >> shift) & 255u], 1u);
+            }
         }
         named_sync(bar, GS);
         const int hi_bin = 256 - gt * BPT;   // my bins: [hi_bin - BPT, hi_bin)
