@@ -123,8 +123,9 @@ def prefill(name, dtype, S, H, D, R, base, W, m, kind, H_I=0, d_I=0, topk=0, B=1
 
 # The five workloads.  Bases: one RoPE base per layer, used for q, window keys, entries
 # and the output de-rotation; compressed layers use the slower 160000 base and the
-# sliding-only layer the main 10000 base (HF PR #45616 "compress_rope_parameters ...
-# rope_theta swapped"; mlx-lm PR #1797 "two rotation speeds").
+# sliding-only layer the main 10000 base (HF PR #45616, note on compress_rope_parameters:
+# compressed layers swap in their own rope_theta; mlx-lm PR #1797: two rotation speeds,
+# one per kind of layer).
 TINY_CSA = prefill("tiny_csa_f32", "f32", S=256, H=8, D=64, R=16, base=10000.0, W=32,
                    m=4, kind="csa", H_I=4, d_I=32, topk=16, workload=0)
 CSA_PREFILL = prefill("csa_prefill_s8192", "bf16", S=8192, H=64, D=512, R=64,

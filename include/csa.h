@@ -54,9 +54,10 @@ typedef enum {
 } csa_status_t;
 
 /*
- * csa_compress -- KV Compressor (HF docs model_doc/deepseek_v4 section 2.3.1 "low
- * compression with overlapping windows", 2.3.2 "m'=128, non-overlapping"; HF PR #45616
- * "Compressor.forward always returns a tensor ... empty when no window has closed").
+ * csa_compress -- KV Compressor (HF docs model_doc/deepseek_v4 section 2.3.1: CSA pools
+ * with ratio m=4 over overlapping windows; section 2.3.2: HCA pools with m'=128 over
+ * non-overlapping windows; HF PR #45616, compressor note: the module returns a tensor,
+ * empty before the first window closes).
  *
  *   pool[b,j,d] = sum_{s in Win_j} softmax_{s in Win_j}(gate[b,s,d]) * kv[b,s,d]
  *   Win_j = [max(0,(j-1)*ratio), (j+1)*ratio) if overlap, else [j*ratio, (j+1)*ratio)
@@ -71,10 +72,10 @@ csa_status_t csa_compress(const void *kv, const void *gate, void *pool, int64_t 
                           void *stream);
 
 /*
- * csa_compress_append -- decode-time compressor cache update (HF PR #45616 "Compressor/
- * Indexer statefulness ... per-layer compressor_state and indexer_state (buffer_kv,
- * buffer_gate, pooled_kv)", "_accumulate_windows and _update_pool ... single cache update
- * per call"; HF docs model_doc/deepseek_v4 section "Cache layers": buffer / pool / counter,
+ * csa_compress_append -- decode-time compressor cache update (HF PR #45616, note on
+ * compressor and indexer state: each layer keeps, per compressor, a buffer of raw kv and
+ * gate rows and the pooled cache, and one call accumulates the new rows and updates the
+ * pool once; HF docs model_doc/deepseek_v4 section "Cache layers": buffer, pool, counter,
  * plus the overlap state for CSA).  The same call serves the main compressor (D = head_dim)
  * and the indexer's key compressor (D = d_I), each with its own state.
  *
@@ -133,9 +134,9 @@ csa_status_t csa_index_topk(const void *q_I, const void *w, const void *k_I, int
 
 /*
  * csa_rope_rows -- interleaved-pair partial RoPE over rows, for the Lightning Indexer's
- * own rotary embedding (TransformerLens deepseek_v4 bridge: the indexer carries a
- * rotary_emb; HF PR #45616 "RoPE apply: interleaved-pair rotation"; HF docs
- * model_doc/deepseek_v4 section 2.3.3).  With it the indexer scores rotated queries
+ * own rotary embedding (TransformerLens deepseek_v4 bridge: the indexer's submodules
+ * include a rotary embedding; HF PR #45616, note on the RoPE application: interleaved
+ * channel pairs are rotated; HF docs model_doc/deepseek_v4 section 2.3.3).  With it the indexer scores rotated queries
  * against rotated pooled keys, so a score depends on t - j*ratio:
  *
  *   out[r] = Rot(x[r], pos0 + ((r / group) mod period) * step),  r in [0, rows)
@@ -163,10 +164,11 @@ size_t csa_index_topk_workspace_bytes(int64_t B, int64_t S_q, int64_t q_pos0, in
 /*
  * csa_attend -- CSA attention: shared K=V single-head MQA over the sliding window plus
  * the selected entries, with sink, partial RoPE and output de-rotation (HF docs
- * model_doc/deepseek_v4 section 2.3 "shared K=V Multi-Query Attention", "partial
- * rotary positional embedding ... position -i (eq. 26)", "learnable attention sink per
- * head (eq. 27)", "additional branch of sliding window attention"; HF PR #45616 "port
- * eager_attention_forward from GPT-OSS", un-rotation of the output rope slice).
+ * model_doc/deepseek_v4 section 2.3: one K=V head shared by all query heads; section
+ * 2.3.3 and eq. 26: partial RoPE, and the output's rope slice turned back by the query's
+ * position; eq. 27: one learned sink logit per head; the sliding window as an extra
+ * branch of keys; HF PR #45616: the eager attention is the GPT-OSS one, with the output
+ * rope slice un-rotated).
  *
  * For query row i at t = q_pos0 + i, head h:
  *   keys K_t = { raw rows r : t - window < kv_pos0 + r <= t, 0 <= r < S_kv }
@@ -193,10 +195,11 @@ csa_status_t csa_attend(const void *q, const void *kv, int64_t S_kv, int64_t kv_
                         size_t workspace_bytes, csa_dtype_t dtype, void *stream);
 
 /*
- * hca_attend -- HCA attention (HF docs model_doc/deepseek_v4 section 2.3.2 "no indexer
- * -- every pool entry participates"; "Attention mask layout": entry w is visible iff
- * w < (t+1)//m).  Same as csa_attend with K_t's entry part replaced by every visible
- * entry j < n_vis(t).  P == 0 gives the sliding-window-only layer ("sliding_attention").
+ * hca_attend -- HCA attention (HF docs model_doc/deepseek_v4 section 2.3.2: no indexer,
+ * the query attends to every compressed entry; section "Attention mask layout": entry w
+ * is visible to the query at t iff w < (t+1)//m).  Same as csa_attend with K_t's entry
+ * part replaced by every visible entry j < n_vis(t).  P == 0 gives the sliding-window-only
+ * layer.
  */
 csa_status_t hca_attend(const void *q, const void *kv, int64_t S_kv, int64_t kv_pos0,
                         const void *pool, int64_t P, const float *sink, void *out, int64_t B,

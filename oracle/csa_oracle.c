@@ -108,11 +108,12 @@ int orc_compress(const double *kv, const double *gate, double *pool,
 }
 
 /* ---------------------------------------------------------------------------------
- * Stateful compressor for decode, [HF-PR] "Compressor/Indexer statefulness ... state
- * lives on a new DeepseekV4Cache ... per-layer compressor_state and indexer_state dicts
- * (buffer_kv, buffer_gate, pooled_kv)" and "_accumulate_windows and _update_pool ...
- * single cache update per call"; [HF-DOC] "Cache layers": the HCA cache keeps a
- * compressor buffer / pool / counter, the CSA cache the same plus its overlap state.
+ * Stateful compressor for decode, [HF-PR] note on compressor and indexer state: the state
+ * lives in the model's cache, one compressor state and one indexer state per layer, each
+ * a buffer of raw kv and gate rows plus the pooled cache, and one call accumulates the
+ * new rows and updates the pool once; [HF-DOC] section "Cache layers": the HCA cache
+ * keeps a compressor buffer, pool and counter, the CSA cache the same plus its overlap
+ * state.
  *
  * State of sequence b (the layout is this oracle's own):
  *   buf_kv, buf_gate [B, m, D]  tokens of the window that has not closed yet; the first

@@ -1,7 +1,8 @@
 // compress.cu -- KV Compressor: learned gated pooling of raw K=V rows into compressed
-// entries (HF docs model_doc/deepseek_v4, section 2.3.1 "compressed sparse attention:
-// m=4, overlapping windows" and 2.3.2 "heavily compressed attention: m'=128,
-// non-overlapping windows"; HF PR #45616 "Compressor.forward always returns a tensor").
+// entries (HF docs model_doc/deepseek_v4, section 2.3.1: CSA compresses every m=4 tokens
+// with overlapping windows; section 2.3.2: HCA compresses every m'=128 tokens without
+// overlap; HF PR #45616, compressor note: the forward returns a tensor even when no
+// window has closed yet, an empty one).
 //
 // pool[b,j,d] = sum_{s in Win_j} exp(g[s,d] - M) kv[s,d] / sum_{s in Win_j} exp(g[s,d] - M)
 //
@@ -250,10 +251,10 @@ csa_status_t launch_compress(const T *kv, const T *gate, T *pool, int64_t B, int
 }
 
 // ---------------------------------------------------------------- decode-time cache update
-// HF PR #45616 "Compressor/Indexer statefulness ... per-layer compressor_state and
-// indexer_state (buffer_kv, buffer_gate, pooled_kv)" and "_accumulate_windows and
-// _update_pool ... single cache update per call"; HF docs "Cache layers" (buffer / pool /
-// counter, plus the CSA overlap state).
+// HF PR #45616, note on compressor and indexer state: each layer keeps a compressor state
+// and an indexer state (a buffer of raw kv and gate rows and the pooled cache), and one
+// call accumulates the new rows and updates the pool once; HF docs model_doc/deepseek_v4,
+// section "Cache layers": buffer, pool and counter, plus the overlap state for CSA.
 //
 // The state of a sequence is a ring of its last L = (1+overlap)*ratio raw rows, kv and
 // gate, the row of position p in slot p mod L: exactly the rows that a window closing in

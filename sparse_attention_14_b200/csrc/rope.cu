@@ -1,8 +1,8 @@
 // rope.cu -- interleaved-pair partial RoPE over rows, for the Lightning Indexer's own
-// rotary embedding (TransformerLens deepseek_v4 bridge: the indexer carries a rotary_emb
-// next to its kv_proj / gate_proj / kv_norm; HF PR #45616 "RoPE apply: interleaved-pair
-// rotation"; HF docs model_doc/deepseek_v4 section 2.3.3, partial RoPE on the last
-// channels of each head).
+// rotary embedding (TransformerLens deepseek_v4 bridge: the indexer's submodules include
+// a rotary embedding beside kv_proj / gate_proj / kv_norm; HF PR #45616, its note on the
+// RoPE application, which rotates interleaved channel pairs; HF docs model_doc/deepseek_v4
+// section 2.3.3: the rotation covers only the last channels of each head).
 //
 //   out[r] = Rot(x[r], pos0 + ((r / group) mod period) * step)
 //
