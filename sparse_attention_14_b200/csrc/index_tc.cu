@@ -445,23 +445,22 @@ __global__ void __launch_bounds__(Cfg<QB>::kThreads, Cfg<QB>::kMinBlocks) index_
 #pragma unroll
             for (int qq = 0; qq < C::QPT; ++qq) {
                 const int q = qa + qq;
-                float v[32];
-                float s = 0.f;
+                // all of this query's head columns in flight at once, one wait
+                float v[C::CPT];
 #pragma unroll
-                for (int hc = 0; hc < C::CPT / 32; ++hc) {
-                    tmem_ld32(trow + (uint32_t)(q * 64 + cb + hc * 32), v);
-                    tmem_ld_wait();
-                    const float4 *wq = reinterpret_cast<const float4 *>(w_s + q * 64 + cb + hc * 32);
+                for (int hc = 0; hc < C::CPT / 32; ++hc) tmem_ld32(trow + (uint32_t)(q * 64 + cb + hc * 32), v + 32 * hc);
+                tmem_ld_wait();
+                float s4[4] = {0.f, 0.f, 0.f, 0.f};
+                const float4 *wq = reinterpret_cast<const float4 *>(w_s + q * 64 + cb);
 #pragma unroll
-                    for (int h4 = 0; h4 < 8; ++h4) {
-                        const float4 ww = wq[h4];
-                        s = fmaf(ww.x, fmaxf(v[4 * h4 + 0], 0.f), s);
-                        s = fmaf(ww.y, fmaxf(v[4 * h4 + 1], 0.f), s);
-                        s = fmaf(ww.z, fmaxf(v[4 * h4 + 2], 0.f), s);
-                        s = fmaf(ww.w, fmaxf(v[4 * h4 + 3], 0.f), s);
-                    }
+                for (int h4 = 0; h4 < C::CPT / 4; ++h4) {
+                    const float4 ww = wq[h4];
+                    s4[0] = fmaf(ww.x, fmaxf(v[4 * h4 + 0], 0.f), s4[0]);
+                    s4[1] = fmaf(ww.y, fmaxf(v[4 * h4 + 1], 0.f), s4[1]);
+                    s4[2] = fmaf(ww.z, fmaxf(v[4 * h4 + 2], 0.f), s4[2]);
+                    s4[3] = fmaf(ww.w, fmaxf(v[4 * h4 + 3], 0.f), s4[3]);
                 }
-                sc[qq] = s;
+                sc[qq] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
             }
             tc_fence_before();
             __syncwarp();
