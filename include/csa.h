@@ -219,12 +219,15 @@ csa_status_t hca_attend(const void *q, const void *kv, int64_t S_kv, int64_t kv_
  * latency-critical serving loop that must not allocate per call because cudaMalloc can
  * synchronise the device.  This entry point takes the same arguments as csa_attend
  * minus the workspace and allocates nothing: its scratch (the rotated window rows and
- * compressed entries of the call) lives in one fixed device array of 16 MiB compiled
+ * compressed entries and the rotated query chunks of the call) lives in one fixed device
+ * array of 16 MiB compiled
  * into the library, created on each GPU that loads the library and held until the
  * process exits.  The caller still provides q, kv, pool, idx, sink and out.
  *
- *  - Handles the bf16, H = 64, D = 512 prefill shape (S_q * 64 >= S_kv + P) with
- *    B * (S_kv + P) <= 16384 rows of scratch; anything else returns
+ *  - Handles the bf16, H = 64, D = 512 prefill shape (S_q * 64 >= S_kv + P) whose
+ *    scratch fits the array: B * (S_kv + P) rotated key rows of 1 KB plus B * S_q * 64
+ *    rotated query chunks of 128 B (each part rounded up to 256 B) within 16 MiB, e.g.
+ *    B = 1, S_q = S_kv = 1024, P = 256 (9.3 MiB); anything else returns
  *    CSA_ERR_UNSUPPORTED with a message naming the limit.
  *  - The first call on a device looks up the array's device address (set-up, once per
  *    device, with that device current); make that first call before any stream capture.

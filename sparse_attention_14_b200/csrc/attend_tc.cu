@@ -6,13 +6,15 @@
 // mask layout" for the key sets).
 //
 // Design (one persistent CTA per SM, one query at a time, 64 heads per query):
-//  * keys are rotated once per call into the workspace (rope_rows_kernel); a key tile is
-//    128 rows of 1 KB in 128B-swizzled shared memory, split into eight 16 KB chunks
-//    (64 dims each) with their own mbarriers: window rows (contiguous) arrive by 2-D TMA
-//    boxes, selected entries by 16-byte async copies from the loader warp;
-//  * warp roles: warp 0 loads (idx compaction, Q by TMA with its rope channels rotated in
-//    place, key tiles), warp 1 issues the MMAs (one thread), warps 2-9 run the softmax
-//    and the epilogue (two warps per TMEM lane group, 32 heads each);
+//  * keys are rotated once per call into the workspace (rope_rows_kernel), and so is the
+//    last 64-channel chunk of every query row (rope_q_chunk_kernel), which holds the rope
+//    channels; a key tile is 128 rows of 1 KB in 128B-swizzled shared memory, split into
+//    eight 16 KB chunks (64 dims each) with their own mbarriers: window rows (contiguous)
+//    arrive by 2-D TMA boxes, selected entries by 16-byte async copies from the loaders;
+//  * warp roles: warps 0 and 10 load (each its own half of every tile's chunk pairs and
+//    its own copy of the compacted entry list; warp 0 also Q by TMA: seven chunks from q,
+//    the rotated chunk from the workspace), warp 1 issues the MMAs (one thread), warps 2-9
+//    run the softmax and the epilogue (two warps per TMEM lane group, 32 heads each);
 //  * the MMAs are transposed so that M = 128 keys / 128 head-dims (M=128 tcgen05 tiles)
 //    and N = 64 heads:
 //      S^T[key, h]  = K[key, :] . Qr[h, :]          (A = key tile, K-major; B = Q, K-major)
@@ -69,13 +71,12 @@ struct Meta {
 };
 
 struct Small {
-    uint64_t full[8], free_[4], s_full, p_full, o_full, q_tma, q_full, q_free, meta_full[2], drain;
+    uint64_t full[8], free_[4], s_full, p_full, o_full, q_tma, q_free, meta_full[2], drain;
     uint32_t tmem_base;
     int abort_;
     int last_tma[8];   // per key slot: tile counter of its last TMA load, -1 if its last load was not one
     Meta meta[2];
     int32_t rows[kTile];
-    float qcs[2][32];
     alignas(16) float m_used[kH];
     float alpha[kH];
     float red[4][kH];
@@ -115,6 +116,33 @@ __global__ void rope_rows_kernel(const __nv_bfloat16 *__restrict__ src, __nv_bfl
         }
     }
     store8(dst + ((int64_t)b * rows + r) * D + pc * 8, x);
+}
+
+// The last 64 channels of every query row (query, head), rotated at the query's position,
+// into a [rows, 64] buffer: the attention loads Q's last 64-column chunk from there, so
+// no rotation of Q sits between a query's Q load and its first MMAs.  Only channels at
+// or after rope.first (>= 448 on this path) are turned; the others are copied.
+__global__ void rope_q_chunk_kernel(const __nv_bfloat16 *__restrict__ q, __nv_bfloat16 *__restrict__ q7,
+                                    int64_t rows, int64_t S_q, int64_t q_pos0, RopeTable rope) {
+    const int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t r = v >> 3;
+    if (r >= rows) return;
+    const int pc = (int)(v & 7);
+    float x[8];
+    load8(q + r * kD + 7 * 64 + pc * 8, x);
+    const double pos = (double)(q_pos0 + (r / kH) % S_q);
+#pragma unroll
+    for (int c = 0; c < 8; c += 2) {
+        const int d = 7 * 64 + pc * 8 + c;
+        if (d >= rope.first) {
+            float cs, sn;
+            rope_cs(pos, rope.inv_freq[(d - rope.first) >> 1], &cs, &sn);
+            const float a = x[c], bb = x[c + 1];
+            x[c] = a * cs - bb * sn;
+            x[c + 1] = a * sn + bb * cs;
+        }
+    }
+    store8(q7 + r * 64 + pc * 8, x);
 }
 
 // Decode-sized calls: gather each query's keys (window rows, then its valid entries in
@@ -313,8 +341,9 @@ __device__ __forceinline__ QueryGeom query_geom(int64_t qi, int64_t S_q, int64_t
 }
 
 __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
-    const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kv,
-    const __grid_constant__ CUtensorMap map_pool, const __nv_bfloat16 *__restrict__ pool_rot, int64_t S_kv,
+    const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_q7,
+    const __grid_constant__ CUtensorMap map_kv, const __grid_constant__ CUtensorMap map_pool,
+    const __nv_bfloat16 *__restrict__ pool_rot, int64_t S_kv,
     int64_t kv_pos0, int64_t P,
     const int32_t *__restrict__ idx, int topk, int mode, const float *__restrict__ sink,
     __nv_bfloat16 *__restrict__ out, int64_t B, int64_t S_q, int64_t q_pos0, int window, int ratio,
@@ -342,7 +371,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         mbar_init(&sm.p_full, kSoftThreads);
         mbar_init(&sm.o_full, 1);
         mbar_init(&sm.q_tma, 1);
-        mbar_init(&sm.q_full, 1);
         mbar_init(&sm.q_free, 1);
         mbar_init(&sm.meta_full[0], 1);
         mbar_init(&sm.meta_full[1], 1);
@@ -365,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         const int li = warp == 0 ? 0 : 1;
         int32_t *ent = reinterpret_cast<int32_t *>(smem + kOffEnt + li * ent_bytes);
         uint32_t g = 0, qc = 0;
-        int q_pending = -1;   // work item whose Q TMA has not been waited for yet
+        int q_pending = -1;   // work item of the last Q TMA issued (its phase completes when it lands)
         for (int64_t w = blockIdx.x; w < nw && !sm.abort_ && !withhold; w += gridDim.x, ++qc) {
             const int64_t qi = w / n_split;
             const int64_t qn = (w + gridDim.x) / n_split;   // query of the next work item
@@ -408,7 +436,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 sm.meta[qc & 1].n_ent = n_ent;
                 mbar_arrive(&sm.meta_full[qc & 1]);
             }
-            // Q of this query: start its TMA now, rotate it once the first tile is issued
+            // Q of this query (its rope channels already rotated by rope_q_chunk_kernel): start
+            // its TMA once the previous query's scores are done; the MMA issuer waits for it
             if (li == 0 && qc > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(&sm.q_free, (qc - 1) & 1u, kWaitIter))) {
                 atomicOr(&g_attend_tc_status, 1u);
                 sm.abort_ = 1;
@@ -417,62 +446,26 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             if (li == 0) q_pending = (int)qc;
             if (li == 0 && lane == 0) {
                 mbar_expect_tx(&sm.q_tma, kQBytes);
-                for (int c = 0; c < 8; ++c)
+                for (int c = 0; c < 7; ++c)
                     tma_load_2d(s_q + (uint32_t)c * 8192u, &map_q, 64 * c, (int)(qi * kH), &sm.q_tma);
+                tma_load_2d(s_q + 7u * 8192u, &map_q7, 0, (int)(qi * kH), &sm.q_tma);
                 // bring the next query's Q into L2 while this query runs
-                if (w + gridDim.x < nw)
-                    for (int c = 0; c < 8; ++c)
+                if (w + gridDim.x < nw) {
+                    for (int c = 0; c < 7; ++c)
                         asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
                                          reinterpret_cast<uint64_t>(&map_q)),
                                      "r"(64 * c), "r"((int)(qn * kH))
                                      : "memory");
-            }
-            if (li == 0 && lane < rope.n_pairs) {
-                float cs, sn;
-                rope_cs((double)qg.t, rope.inv_freq[lane], &cs, &sn);
-                sm.qcs[0][lane] = cs;
-                sm.qcs[1][lane] = sn;
+                    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
+                                     reinterpret_cast<uint64_t>(&map_q7)),
+                                 "r"(0), "r"((int)(qn * kH))
+                                 : "memory");
+                }
             }
             int kt0, kt1;
             split_range(qg.n_wt + (n_ent + kTile - 1) / kTile, n_split, (int)(w % n_split), &kt0, &kt1);
-            bool q_done = false;
             bool ok = true;
             for (int kt = kt0; kt <= kt1 && ok; ++kt) {
-                if (li == 0 && (kt == kt0 + 1 || (kt == kt1 && !q_done))) {
-                    // rotate the rope channels of Q in place and publish it
-                    ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.q_tma, qc & 1u, kWaitIter));
-                    if (!ok) break;
-                    q_pending = -1;
-                    __syncwarp();
-                    for (int v = lane; v < kH * 8; v += 32) {
-                        const int h = v >> 3, pc = v & 7;
-                        const int d0 = 7 * 64 + pc * 8;
-                        if (d0 + 8 <= rope.first) continue;
-                        const uint32_t addr = s_q + 7u * 8192u + sw128((uint32_t)h, (uint32_t)pc);
-                        uint32_t w0, w1, w2, w3;
-                        asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3) : "r"(addr));
-                        uint32_t wv[4] = {w0, w1, w2, w3};
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const int d = d0 + 2 * k;
-                            if (d >= rope.first) {
-                                __nv_bfloat162 hv = *reinterpret_cast<__nv_bfloat162 *>(&wv[k]);
-                                float2 f = __bfloat1622float2(hv);
-                                const int pr = (d - rope.first) >> 1;
-                                const float cs = sm.qcs[0][pr], sn = sm.qcs[1][pr];
-                                __nv_bfloat162 r = __floats2bfloat162_rn(f.x * cs - f.y * sn, f.x * sn + f.y * cs);
-                                wv[k] = *reinterpret_cast<uint32_t *>(&r);
-                            }
-                        }
-                        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(wv[0]), "r"(wv[1]),
-                                     "r"(wv[2]), "r"(wv[3])
-                                     : "memory");
-                    }
-                    fence_async_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm.q_full);
-                    q_done = true;
-                }
                 if (kt == kt1) break;
                 const bool win = kt < qg.n_wt;
                 // HCA entries (every visible one, in order) are contiguous rows of the rotated
@@ -600,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 const int n_ent = sm.meta[qc & 1].n_ent;
                 int kt0, kt1;
                 split_range(qg.n_wt + (n_ent + kTile - 1) / kTile, n_split, (int)(w % n_split), &kt0, &kt1);
-                ok = mbar_wait(&sm.q_full, qc & 1u, kWaitIter);
+                ok = mbar_wait(&sm.q_tma, qc & 1u, kWaitIter);
                 if (!ok) break;
                 tc_fence_after();
                 for (int kt = kt0; ok && kt < kt1; ++kt, ++g) {
@@ -955,10 +948,12 @@ static size_t split_part_bytes(const AttendArgs &a, int n_split) {
     return (size_t)a.B * a.S_q * n_split * (size_t)(kH * kD + 2 * kH) * sizeof(float);
 }
 
-size_t attend_tc_workspace(const AttendArgs &a) {
+// Workspace: the keys part (packed keys, key counts, entry lists and split partials for
+// decode-sized calls; rotated window rows and entries for prefill), then the rotated last
+// 64-column chunk of every query row [B*S_q*H, 64].
+static size_t keys_ws_bytes(const AttendArgs &a) {
     if (attend_tc_packed(a)) {
         const size_t rows = (size_t)a.B * a.S_q * attend_tc_kmax(a);
-        // packed keys, key counts, entry lists, then the split partials
         return ((rows * kD * 2 + 255) & ~(size_t)255) + (((size_t)a.B * a.S_q * 4 + 255) & ~(size_t)255) +
                ((rows * 4 + 255) & ~(size_t)255) + split_part_bytes(a, attend_tc_split(a));
     }
@@ -966,6 +961,10 @@ size_t attend_tc_workspace(const AttendArgs &a) {
     size_t pl = ((size_t)a.B * a.P * a.D * 2 + 255) & ~(size_t)255;
     return kv + pl;
 }
+
+static size_t q7_ws_bytes(const AttendArgs &a) { return ((size_t)a.B * a.S_q * kH * 64 * 2 + 255) & ~(size_t)255; }
+
+size_t attend_tc_workspace(const AttendArgs &a) { return keys_ws_bytes(a) + q7_ws_bytes(a); }
 
 csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st) {
     char *ws = reinterpret_cast<char *>(a.workspace);
@@ -1007,8 +1006,17 @@ csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st) {
             CSA_CHECK_LAUNCH("attend: rotate entries");
         }
     }
-    CUtensorMap map_q, map_kv, map_pool;
-    CSA_REQUIRE(encode_map_bf16_2d(&map_q, a.q, kD, (uint64_t)(a.B * a.S_q * kH), 64u, 64u) &&
+    // Q's last chunk, rotated once per call
+    __nv_bfloat16 *q7 = reinterpret_cast<__nv_bfloat16 *>(ws + keys_ws_bytes(a));
+    const int64_t q_rows = a.B * a.S_q * kH;
+    if (q_rows > 0) {
+        rope_q_chunk_kernel<<<(unsigned)ceil_div(q_rows * 8, 256), 256, 0, st>>>((const __nv_bfloat16 *)a.q, q7, q_rows,
+                                                                             a.S_q, a.q_pos0, a.rope);
+        CSA_CHECK_LAUNCH("attend: rotate query rows");
+    }
+    CUtensorMap map_q, map_q7, map_kv, map_pool;
+    CSA_REQUIRE(encode_map_bf16_2d(&map_q, a.q, kD, (uint64_t)q_rows, 64u, 64u) &&
+                    encode_map_bf16_2d(&map_q7, q7, 64u, (uint64_t)q_rows, 64u, 64u) &&
                     encode_map_bf16_2d(&map_kv, kv_rot, kD, kv_rows, 64u, (uint32_t)kTile),
                 CSA_ERR_CUDA, "attend: cannot encode the TMA tensor maps");
     // the rotated pool as TMA rows (HCA entry tiles); other calls never use it
@@ -1033,7 +1041,7 @@ csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st) {
     const int64_t nw = nq * n_split;
     const int grid = (int)(nw < sms ? nw : sms);
     attend_tc_kernel<<<grid, kThreads, smem, st>>>(
-        map_q, map_kv, map_pool, pool_rot, a.S_kv, a.kv_pos0, a.P, a.idx, a.mode == 0 && !packed ? a.topk : 0, a.mode,
+        map_q, map_q7, map_kv, map_pool, pool_rot, a.S_kv, a.kv_pos0, a.P, a.idx, a.mode == 0 && !packed ? a.topk : 0, a.mode,
         a.sink, (__nv_bfloat16 *)a.out, a.B, a.S_q, a.q_pos0, a.window, a.ratio, a.scale, a.rope, n_keys, kmax,
         n_split, part);
     CSA_CHECK_LAUNCH(a.mode == 0 ? "csa_attend" : "hca_attend");
@@ -1064,9 +1072,9 @@ csa_status_t attend_tc_noalloc(AttendArgs &a, cudaStream_t st) {
                 "handled (S_q * 64 >= S_kv + P)");
     const size_t need = attend_tc_workspace(a);
     CSA_REQUIRE(need <= kNoAllocScratchBytes, CSA_ERR_UNSUPPORTED,
-                "csa_attend_noalloc: needs %zu B of scratch for B*(S_kv+P) rotated rows, the "
-                "fixed scratch holds %zu B (at most %zu rows of 512 bf16)",
-                need, kNoAllocScratchBytes, kNoAllocScratchBytes / 1024);
+                "csa_attend_noalloc: needs %zu B of scratch (B*(S_kv+P) rotated rows of 1 KB and "
+                "B*S_q*64 rotated query chunks of 128 B), the fixed scratch holds %zu B",
+                need, kNoAllocScratchBytes);
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     CSA_REQUIRE(e == cudaSuccess && dev >= 0 && dev < kMaxDevices, CSA_ERR_CUDA,
