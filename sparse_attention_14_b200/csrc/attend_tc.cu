@@ -399,6 +399,33 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             const int64_t qn = (w + gridDim.x) / n_split;   // query of the next work item
             const QueryGeom qg = query_geom(qi, S_q, q_pos0, kv_pos0, S_kv, window, packed_n);
             const int64_t nv = n_visible(qg.t, ratio, P);
+            // Q of this query (its rope channels already rotated by rope_q_chunk_kernel): start
+            // its TMA as soon as the previous query's scores are done, ahead of the entry
+            // compaction; the MMA issuer waits for it
+            if (li == 0 && qc > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(&sm.q_free, (qc - 1) & 1u, kWaitIter))) {
+                atomicOr(&g_attend_tc_status, 1u);
+                sm.abort_ = 1;
+                break;
+            }
+            if (li == 0) q_pending = (int)qc;
+            if (li == 0 && lane == 0) {
+                mbar_expect_tx(&sm.q_tma, kQBytes);
+                for (int c = 0; c < 7; ++c)
+                    tma_load_2d(s_q + (uint32_t)c * 8192u, &map_q, 64 * c, (int)(qi * kH), &sm.q_tma);
+                tma_load_2d(s_q + 7u * 8192u, &map_q7, 0, (int)(qi * kH), &sm.q_tma);
+                // bring the next query's Q into L2 while this query runs
+                if (w + gridDim.x < nw) {
+                    for (int c = 0; c < 7; ++c)
+                        asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
+                                         reinterpret_cast<uint64_t>(&map_q)),
+                                     "r"(64 * c), "r"((int)(qn * kH))
+                                     : "memory");
+                    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
+                                     reinterpret_cast<uint64_t>(&map_q7)),
+                                 "r"(0), "r"((int)(qn * kH))
+                                 : "memory");
+                }
+            }
             int n_ent;
             if (packed_n) {
                 n_ent = 0;
@@ -435,32 +462,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             if (li == 0 && lane == 0) {
                 sm.meta[qc & 1].n_ent = n_ent;
                 mbar_arrive(&sm.meta_full[qc & 1]);
-            }
-            // Q of this query (its rope channels already rotated by rope_q_chunk_kernel): start
-            // its TMA once the previous query's scores are done; the MMA issuer waits for it
-            if (li == 0 && qc > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(&sm.q_free, (qc - 1) & 1u, kWaitIter))) {
-                atomicOr(&g_attend_tc_status, 1u);
-                sm.abort_ = 1;
-                break;
-            }
-            if (li == 0) q_pending = (int)qc;
-            if (li == 0 && lane == 0) {
-                mbar_expect_tx(&sm.q_tma, kQBytes);
-                for (int c = 0; c < 7; ++c)
-                    tma_load_2d(s_q + (uint32_t)c * 8192u, &map_q, 64 * c, (int)(qi * kH), &sm.q_tma);
-                tma_load_2d(s_q + 7u * 8192u, &map_q7, 0, (int)(qi * kH), &sm.q_tma);
-                // bring the next query's Q into L2 while this query runs
-                if (w + gridDim.x < nw) {
-                    for (int c = 0; c < 7; ++c)
-                        asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
-                                         reinterpret_cast<uint64_t>(&map_q)),
-                                     "r"(64 * c), "r"((int)(qn * kH))
-                                     : "memory");
-                    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
-                                     reinterpret_cast<uint64_t>(&map_q7)),
-                                 "r"(0), "r"((int)(qn * kH))
-                                 : "memory");
-                }
             }
             int kt0, kt1;
             split_range(qg.n_wt + (n_ent + kTile - 1) / kTile, n_split, (int)(w % n_split), &kt0, &kt1);
