@@ -56,7 +56,9 @@ struct Misc {
 template <int QB>
 struct Cfg {
     static constexpr int N = QB * 64;
-    static constexpr int NE = 8;                         // epilogue warps (two per TMEM lane group)
+    // epilogue warps: QB=4 two per TMEM lane group (each thread 2 queries x 64 heads);
+    // QB=1 one per lane group (each thread all 64 heads of its entry row)
+    static constexpr int NE = QB == 4 ? 8 : 4;
     static constexpr int kThreads = (2 + NE) * 32;
     static constexpr int NST = 2;                        // entry-tile stages
     static constexpr int kMinBlocks = QB == 4 ? 1 : 2;
@@ -65,7 +67,7 @@ struct Cfg {
     static constexpr uint32_t kABytes = kTileE * kDI * 2;
     static constexpr int GS = NE * 32 / QB;              // threads per query group
     static constexpr int QPT = QB == 4 ? 2 : 1;          // queries per epilogue thread
-    static constexpr int CPT = QB == 4 ? 64 : 32;        // head columns per query per thread
+    static constexpr int CPT = 64;                       // head columns per query per thread
     static constexpr uint32_t kTmemCols = 2 * N <= 128 ? 128 : (2 * N <= 256 ? 256 : 512);
     static constexpr uint32_t kOffB = 0;
     static constexpr uint32_t kOffA = kBBytes;
@@ -425,7 +427,7 @@ __global__ void __launch_bounds__(Cfg<QB>::kThreads, Cfg<QB>::kMinBlocks) index_
         const int g4 = warp & 3;                     // TMEM lane group of this warp
         const int row = g4 * 32 + lane;              // entry row inside the tile
         const int qa = QB == 4 ? 2 * (e >> 2) : 0;   // first query of this thread
-        const int cb = QB == 4 ? 0 : 32 * (e >> 2);  // first head column (QB=1: half of 64)
+        const int cb = 0;                            // first head column
         const int et = e * 32 + lane;                // epilogue thread id
         const int grp = et / C::GS, gt = et % C::GS;
         int64_t nvq[QB];
@@ -465,8 +467,8 @@ __global__ void __launch_bounds__(Cfg<QB>::kThreads, Cfg<QB>::kMinBlocks) index_
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&ms.tempty[acc]);
-            if (QB == 1) {
-                // QB=1: warps e and e+4 hold the two halves of the head sum of the same rows
+            if (QB == 1 && C::NE == 8) {
+                // warps e and e+4 hold the two halves of the head sum of the same rows
                 float *part = reinterpret_cast<float *>(hist_all);   // 128 floats, free here
                 if (e >= 4) part[row] = sc[0];
                 named_sync(1, C::NE * 32);
