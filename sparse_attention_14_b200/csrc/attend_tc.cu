@@ -121,28 +121,44 @@ __global__ void rope_rows_kernel(const __nv_bfloat16 *__restrict__ src, __nv_bfl
 // The last 64 channels of every query row (query, head), rotated at the query's position,
 // into a [rows, 64] buffer: the attention loads Q's last 64-column chunk from there, so
 // no rotation of Q sits between a query's Q load and its first MMAs.  Only channels at
-// or after rope.first (>= 448 on this path) are turned; the others are copied.
-__global__ void rope_q_chunk_kernel(const __nv_bfloat16 *__restrict__ q, __nv_bfloat16 *__restrict__ q7,
-                                    int64_t rows, int64_t S_q, int64_t q_pos0, RopeTable rope) {
-    const int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t r = v >> 3;
-    if (r >= rows) return;
-    const int pc = (int)(v & 7);
-    float x[8];
-    load8(q + r * kD + 7 * 64 + pc * 8, x);
-    const double pos = (double)(q_pos0 + (r / kH) % S_q);
-#pragma unroll
-    for (int c = 0; c < 8; c += 2) {
-        const int d = 7 * 64 + pc * 8 + c;
-        if (d >= rope.first) {
-            float cs, sn;
-            rope_cs(pos, rope.inv_freq[(d - rope.first) >> 1], &cs, &sn);
-            const float a = x[c], bb = x[c + 1];
-            x[c] = a * cs - bb * sn;
-            x[c + 1] = a * sn + bb * cs;
-        }
+// or after rope.first (>= 448 on this path) are turned; the others are copied.  One
+// block per query: its rotation angles are computed once and shared by the 64 heads.
+constexpr int kRopeQThreads = 128;
+__global__ void __launch_bounds__(kRopeQThreads) rope_q_chunk_kernel(const __nv_bfloat16 *__restrict__ q,
+                                                                     __nv_bfloat16 *__restrict__ q7, int64_t S_q,
+                                                                     int64_t q_pos0, RopeTable rope) {
+    __shared__ float cs_s[32], sn_s[32];
+    const int64_t qi = blockIdx.x;   // query row (b * S_q + i)
+    const int tid = threadIdx.x;
+    if (tid < rope.n_pairs) {
+        float cs, sn;
+        rope_cs((double)(q_pos0 + qi % S_q), rope.inv_freq[tid], &cs, &sn);
+        cs_s[tid] = cs;
+        sn_s[tid] = sn;
     }
-    store8(q7 + r * 64 + pc * 8, x);
+    __syncthreads();
+    // 64 heads x 8 pieces of 8 channels; four pieces per thread, loaded together
+    float x[4][8];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int v = tid + u * kRopeQThreads, h = v >> 3, pc = v & 7;
+        load8(q + ((qi * kH + h) * kD) + 7 * 64 + pc * 8, x[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int v = tid + u * kRopeQThreads, h = v >> 3, pc = v & 7;
+#pragma unroll
+        for (int c = 0; c < 8; c += 2) {
+            const int d = 7 * 64 + pc * 8 + c;
+            if (d >= rope.first) {
+                const int pr = (d - rope.first) >> 1;
+                const float a = x[u][c], bb = x[u][c + 1];
+                x[u][c] = a * cs_s[pr] - bb * sn_s[pr];
+                x[u][c + 1] = a * sn_s[pr] + bb * cs_s[pr];
+            }
+        }
+        store8(q7 + (qi * kH + h) * 64 + pc * 8, x[u]);
+    }
 }
 
 // Decode-sized calls: gather each query's keys (window rows, then its valid entries in
@@ -1011,8 +1027,8 @@ csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st) {
     __nv_bfloat16 *q7 = reinterpret_cast<__nv_bfloat16 *>(ws + keys_ws_bytes(a));
     const int64_t q_rows = a.B * a.S_q * kH;
     if (q_rows > 0) {
-        rope_q_chunk_kernel<<<(unsigned)ceil_div(q_rows * 8, 256), 256, 0, st>>>((const __nv_bfloat16 *)a.q, q7, q_rows,
-                                                                             a.S_q, a.q_pos0, a.rope);
+        rope_q_chunk_kernel<<<(unsigned)(a.B * a.S_q), kRopeQThreads, 0, st>>>((const __nv_bfloat16 *)a.q, q7, a.S_q,
+                                                                            a.q_pos0, a.rope);
         CSA_CHECK_LAUNCH("attend: rotate query rows");
     }
     CUtensorMap map_q, map_q7, map_kv, map_pool;
