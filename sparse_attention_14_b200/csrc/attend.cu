@@ -36,8 +36,11 @@ __global__ void __launch_bounds__(kThreads) attend_simt_kernel(
     float *p_s = kt + (size_t)D * (kKT + 1);                  // [kHG][kKT]
     int32_t *ent_s = reinterpret_cast<int32_t *>(p_s + kHG * kKT);  // [topk] (CSA)
     __shared__ int64_t key_off[kKT];
-    __shared__ double key_pos[kKT];
+    __shared__ int64_t key_pos[kKT];
     __shared__ int n_ent_s;
+    __shared__ uint64_t turn_s[kMaxRopePairs];
+    stage_turns(rope, turn_s, threadIdx.x, kThreads);
+    __syncthreads();
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t i = blockIdx.x, b = blockIdx.y;
@@ -84,7 +87,7 @@ __global__ void __launch_bounds__(kThreads) attend_simt_kernel(
                 int d = g * 8 + c;
                 if (d >= rope.first) {
                     float cs, sn;
-                    rope_cs((double)t, rope.inv_freq[(d - rope.first) >> 1], &cs, &sn);
+                    rope_cs(t, turn_s[(d - rope.first) >> 1], &cs, &sn);
                     float a = x[c], bb = x[c + 1];
                     x[c] = a * cs - bb * sn;
                     x[c + 1] = a * sn + bb * cs;
@@ -114,11 +117,11 @@ __global__ void __launch_bounds__(kThreads) attend_simt_kernel(
             int x = x0 + tid;
             if (x < n_win) {
                 key_off[tid] = (b * S_kv + (lo_w - kv_pos0) + x) * D;   // into kv
-                key_pos[tid] = (double)(lo_w + x);
+                key_pos[tid] = lo_w + x;
             } else {
                 int64_t j = (mode == 0) ? (int64_t)ent_s[x - n_win] : (int64_t)(x - n_win);
                 key_off[tid] = -1 - (b * P + j) * D;                    // into pool (encoded)
-                key_pos[tid] = (double)j * (double)ratio;
+                key_pos[tid] = (int64_t)j * ratio;
             }
         }
         __syncthreads();
@@ -133,7 +136,7 @@ __global__ void __launch_bounds__(kThreads) attend_simt_kernel(
                 int d = g * 8 + c;
                 if (d >= rope.first) {
                     float cs, sn;
-                    rope_cs(key_pos[xl], rope.inv_freq[(d - rope.first) >> 1], &cs, &sn);
+                    rope_cs(key_pos[xl], turn_s[(d - rope.first) >> 1], &cs, &sn);
                     float a = x[c], bb = x[c + 1];
                     x[c] = a * cs - bb * sn;
                     x[c + 1] = a * sn + bb * cs;
@@ -185,7 +188,7 @@ __global__ void __launch_bounds__(kThreads) attend_simt_kernel(
         float partner = __shfl_xor_sync(0xFFFFFFFFu, o, 1);
         if (d < D && d >= rope.first) {
             float cs, sn;
-            rope_cs(-(double)t, rope.inv_freq[(d - rope.first) >> 1], &cs, &sn);
+            rope_cs(-t, turn_s[(d - rope.first) >> 1], &cs, &sn);
             o = (d & 1) == 0 ? o * cs - partner * sn : partner * sn + o * cs;
         }
         if (d < D) out[(row * H + h) * D + d] = Elem<T>::from_f(o);

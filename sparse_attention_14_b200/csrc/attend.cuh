@@ -41,8 +41,8 @@ size_t attend_workspace(const AttendArgs &a);
 
 // Tensor-core path (bf16, H = 64, D = 512): eligibility, workspace, launch.
 bool attend_tc_eligible(const AttendArgs &a);
-bool attend_tc_packed(const AttendArgs &a);
-int attend_tc_kmax(const AttendArgs &a);
+bool attend_tc_decode(const AttendArgs &a);
+int attend_tc_kmax7(const AttendArgs &a);
 size_t attend_tc_workspace(const AttendArgs &a);
 csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st);
 unsigned int read_attend_tc_status();

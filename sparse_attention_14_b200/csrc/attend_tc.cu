@@ -31,8 +31,11 @@
 //  * epilogue: O^T / l and the -t de-rotation of the rope channels (partner channel via a
 //    lane shuffle), stored as bf16 pairs straight from registers while the next query's
 //    first tile loads and multiplies;
-//  * decode-sized calls (few queries over a long cache) pack each query's rotated keys
-//    first; with few queries, each query's key tiles are split over two CTAs that write
+//  * decode-sized calls (few queries over a long cache) read the key rows in place: chunks
+//    0-6 of window rows by TMA from the raw rows, of entries by 16-byte copies from the
+//    pool, and chunk 7 (the rope channels) by TMA from a small buffer that
+//    pack_k7_kernel fills with the rotated last chunk of just the keys each query uses;
+//    with few queries, each query's key tiles are split over two CTAs that write
 //    unnormalised partials, merged (sink, division, de-rotation) by attend_combine_kernel.
 #include <mutex>
 
@@ -89,8 +92,11 @@ __host__ __device__ __forceinline__ size_t tc_ent_bytes(int topk) {
 
 size_t tc_smem_bytes(int topk) { return 1024 + kOffEnt + kLoaders * tc_ent_bytes(topk) + sizeof(Small); }
 
-__global__ void rope_rows_kernel(const __nv_bfloat16 *__restrict__ src, __nv_bfloat16 *__restrict__ dst,
-                                 int64_t rows, int64_t pos0, int64_t pos_step, int D, RopeTable rope) {
+__global__ void __launch_bounds__(256) rope_rows_kernel(const __nv_bfloat16 *__restrict__ src,
+                                                        __nv_bfloat16 *__restrict__ dst, int64_t rows, int64_t pos0,
+                                                        int64_t pos_step, int D, RopeTable rope) {
+    // only the 8 lanes of a warp holding rope pieces read the table (a divergent read,
+    // measured cheaper here than staging it in shared memory behind a barrier)
     const int pieces = D / 8;
     int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     int64_t r = v / pieces;
@@ -102,13 +108,13 @@ __global__ void rope_rows_kernel(const __nv_bfloat16 *__restrict__ src, __nv_bfl
     load8(s, x);
     int d0 = pc * 8;
     if (d0 + 8 > rope.first) {
-        double pos = (double)(pos0 + r * pos_step);
+        const int64_t pos = pos0 + r * pos_step;
 #pragma unroll
         for (int c = 0; c < 8; c += 2) {
             int d = d0 + c;
             if (d >= rope.first) {
                 float cs, sn;
-                rope_cs(pos, rope.inv_freq[(d - rope.first) >> 1], &cs, &sn);
+                rope_cs(pos, rope.turn[(d - rope.first) >> 1], &cs, &sn);
                 float a = x[c], bb = x[c + 1];
                 x[c] = a * cs - bb * sn;
                 x[c + 1] = a * sn + bb * cs;
@@ -124,19 +130,23 @@ __global__ void rope_rows_kernel(const __nv_bfloat16 *__restrict__ src, __nv_bfl
 // or after rope.first (>= 448 on this path) are turned; the others are copied.  One
 // block per query: its rotation angles are computed once and shared by the 64 heads.
 constexpr int kRopeQThreads = 128;
-__global__ void __launch_bounds__(kRopeQThreads) rope_q_chunk_kernel(const __nv_bfloat16 *__restrict__ q,
-                                                                     __nv_bfloat16 *__restrict__ q7, int64_t S_q,
-                                                                     int64_t q_pos0, RopeTable rope) {
-    __shared__ float cs_s[32], sn_s[32];
-    const int64_t qi = blockIdx.x;   // query row (b * S_q + i)
-    const int tid = threadIdx.x;
+
+// The rotation of query row qi's last chunk by the first kRopeQThreads threads of a block
+// (tid): angles once in shared memory, then four 8-channel pieces per thread.
+__device__ __forceinline__ void rotate_q_chunk_part(const __nv_bfloat16 *__restrict__ q,
+                                                    __nv_bfloat16 *__restrict__ q7, int64_t qi, int64_t S_q,
+                                                    int64_t q_pos0, const RopeTable &rope, int tid, float *cs_s,
+                                                    float *sn_s) {
     if (tid < rope.n_pairs) {
+        // one divergent read of the kernel-parameter table per block (measured cheaper here
+        // than a warp-uniform loop over it)
         float cs, sn;
-        rope_cs((double)(q_pos0 + qi % S_q), rope.inv_freq[tid], &cs, &sn);
+        rope_cs(q_pos0 + qi % S_q, rope.turn[tid], &cs, &sn);
         cs_s[tid] = cs;
         sn_s[tid] = sn;
     }
-    __syncthreads();
+    // the kRopeQThreads threads of the caller synchronise among themselves (named barrier 1)
+    asm volatile("bar.sync 1, %0;" ::"n"(kRopeQThreads) : "memory");
     // 64 heads x 8 pieces of 8 channels; four pieces per thread, loaded together
     float x[4][8];
 #pragma unroll
@@ -161,128 +171,146 @@ __global__ void __launch_bounds__(kRopeQThreads) rope_q_chunk_kernel(const __nv_
     }
 }
 
-// Decode-sized calls: gather each query's keys (window rows, then its valid entries in
-// slot order / every visible entry) into a packed buffer [B*S_q][kmax][D], rotated at
-// their positions, and record the key count per query.  Only the rows a query reads are
-// touched, instead of rotating the whole cache.  Two kernels: one warp per query lists
-// the key sources; then (query, 16-row slice) blocks copy and rotate the rows.
-__global__ void __launch_bounds__(32) pack_list_kernel(const int32_t *__restrict__ idx, int topk, int mode,
-                                                       int64_t S_kv, int64_t kv_pos0, int64_t P, int64_t S_q,
-                                                       int64_t q_pos0, int window, int ratio, int kmax,
-                                                       int32_t *__restrict__ ent_ws, int32_t *__restrict__ n_keys) {
+__global__ void __launch_bounds__(kRopeQThreads) rope_q_chunk_kernel(const __nv_bfloat16 *__restrict__ q,
+                                                                     __nv_bfloat16 *__restrict__ q7, int64_t S_q,
+                                                                     int64_t q_pos0, RopeTable rope) {
+    __shared__ float cs_s[32], sn_s[32];
+    rotate_q_chunk_part(q, q7, blockIdx.x, S_q, q_pos0, rope, threadIdx.x, cs_s, sn_s);
+}
+
+// Decode-sized calls (few queries over a long cache): the attention reads the first seven
+// 64-channel chunks of every key straight from the window rows and the pool, and the last
+// chunk (the one holding the rope channels) from a small per-query buffer k7 that this
+// kernel fills, rotated at each key's position.  k7 rows of query qi are tile-major like
+// the attention's key tiles: rows qi*kmax7 + kt*128 + r hold window row kt*128 + r for the
+// n_wt window tiles, then entry (kt - n_wt)*128 + r (the valid idx values in slot order for
+// CSA, every visible entry for HCA); rows past the last key are zero.  Block (qi, kt) fills
+// tile kt of query qi; block (qi, 0) also writes the query's rotated chunk to q7.
+constexpr int kK7Threads = 256;
+__global__ void __launch_bounds__(kK7Threads) pack_k7_kernel(
+    const __nv_bfloat16 *__restrict__ kv, int64_t S_kv, int64_t kv_pos0, const __nv_bfloat16 *__restrict__ pool,
+    int64_t P, const int32_t *__restrict__ idx, int topk, int mode, int64_t S_q, int64_t q_pos0, int window,
+    int ratio, RopeTable rope, int kmax7, __nv_bfloat16 *__restrict__ k7, const __nv_bfloat16 *__restrict__ q,
+    __nv_bfloat16 *__restrict__ q7) {
+    __shared__ float cs_s[32], sn_s[32];
+    __shared__ const __nv_bfloat16 *row_src[kTile];
+    __shared__ int64_t row_pos[kTile];
+    // (cos, sin) per rope pair and row; the row stride of 129 keeps both the writes (lanes =
+    // rows) and the reads (lanes = rows x pairs) free of bank conflicts
+    __shared__ float2 ang[32][kTile + 1];
+    __shared__ int warp_cnt[kK7Threads / 32];
     const int64_t qi = blockIdx.x;
-    const int lane = threadIdx.x;
-    const int64_t t = q_pos0 + qi % S_q;
+    const int kt = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
+    if (kt == 0 && tid < kRopeQThreads) rotate_q_chunk_part(q, q7, qi, S_q, q_pos0, rope, tid, cs_s, sn_s);
+    const int64_t b = qi / S_q, t = q_pos0 + qi % S_q;
     const int64_t nv = n_visible(t, ratio, P);
     int64_t lo = t - window + 1;
     if (lo < kv_pos0) lo = kv_pos0;
     const int64_t hi = t < kv_pos0 + S_kv - 1 ? t : kv_pos0 + S_kv - 1;
     const int n_win = hi >= lo ? (int)(hi - lo + 1) : 0;
-    int n_ent;
-    if (mode == 0) {
-        int cnt = 0;
-        const int32_t *ip = idx + qi * topk;
-        int32_t *ep = ent_ws + qi * (int64_t)kmax;
-        for (int c0 = 0; c0 < topk; c0 += 256) {
-            int32_t jv[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int c = c0 + k * 32 + lane;
-                jv[k] = c < topk ? ip[c] : -1;
-            }
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const bool ok = jv[k] >= 0 && (int64_t)jv[k] < nv;
-                const unsigned ball = __ballot_sync(0xFFFFFFFFu, ok);
-                if (ok) ep[cnt + __popc(ball & ((1u << lane) - 1u))] = jv[k];
-                cnt += __popc(ball);
-            }
+    const int n_wt = (n_win + kTile - 1) / kTile;
+    if (tid < kTile) row_src[tid] = nullptr;
+    __syncthreads();
+    if (kt < n_wt) {
+        if (tid < kTile && kt * kTile + tid < n_win) {
+            const int x = kt * kTile + tid;
+            row_src[tid] = kv + (b * S_kv + (lo - kv_pos0) + x) * kD;
+            row_pos[tid] = lo + x;
         }
-        n_ent = cnt;
     } else {
-        n_ent = (int)nv;
-    }
-    int nk = n_win + n_ent;
-    if (nk > kmax) nk = kmax;
-    if (lane == 0) n_keys[qi] = nk;
-}
-
-constexpr int kPackRows = 64;
-__global__ void __launch_bounds__(256) pack_rows_kernel(
-    const __nv_bfloat16 *__restrict__ kv, int64_t S_kv, int64_t kv_pos0, const __nv_bfloat16 *__restrict__ pool,
-    int64_t P, int mode, int64_t S_q, int64_t q_pos0, int window, int ratio, RopeTable rope,
-    const int32_t *__restrict__ ent_ws, const int32_t *__restrict__ n_keys, __nv_bfloat16 *__restrict__ packed,
-    int kmax) {
-    __shared__ const __nv_bfloat16 *row_src[kPackRows];
-    __shared__ double row_pos[kPackRows];
-    const int64_t qi = blockIdx.x;
-    const int x0 = blockIdx.y * kPackRows;
-    const int nk = n_keys[qi];
-    {
-        // rows [nk, kmax) hold no key but are read (with zero weight) by the last key tile
-        // of the query: zero them so that stale workspace bits cannot turn into NaN
-        const int z0 = nk > x0 ? nk : x0;
-        const int z1 = x0 + kPackRows < kmax ? x0 + kPackRows : kmax;
-        for (int v = threadIdx.x; v < (z1 - z0) * (kD / 8); v += blockDim.x)
-            *reinterpret_cast<uint4 *>(packed + (qi * kmax + z0 + v / (kD / 8)) * kD + (v % (kD / 8)) * 8) =
-                make_uint4(0u, 0u, 0u, 0u);
-    }
-    if (x0 >= nk) return;
-    const int64_t b = qi / S_q, t = q_pos0 + qi % S_q;
-    int64_t lo = t - window + 1;
-    if (lo < kv_pos0) lo = kv_pos0;
-    const int64_t hi = t < kv_pos0 + S_kv - 1 ? t : kv_pos0 + S_kv - 1;
-    const int n_win = hi >= lo ? (int)(hi - lo + 1) : 0;
-    const int rows = nk - x0 < kPackRows ? nk - x0 : kPackRows;
-    // resolve this slice's source rows once
-    if (threadIdx.x < rows) {
-        const int x = x0 + threadIdx.x;
-        if (x < n_win) {
-            row_src[threadIdx.x] = kv + (b * S_kv + (lo - kv_pos0) + x) * kD;
-            row_pos[threadIdx.x] = (double)(lo + x);
-        } else {
-            const int64_t j = mode == 0 ? (int64_t)ent_ws[qi * (int64_t)kmax + (x - n_win)] : (int64_t)(x - n_win);
-            row_src[threadIdx.x] = pool + (b * P + j) * kD;
-            row_pos[threadIdx.x] = (double)j * (double)ratio;
+        const int e0 = (kt - n_wt) * kTile;
+        if (mode == 0) {
+            // rank of every valid idx slot: thread tid owns slots [tid*per, tid*per + per)
+            const int per = (topk + kK7Threads - 1) / kK7Threads;
+            const int32_t *ip = idx + qi * (int64_t)topk;
+            int cnt = 0;
+            for (int u = 0; u < per; ++u) {
+                const int c = tid * per + u;
+                if (c < topk) {
+                    const int32_t j = ip[c];
+                    cnt += (j >= 0 && (int64_t)j < nv) ? 1 : 0;
+                }
+            }
+            int incl = cnt;   // inclusive scan over the warp, then over the warps
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+                if (lane >= off) incl += v;
+            }
+            if (lane == 31) warp_cnt[wp] = incl;
+            __syncthreads();
+            int rank = incl - cnt;
+            for (int k = 0; k < wp; ++k) rank += warp_cnt[k];
+            for (int u = 0; u < per; ++u) {
+                const int c = tid * per + u;
+                if (c < topk) {
+                    const int32_t j = ip[c];
+                    if (j >= 0 && (int64_t)j < nv) {
+                        if (rank >= e0 && rank < e0 + kTile) {
+                            row_src[rank - e0] = pool + (b * P + j) * kD;
+                            row_pos[rank - e0] = (int64_t)j * ratio;
+                        }
+                        ++rank;
+                    }
+                }
+            }
+        } else if (tid < kTile && (int64_t)(e0 + tid) < nv) {
+            const int64_t j = e0 + tid;
+            row_src[tid] = pool + (b * P + j) * kD;
+            row_pos[tid] = j * ratio;
         }
     }
     __syncthreads();
-    constexpr int kPieces = kD / 8;                       // 64 pieces of 16 bytes per row
-    const int rope_p0 = rope.first / 8;                   // first piece holding rope channels
-    // un-rotated pieces: raw 16-byte copies, eight in flight per thread
-    const int plain = rows * rope_p0;
-    for (int v0 = 0; v0 < plain; v0 += 8 * 256) {
-        uint4 w[8];
+    // 128 rows x 8 pieces of 16 bytes (the last 64 channels), four pieces per thread, all
+    // loads in flight together; the angles are computed meanwhile
+    const int pc = tid & 7, r0 = tid >> 3;
+    uint4 w[kTile * 8 / kK7Threads];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int v = v0 + u * 256 + threadIdx.x;
-            if (v < plain) w[u] = *reinterpret_cast<const uint4 *>(row_src[v / rope_p0] + (v % rope_p0) * 8);
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int v = v0 + u * 256 + threadIdx.x;
-            if (v < plain)
-                *reinterpret_cast<uint4 *>(packed + (qi * kmax + x0 + v / rope_p0) * kD + (v % rope_p0) * 8) = w[u];
+    for (int u = 0; u < kTile * 8 / kK7Threads; ++u) {
+        const int xr = r0 + u * (kK7Threads / 8);
+        w[u] = row_src[xr] ? *reinterpret_cast<const uint4 *>(row_src[xr] + 7 * 64 + pc * 8)
+                           : make_uint4(0u, 0u, 0u, 0u);
+    }
+    {
+        // thread: row tid % 128, pairs of its half (tid / 128) of the table -- the pair index
+        // is the same across a warp, so the table reads are broadcasts
+        const int xr = tid % kTile, half = tid / kTile;
+        const int per = (rope.n_pairs + 1) / 2;
+        if (row_src[xr]) {
+            const int64_t pos = row_pos[xr];
+            for (int pr = half * per; pr < (half + 1) * per && pr < rope.n_pairs; ++pr)
+                rope_cs(pos, rope.turn[pr], &ang[pr][xr].x, &ang[pr][xr].y);
         }
     }
-    // rope pieces: every lane rotates whole pieces (no divergence around the angle math)
-    const int rp = kPieces - rope_p0;
-    for (int v = threadIdx.x; v < rows * rp; v += 256) {
-        const int xr = v / rp, pc = rope_p0 + v % rp;
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < kTile * 8 / kK7Threads; ++u) {
+        const int xr = r0 + u * (kK7Threads / 8);
+        __nv_bfloat16 *dst = k7 + (qi * kmax7 + (int64_t)kt * kTile + xr) * 64 + pc * 8;
+        if (!row_src[xr] || 7 * 64 + pc * 8 + 8 <= rope.first) {
+            *reinterpret_cast<uint4 *>(dst) = w[u];
+            continue;
+        }
         float e[8];
-        load8(row_src[xr] + pc * 8, e);
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&w[u]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const float2 f = __bfloat1622float2(h[c]);
+            e[2 * c] = f.x;
+            e[2 * c + 1] = f.y;
+        }
 #pragma unroll
         for (int c = 0; c < 8; c += 2) {
-            const int d = pc * 8 + c;
+            const int d = 7 * 64 + pc * 8 + c;
             if (d >= rope.first) {
-                float cs, sn;
-                rope_cs(row_pos[xr], rope.inv_freq[(d - rope.first) >> 1], &cs, &sn);
+                const float2 cs = ang[(d - rope.first) >> 1][xr];
                 const float a0 = e[c], a1 = e[c + 1];
-                e[c] = a0 * cs - a1 * sn;
-                e[c + 1] = a0 * sn + a1 * cs;
+                e[c] = a0 * cs.x - a1 * cs.y;
+                e[c + 1] = a0 * cs.y + a1 * cs.x;
             }
         }
-        store8(packed + (qi * kmax + x0 + xr) * kD + pc * 8, e);
+        store8(dst, e);
     }
 }
 
@@ -333,20 +361,12 @@ struct QueryGeom {
     int n_win, n_wt;
 };
 
-// packed != nullptr: the keys of query qi are the n_keys[qi] rows qi*kmax... of a packed,
-// already rotated buffer (decode-sized calls), all loaded like window rows.
 __device__ __forceinline__ QueryGeom query_geom(int64_t qi, int64_t S_q, int64_t q_pos0, int64_t kv_pos0,
-                                                int64_t S_kv, int window, const int32_t *packed_n) {
+                                                int64_t S_kv, int window) {
     QueryGeom g;
     g.b = qi / S_q;
     g.i = qi % S_q;
     g.t = q_pos0 + g.i;
-    if (packed_n) {
-        g.lo_w = 0;
-        g.n_win = packed_n[qi];
-        g.n_wt = (g.n_win + kTile - 1) / kTile;
-        return g;
-    }
     int64_t lo = g.t - window + 1;
     if (lo < kv_pos0) lo = kv_pos0;
     int64_t hi = g.t < kv_pos0 + S_kv - 1 ? g.t : kv_pos0 + S_kv - 1;
@@ -356,14 +376,17 @@ __device__ __forceinline__ QueryGeom query_geom(int64_t qi, int64_t S_q, int64_t
     return g;
 }
 
+// kK7: decode-sized calls (chunk 7 of every key from k7, rows qi*kmax7 + kt*128, the key
+// rows read in place); prefill otherwise.
+template <bool kK7>
 __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_q7,
     const __grid_constant__ CUtensorMap map_kv, const __grid_constant__ CUtensorMap map_pool,
-    const __nv_bfloat16 *__restrict__ pool_rot, int64_t S_kv,
+    const __grid_constant__ CUtensorMap map_k7, const __nv_bfloat16 *__restrict__ pool_rot, int64_t S_kv,
     int64_t kv_pos0, int64_t P,
     const int32_t *__restrict__ idx, int topk, int mode, const float *__restrict__ sink,
     __nv_bfloat16 *__restrict__ out, int64_t B, int64_t S_q, int64_t q_pos0, int window, int ratio,
-    float scale, RopeTable rope, const int32_t *__restrict__ packed_n, int kmax, int n_split,
+    float scale, RopeTable rope, int kmax7, int n_split,
     float *__restrict__ part) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
@@ -413,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         for (int64_t w = blockIdx.x; w < nw && !sm.abort_ && !withhold; w += gridDim.x, ++qc) {
             const int64_t qi = w / n_split;
             const int64_t qn = (w + gridDim.x) / n_split;   // query of the next work item
-            const QueryGeom qg = query_geom(qi, S_q, q_pos0, kv_pos0, S_kv, window, packed_n);
+            const QueryGeom qg = query_geom(qi, S_q, q_pos0, kv_pos0, S_kv, window);
             const int64_t nv = n_visible(qg.t, ratio, P);
             // Q of this query (its rope channels already rotated by rope_q_chunk_kernel): start
             // its TMA as soon as the previous query's scores are done, ahead of the entry
@@ -443,9 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 }
             }
             int n_ent;
-            if (packed_n) {
-                n_ent = 0;
-            } else if (mode == 0) {
+            if (mode == 0) {
                 // compact the valid idx values in slot order; eight loads per lane in flight
                 int cnt = 0;
                 const int32_t *ip = idx + qi * topk;
@@ -487,19 +508,24 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 const bool win = kt < qg.n_wt;
                 // HCA entries (every visible one, in order) are contiguous rows of the rotated
                 // pool, like window rows: both come as 2-D TMA boxes of 128 rows per chunk
-                const bool hca_ent = !win && mode == 1 && !packed_n;
+                const bool hca_ent = !win && mode == 1;
+                // decode-sized calls: the last chunk of every key comes rotated from k7, rows
+                // qi*kmax7 + kt*128 ...
                 if (win || hca_ent) {
                     const CUtensorMap *map = win ? &map_kv : &map_pool;
                     const int y0 = hca_ent ? (int)(qg.b * P + (int64_t)(kt - qg.n_wt) * kTile)
-                                   : packed_n ? (int)(qi * kmax + (int64_t)kt * kTile)
-                                              : (int)(qg.b * S_kv + (qg.lo_w - kv_pos0) + (int64_t)kt * kTile);
+                                           : (int)(qg.b * S_kv + (qg.lo_w - kv_pos0) + (int64_t)kt * kTile);
                     for (int c = 0; c < 8 && ok; ++c) {
                         if (((c >> 1) & 1) != li) continue;
                         if ((c & 1) == 0 && g > 0)
                             ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.free_[c >> 1], (g - 1) & 1u, kWaitIter));
                         if (ok && lane == 0) {
                             mbar_expect_tx(&sm.full[c], 16384u);
-                            tma_load_2d(s_kv + (uint32_t)c * 16384u, map, 64 * c, y0, &sm.full[c]);
+                            if (kK7 && c == 7)
+                                tma_load_2d(s_kv + 7u * 16384u, &map_k7, 0, (int)(qi * kmax7 + (int64_t)kt * kTile),
+                                            &sm.full[7]);
+                            else
+                                tma_load_2d(s_kv + (uint32_t)c * 16384u, map, 64 * c, y0, &sm.full[c]);
                             sm.last_tma[c] = (int)g;
                         }
                     }
@@ -512,7 +538,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                     const int et = kt - qg.n_wt;
                     const int pc = lane & 7;
                     const __nv_bfloat16 *src[32];
-                    uint32_t dsto[32];
 #pragma unroll
                     for (int k = 0; k < 32; ++k) {
                         const int xr = 4 * k + (lane >> 3);
@@ -520,20 +545,24 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                         const int rr = r < n_ent ? r : 0;
                         const int64_t j = mode == 0 ? (int64_t)ent[rr] : (int64_t)rr;
                         src[k] = pool_rot + (qg.b * P + j) * kD + pc * 8;
-                        dsto[k] = sw128((uint32_t)xr, (uint32_t)pc);
                     }
+                    // swizzled destination of row 4k + (lane >> 3): k * 512 plus one of two
+                    // lane constants (the row's low three bits alternate with k's parity)
+                    const uint32_t r8 = (uint32_t)(lane >> 3);
+                    const uint32_t dst_even = sw128(r8, (uint32_t)pc), dst_odd = sw128(4u + r8, (uint32_t)pc) - 512u;
                     // this loader's two pairs: both chunks of a pair in flight, published
                     // (own copies complete, proxy fence, warp sync, one arrive per chunk) as
                     // soon as the next pair would have to wait for its slots, else after the
                     // next pair is issued
                     int pend = -1;   // first chunk of the pair issued but not yet published
+                    // with k7 the last chunk is a TMA load whose bytes complete its barrier
                     auto publish_pair = [&](int c0) {
                         asm volatile("cp.async.wait_group 0;" ::: "memory");
                         fence_async_smem();
                         __syncwarp();
                         if (lane == 0) {
                             mbar_arrive(&sm.full[c0]);
-                            mbar_arrive(&sm.full[c0 + 1]);
+                            if (!(kK7 && c0 == 6)) mbar_arrive(&sm.full[c0 + 1]);
                         }
                     };
                     for (int p = li; p < 4 && ok; p += kLoaders) {
@@ -553,9 +582,18 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                         for (int h = 0; h < 2; ++h) {
                             const int c = 2 * p + h;
                             const uint32_t dst = s_kv + (uint32_t)c * 16384u;
+                            if (kK7 && c == 7) {
+                                if (lane == 0) {
+                                    mbar_expect_tx(&sm.full[7], 16384u);
+                                    tma_load_2d(dst, &map_k7, 0, (int)(qi * kmax7 + (int64_t)kt * kTile), &sm.full[7]);
+                                    sm.last_tma[7] = (int)g;
+                                }
+                                continue;
+                            }
                             if (lane == 0) sm.last_tma[c] = -1;
 #pragma unroll
-                            for (int k = 0; k < 32; ++k) cp_async16(dst + dsto[k], src[k] + c * 64, 16u);
+                            for (int k = 0; k < 32; ++k)
+                                cp_async16(dst + (uint32_t)k * 512u + ((k & 1) ? dst_odd : dst_even), src[k] + c * 64, 16u);
                         }
                         cp_async_commit();
                         if (pend >= 0) {
@@ -565,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                             __syncwarp();
                             if (lane == 0) {
                                 mbar_arrive(&sm.full[pend]);
-                                mbar_arrive(&sm.full[pend + 1]);
+                                if (!(kK7 && pend == 6)) mbar_arrive(&sm.full[pend + 1]);
                             }
                         }
                         pend = 2 * p;
@@ -604,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             uint32_t g = 0, qc = 0;
             bool ok = true;
             for (int64_t w = blockIdx.x; ok && w < nw; w += gridDim.x, ++qc) {
-                const QueryGeom qg = query_geom(w / n_split, S_q, q_pos0, kv_pos0, S_kv, window, packed_n);
+                const QueryGeom qg = query_geom(w / n_split, S_q, q_pos0, kv_pos0, S_kv, window);
                 ok = mbar_wait(&sm.meta_full[qc & 1], (qc >> 1) & 1u, kWaitIter);
                 if (!ok) break;
                 const int n_ent = sm.meta[qc & 1].n_ent;
@@ -667,7 +705,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         bool ok = true;
         for (int64_t w = blockIdx.x; ok && w < nw; w += gridDim.x, ++qc) {
             const int64_t qi = w / n_split;
-            const QueryGeom qg = query_geom(qi, S_q, q_pos0, kv_pos0, S_kv, window, packed_n);
+            const QueryGeom qg = query_geom(qi, S_q, q_pos0, kv_pos0, S_kv, window);
             // every exit after a wait that ran out is decided together (vote at the named
             // barrier), so no thread is left waiting for the others at a later barrier
             ok = !named_sync_any(1, kSoftThreads, !mbar_wait(&sm.meta_full[qc & 1], (qc >> 1) & 1u, kWaitIter));
@@ -812,7 +850,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 const int d = mt * 128 + x;
                 float cs = 1.f, sn = 0.f;
                 const bool rot = d >= rope.first;
-                if (rot) rope_cs(-(double)qg.t, rope.inv_freq[(d - rope.first) >> 1], &cs, &sn);
+                // (a divergent read of the kernel-parameter table, once per query and thread:
+                // measured faster here than a shared-memory copy)
+                if (rot) rope_cs(-qg.t, rope.turn[(d - rope.first) >> 1], &cs, &sn);
                 float o[32];
                 if (kt1 > kt0) {
                     tmem_ld32(trow + kColO + mt * 64 + hb, o);
@@ -885,11 +925,20 @@ __global__ void __launch_bounds__(256) attend_combine_kernel(const float *__rest
         if (sk != -INFINITY && M != -INFINITY) l += exp2f(sk * kLog2e - M);
         inv_l[tid] = l > 0.f ? 1.f / l : 0.f;
     }
-    if (tid >= 32 && tid - 32 < rope.n_pairs) {
-        float cs, sn;
-        rope_cs(-(double)(q_pos0 + qi % S_q), rope.inv_freq[tid - 32], &cs, &sn);
-        rcs[0][tid - 32] = cs;
-        rcs[1][tid - 32] = sn;
+    if (tid >= 32 && tid < 64) {
+        // warp 1, lane p: pair p (n_pairs <= 32 on this path), table read warp-uniformly
+        const int p = tid - 32;
+        uint64_t tv = 0;
+        for (int k = 0; k < rope.n_pairs; ++k) {
+            const uint64_t v = rope.turn[k];
+            if (p == k) tv = v;
+        }
+        if (p < rope.n_pairs) {
+            float cs, sn;
+            rope_cs(-(q_pos0 + qi % S_q), tv, &cs, &sn);
+            rcs[0][p] = cs;
+            rcs[1][p] = sn;
+        }
     }
     // thread: channel pair d = 2 * tid of the 8 heads
     const int d = 2 * tid;
@@ -931,33 +980,40 @@ bool attend_tc_eligible(const AttendArgs &a) {
     if (a.rope_dim > 64) return false;               // rope channels inside the last chunk
     if (a.mode == 0 && a.topk > 2048) return false;
     // both loaders' entry lists must fit next to the key tile, Q and P in shared memory
-    if (tc_smem_bytes(a.mode == 0 && !attend_tc_packed(a) ? a.topk : 1) > 232448) return false;
+    if (tc_smem_bytes(a.mode == 0 ? a.topk : 1) > 232448) return false;
     // TMA row coordinates are 32-bit
     if (a.B * a.S_q * kH >= (1ll << 31) || a.B * a.S_kv + kTile >= (1ll << 31) ||
         a.B * a.P >= (1ll << 31))
         return false;
-    if (attend_tc_packed(a) && a.B * a.S_q * (int64_t)attend_tc_kmax(a) + kTile >= (1ll << 31)) return false;
+    if (attend_tc_decode(a)) {
+        if (a.B * a.S_q * (int64_t)attend_tc_kmax7(a) + kTile >= (1ll << 31)) return false;
+        // the key rows are read in place (TMA boxes and 16-byte copies): 16-byte aligned
+        if (((uintptr_t)a.kv | (uintptr_t)a.pool) & 15u) return false;
+    }
     return true;
 }
 
 // Prefill (the queries outnumber the key rows): every window row and entry is rotated once
-// into the workspace and tiles gather from there.  Decode-sized calls (few queries over a
-// long cache) instead pack just the rows each query reads.
-bool attend_tc_packed(const AttendArgs &a) { return (double)a.S_q * 64.0 < (double)(a.S_kv + a.P); }
+// into the workspace and tiles read from there.  Decode-sized calls (few queries over a
+// long cache) read the key rows in place and only the rope chunk of the keys each query
+// uses is rotated (pack_k7_kernel).
+bool attend_tc_decode(const AttendArgs &a) { return (double)a.S_q * 64.0 < (double)(a.S_kv + a.P); }
 
-int attend_tc_kmax(const AttendArgs &a) {
-    // an upper bound that needs no window size (the workspace query does not take one):
-    // every raw row given plus every entry the query can list
+int attend_tc_kmax7(const AttendArgs &a) {
+    // k7 rows per query: an upper bound that needs no window size (the workspace query
+    // does not take one): window tiles for every raw row given, entry tiles for every
+    // entry the query can list
     const int64_t e = a.mode == 0 ? (a.topk < a.P ? a.topk : a.P) : a.P;
-    return (int)(a.S_kv + e > 0 ? a.S_kv + e : 1);
+    const int64_t tiles = (a.S_kv + kTile - 1) / kTile + (e + kTile - 1) / kTile;
+    return (int)(tiles > 0 ? tiles * kTile : kTile);
 }
 
 // Decode-sized calls with few queries split each query's key tiles over two CTAs (the
 // device has 148 SMs) and merge the partials in a second kernel.
 static int attend_tc_split(const AttendArgs &a) {
-    if (!attend_tc_packed(a)) return 1;
+    if (!attend_tc_decode(a)) return 1;
     const int64_t nq = a.B * a.S_q;
-    return (nq * 2 <= 148 && attend_tc_kmax(a) > kTile) ? 2 : 1;
+    return (nq * 2 <= 148 && attend_tc_kmax7(a) > kTile) ? 2 : 1;
 }
 
 static size_t split_part_bytes(const AttendArgs &a, int n_split) {
@@ -965,51 +1021,46 @@ static size_t split_part_bytes(const AttendArgs &a, int n_split) {
     return (size_t)a.B * a.S_q * n_split * (size_t)(kH * kD + 2 * kH) * sizeof(float);
 }
 
-// Workspace: the keys part (packed keys, key counts, entry lists and split partials for
-// decode-sized calls; rotated window rows and entries for prefill), then the rotated last
-// 64-column chunk of every query row [B*S_q*H, 64].
+static size_t round256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+// Workspace: the keys part (decode-sized calls: the rotated rope chunks k7 [B*S_q*kmax7, 64]
+// and the split partials; prefill: the rotated window rows and entries), then the rotated
+// last 64-column chunk of every query row [B*S_q*H, 64].
 static size_t keys_ws_bytes(const AttendArgs &a) {
-    if (attend_tc_packed(a)) {
-        const size_t rows = (size_t)a.B * a.S_q * attend_tc_kmax(a);
-        return ((rows * kD * 2 + 255) & ~(size_t)255) + (((size_t)a.B * a.S_q * 4 + 255) & ~(size_t)255) +
-               ((rows * 4 + 255) & ~(size_t)255) + split_part_bytes(a, attend_tc_split(a));
-    }
-    size_t kv = ((size_t)a.B * a.S_kv * a.D * 2 + 255) & ~(size_t)255;
-    size_t pl = ((size_t)a.B * a.P * a.D * 2 + 255) & ~(size_t)255;
-    return kv + pl;
+    if (attend_tc_decode(a))
+        return round256((size_t)a.B * a.S_q * attend_tc_kmax7(a) * 64 * 2) + split_part_bytes(a, attend_tc_split(a));
+    return round256((size_t)a.B * a.S_kv * a.D * 2) + round256((size_t)a.B * a.P * a.D * 2);
 }
 
-static size_t q7_ws_bytes(const AttendArgs &a) { return ((size_t)a.B * a.S_q * kH * 64 * 2 + 255) & ~(size_t)255; }
+static size_t q7_ws_bytes(const AttendArgs &a) { return round256((size_t)a.B * a.S_q * kH * 64 * 2); }
 
 size_t attend_tc_workspace(const AttendArgs &a) { return keys_ws_bytes(a) + q7_ws_bytes(a); }
 
 csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st) {
     char *ws = reinterpret_cast<char *>(a.workspace);
-    const bool packed = attend_tc_packed(a);
-    const int kmax = packed ? attend_tc_kmax(a) : 0;
-    __nv_bfloat16 *kv_rot = reinterpret_cast<__nv_bfloat16 *>(ws);
-    __nv_bfloat16 *pool_rot = nullptr;
-    int32_t *n_keys = nullptr;
-    uint64_t kv_rows;
+    const bool decode = attend_tc_decode(a);
+    const int kmax7 = decode ? attend_tc_kmax7(a) : 0;
+    const int64_t nq = a.B * a.S_q;
+    const int64_t q_rows = nq * kH;
+    __nv_bfloat16 *q7 = reinterpret_cast<__nv_bfloat16 *>(ws + keys_ws_bytes(a));
+    const __nv_bfloat16 *kv_src, *pool_src;   // key rows the tiles read
+    __nv_bfloat16 *k7 = nullptr;
     const int pieces = a.D / 8;
-    if (packed) {
-        const size_t rows = (size_t)a.B * a.S_q * kmax;
-        const size_t keys_bytes = (rows * kD * 2 + 255) & ~(size_t)255;
-        n_keys = reinterpret_cast<int32_t *>(ws + keys_bytes);
-        int32_t *ent_ws = reinterpret_cast<int32_t *>(ws + keys_bytes + (((size_t)a.B * a.S_q * 4 + 255) & ~(size_t)255));
-        kv_rows = rows;
-        pack_list_kernel<<<(unsigned)(a.B * a.S_q), 32, 0, st>>>(a.idx, a.mode == 0 ? a.topk : 0, a.mode, a.S_kv,
-                                                                 a.kv_pos0, a.P, a.S_q, a.q_pos0, a.window, a.ratio,
-                                                                 kmax, ent_ws, n_keys);
-        CSA_CHECK_LAUNCH("attend: list keys");
-        dim3 pg((unsigned)(a.B * a.S_q), (unsigned)ceil_div(kmax, kPackRows));
-        pack_rows_kernel<<<pg, 256, 0, st>>>((const __nv_bfloat16 *)a.kv, a.S_kv, a.kv_pos0,
-                                            (const __nv_bfloat16 *)a.pool, a.P, a.mode, a.S_q, a.q_pos0, a.window,
-                                            a.ratio, a.rope, ent_ws, n_keys, kv_rot, kmax);
-        CSA_CHECK_LAUNCH("attend: pack keys");
+    if (decode) {
+        kv_src = (const __nv_bfloat16 *)a.kv;
+        pool_src = (const __nv_bfloat16 *)a.pool;
+        k7 = reinterpret_cast<__nv_bfloat16 *>(ws);
+        if (nq > 0) {
+            pack_k7_kernel<<<dim3((unsigned)nq, (unsigned)(kmax7 / kTile)), kK7Threads, 0, st>>>(
+                kv_src, a.S_kv, a.kv_pos0, pool_src, a.P, a.idx, a.mode == 0 ? a.topk : 0, a.mode, a.S_q, a.q_pos0,
+                a.window, a.ratio, a.rope, kmax7, k7, (const __nv_bfloat16 *)a.q, q7);
+            CSA_CHECK_LAUNCH("attend: rotate the keys' rope chunks");
+        }
     } else {
-        pool_rot = reinterpret_cast<__nv_bfloat16 *>(ws + (((size_t)a.B * a.S_kv * a.D * 2 + 255) & ~(size_t)255));
-        kv_rows = (uint64_t)(a.B * a.S_kv > 0 ? a.B * a.S_kv : 1);
+        __nv_bfloat16 *kv_rot = reinterpret_cast<__nv_bfloat16 *>(ws);
+        __nv_bfloat16 *pool_rot = reinterpret_cast<__nv_bfloat16 *>(ws + round256((size_t)a.B * a.S_kv * a.D * 2));
+        kv_src = kv_rot;
+        pool_src = pool_rot;
         if (a.S_kv > 0) {
             dim3 g((unsigned)ceil_div(a.S_kv * pieces, 256), (unsigned)a.B);
             rope_rows_kernel<<<g, 256, 0, st>>>((const __nv_bfloat16 *)a.kv, kv_rot, a.S_kv, a.kv_pos0, 1,
@@ -1022,44 +1073,42 @@ csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st) {
                                                 a.D, a.rope);
             CSA_CHECK_LAUNCH("attend: rotate entries");
         }
+        // Q's last chunk, rotated once per call (decode-sized calls: in pack_k7_kernel)
+        if (q_rows > 0) {
+            rope_q_chunk_kernel<<<(unsigned)nq, kRopeQThreads, 0, st>>>((const __nv_bfloat16 *)a.q, q7, a.S_q,
+                                                                       a.q_pos0, a.rope);
+            CSA_CHECK_LAUNCH("attend: rotate query rows");
+        }
     }
-    // Q's last chunk, rotated once per call
-    __nv_bfloat16 *q7 = reinterpret_cast<__nv_bfloat16 *>(ws + keys_ws_bytes(a));
-    const int64_t q_rows = a.B * a.S_q * kH;
-    if (q_rows > 0) {
-        rope_q_chunk_kernel<<<(unsigned)(a.B * a.S_q), kRopeQThreads, 0, st>>>((const __nv_bfloat16 *)a.q, q7, a.S_q,
-                                                                            a.q_pos0, a.rope);
-        CSA_CHECK_LAUNCH("attend: rotate query rows");
-    }
-    CUtensorMap map_q, map_q7, map_kv, map_pool;
+    const uint64_t kv_rows = (uint64_t)(a.B * a.S_kv > 0 ? a.B * a.S_kv : 1);
+    CUtensorMap map_q, map_q7, map_kv, map_pool, map_k7;
     CSA_REQUIRE(encode_map_bf16_2d(&map_q, a.q, kD, (uint64_t)q_rows, 64u, 64u) &&
                     encode_map_bf16_2d(&map_q7, q7, 64u, (uint64_t)q_rows, 64u, 64u) &&
-                    encode_map_bf16_2d(&map_kv, kv_rot, kD, kv_rows, 64u, (uint32_t)kTile),
+                    encode_map_bf16_2d(&map_kv, kv_src, kD, kv_rows, 64u, (uint32_t)kTile),
                 CSA_ERR_CUDA, "attend: cannot encode the TMA tensor maps");
-    // the rotated pool as TMA rows (HCA entry tiles); other calls never use it
-    if (!packed && a.mode == 1 && a.P > 0)
-        CSA_REQUIRE(encode_map_bf16_2d(&map_pool, pool_rot, kD, (uint64_t)(a.B * a.P), 64u, (uint32_t)kTile),
+    // the pool as TMA rows (HCA entry tiles); other calls never use it
+    if (a.mode == 1 && a.P > 0)
+        CSA_REQUIRE(encode_map_bf16_2d(&map_pool, pool_src, kD, (uint64_t)(a.B * a.P), 64u, (uint32_t)kTile),
                     CSA_ERR_CUDA, "attend: cannot encode the pool tensor map");
     else
         map_pool = map_kv;
-    const size_t smem = tc_smem_bytes(a.mode == 0 && !packed ? a.topk : 1);
+    if (decode)
+        CSA_REQUIRE(encode_map_bf16_2d(&map_k7, k7, 64u, (uint64_t)(nq * kmax7), 64u, (uint32_t)kTile),
+                    CSA_ERR_CUDA, "attend: cannot encode the k7 tensor map");
+    else
+        map_k7 = map_kv;
+    const size_t smem = tc_smem_bytes(a.mode == 0 ? a.topk : 1);
     CSA_REQUIRE(smem <= 232448, CSA_ERR_UNSUPPORTED, "attend: shared memory %zu B too large", smem);
-    ensure_smem((const void *)attend_tc_kernel, smem);
+    auto kern = decode ? attend_tc_kernel<true> : attend_tc_kernel<false>;
+    ensure_smem((const void *)kern, smem);
     const int sms = device_sm_count();
-    const int64_t nq = a.B * a.S_q;
     const int n_split = attend_tc_split(a);
-    float *part = nullptr;
-    if (n_split > 1) {
-        const size_t rows = (size_t)a.B * a.S_q * kmax;
-        part = reinterpret_cast<float *>(ws + ((rows * kD * 2 + 255) & ~(size_t)255) +
-                                         (((size_t)a.B * a.S_q * 4 + 255) & ~(size_t)255) +
-                                         ((rows * 4 + 255) & ~(size_t)255));
-    }
+    float *part = n_split > 1 ? reinterpret_cast<float *>(ws + round256((size_t)nq * kmax7 * 64 * 2)) : nullptr;
     const int64_t nw = nq * n_split;
     const int grid = (int)(nw < sms ? nw : sms);
-    attend_tc_kernel<<<grid, kThreads, smem, st>>>(
-        map_q, map_q7, map_kv, map_pool, pool_rot, a.S_kv, a.kv_pos0, a.P, a.idx, a.mode == 0 && !packed ? a.topk : 0, a.mode,
-        a.sink, (__nv_bfloat16 *)a.out, a.B, a.S_q, a.q_pos0, a.window, a.ratio, a.scale, a.rope, n_keys, kmax,
+    kern<<<grid, kThreads, smem, st>>>(
+        map_q, map_q7, map_kv, map_pool, map_k7, pool_src, a.S_kv, a.kv_pos0, a.P, a.idx, a.mode == 0 ? a.topk : 0,
+        a.mode, a.sink, (__nv_bfloat16 *)a.out, a.B, a.S_q, a.q_pos0, a.window, a.ratio, a.scale, a.rope, kmax7,
         n_split, part);
     CSA_CHECK_LAUNCH(a.mode == 0 ? "csa_attend" : "hca_attend");
     if (n_split > 1) {
@@ -1084,7 +1133,7 @@ void *g_noalloc_ptr[kMaxDevices];  // device address of g_noalloc_scratch, per d
 }  // namespace
 
 csa_status_t attend_tc_noalloc(AttendArgs &a, cudaStream_t st) {
-    CSA_REQUIRE(attend_tc_eligible(a) && !attend_tc_packed(a), CSA_ERR_UNSUPPORTED,
+    CSA_REQUIRE(attend_tc_eligible(a) && !attend_tc_decode(a), CSA_ERR_UNSUPPORTED,
                 "csa_attend_noalloc: only the bf16, 64-head, head_dim-512 prefill shape is "
                 "handled (S_q * 64 >= S_kv + P)");
     const size_t need = attend_tc_workspace(a);

@@ -94,7 +94,15 @@ void make_rope_table(RopeTable *t, int D, int R, double base) {
     memset(t, 0, sizeof(*t));
     t->n_pairs = R / 2;
     t->first = D - R;
-    for (int i = 0; i < R / 2; ++i) t->inv_freq[i] = pow(base, -2.0 * (double)i / (double)R);
+    const long double two_pi = 6.283185307179586476925286766559005768L;
+    for (int i = 0; i < R / 2; ++i) {
+        // the frequency in turns per position (below 1/(2 pi) for base >= 1), as a 64-bit
+        // fraction; for base < 1 only its fractional part matters (whole turns drop out)
+        long double f = powl((long double)base, -2.0L * (long double)i / (long double)R) / two_pi;
+        f -= floorl(f);
+        const long double scaled = ldexpl(f, 64);
+        t->turn[i] = scaled >= 18446744073709551615.0L ? 0ull : (uint64_t)(scaled + 0.5L);
+    }
 }
 
 // ------------------------------------------------------------------ path selection

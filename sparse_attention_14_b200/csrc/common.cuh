@@ -81,24 +81,51 @@ __device__ __forceinline__ void store8(__nv_bfloat16 *p, const float *v) {
 }
 
 // ---------------------------------------------------------------- RoPE
-// Per-pair inverse frequencies base^(-2i/R), computed on the host in double and passed
-// by value so that concurrent calls with different bases never share state.
+// Per-pair frequencies base^(-2i/R) as 64-bit fixed-point turns per position,
+// turn[i] = round(base^(-2i/R) / (2 pi) * 2^64), computed on the host in long double and
+// passed by value so that concurrent calls with different bases never share state.
 constexpr int kMaxRopePairs = 128;
 struct RopeTable {
-    double inv_freq[kMaxRopePairs];
+    uint64_t turn[kMaxRopePairs];
     int n_pairs;   // R / 2
     int first;     // D - R: first rotated channel
 };
 void make_rope_table(RopeTable *t, int D, int R, double base);
 
-// cos/sin of pos * inv_freq.  The angle is reduced to [-pi, pi] in double first, so
-// positions up to 2^31 keep fp32-level accuracy; on that range the hardware
+// cos/sin of the angle pos * base^(-2i/R) for an integer position (negative for the
+// inverse rotation).  The angle's fraction of a turn is (pos * turn) mod 2^64 in integer
+// arithmetic -- exact up to the table's own rounding (|pos| * 2^-65 turns) -- whose top
+// 32 bits give the angle in [-pi, pi) to within 2e-7; on that range the hardware
 // approximation __sincosf is within ~5e-7 absolute, far below bf16/fp32 output rounding.
-__device__ __forceinline__ void rope_cs(double pos, double inv_freq, float *c, float *s) {
-    double phi = pos * inv_freq;
-    const double two_pi = 6.283185307179586476925286766559;
-    phi -= two_pi * rint(phi * (1.0 / two_pi));
-    __sincosf((float)phi, s, c);
+// (No fp64 arithmetic: it is far slower than fp32 on this GPU.)
+__device__ __forceinline__ void rope_cs(int64_t pos, uint64_t turn, float *c, float *s) {
+    const uint64_t frac = (uint64_t)pos * turn;
+    const float phi = (float)(int32_t)(uint32_t)(frac >> 32) * 1.46291807926715968105e-9f;   // 2 pi / 2^32
+    __sincosf(phi, s, c);
+}
+
+// The table is a kernel parameter (constant memory): an index shared by a warp is one
+// broadcast read, an index that differs between lanes is served one lane at a time.  So
+// kernels read it with warp-uniform indices only -- directly in loops over the pairs, or
+// through a shared-memory copy made by stage_turns.
+// Copy turn[0, n_pairs) into dst with the warps of a block of nthreads threads (each warp
+// its own few entries); the caller synchronises before reading dst.
+__device__ __forceinline__ void stage_turns(const RopeTable &rope, uint64_t *dst, int tid, int nthreads) {
+    const int nw = nthreads >> 5, w = tid >> 5, lane = tid & 31;
+    const int per = (rope.n_pairs + nw - 1) / nw;   // entries of warp w: [w*per, w*per + per)
+    for (int k0 = 0; k0 < per; k0 += 32) {
+        uint64_t mine = 0;
+#pragma unroll 4
+        for (int k = 0; k < 32; ++k) {
+            const int p = w * per + k0 + k;           // same index in every lane
+            if (k0 + k < per && p < rope.n_pairs) {
+                const uint64_t v = rope.turn[p];
+                if (lane == k) mine = v;
+            }
+        }
+        const int p = w * per + k0 + lane;
+        if (k0 + lane < per && p < rope.n_pairs) dst[p] = mine;
+    }
 }
 
 // ---------------------------------------------------------------- TMA descriptors

@@ -24,6 +24,9 @@ __global__ void __launch_bounds__(256) rope_any_kernel(const T *x, T *out, int64
                                                        int64_t pos0, int64_t group,
                                                        int64_t period, int64_t step,
                                                        RopeTable rope) {
+    __shared__ uint64_t turn_s[kMaxRopePairs];
+    stage_turns(rope, turn_s, threadIdx.x, blockDim.x);
+    __syncthreads();
     const int pieces = D / 8;
     const int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (v >= rows * pieces) return;
@@ -32,13 +35,13 @@ __global__ void __launch_bounds__(256) rope_any_kernel(const T *x, T *out, int64
     float a[8];
     load8(x + r * D + d0, a);
     if (d0 + 8 > rope.first) {
-        const double pos = (double)(pos0 + ((r / group) % period) * step);
+        const int64_t pos = pos0 + ((r / group) % period) * step;
 #pragma unroll
         for (int c = 0; c < 8; c += 2) {
             const int d = d0 + c;
             if (d >= rope.first) {
                 float cs, sn;
-                rope_cs(pos, rope.inv_freq[(d - rope.first) >> 1], &cs, &sn);
+                rope_cs(pos, turn_s[(d - rope.first) >> 1], &cs, &sn);
                 const float u = a[c], w = a[c + 1];
                 a[c] = u * cs - w * sn;
                 a[c + 1] = u * sn + w * cs;

@@ -224,8 +224,8 @@ def test_sink_minus_inf(name, pattern):
 
 def test_tensor_core_path_selected():
     """The V4-Flash head shape takes the tensor-core attention, which needs a workspace
-    (rotated keys for prefill, packed keys for decode-sized calls); other shapes take the
-    general path."""
+    (rotated keys for prefill, rotated rope chunks of the used keys for decode-sized
+    calls); other shapes take the general path."""
     import sparse_attention_14_b200 as csa
     for spec in MID + cs.WORKLOADS[1] + cs.WORKLOADS[2] + cs.WORKLOADS[3]:
         ws = csa.csa_attend_workspace_bytes(0 if spec.kind == "csa" else 1, spec.B, spec.S_q,
