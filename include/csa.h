@@ -307,9 +307,9 @@ uint32_t csa_device_status(void);
  * every wait on it gives up after a short bound (well under a millisecond); the kernel
  * then skips its work (out is left unwritten or holds partial values), frees its tensor
  * memory, returns and sets bit 0 of csa_device_status().  Nothing faults or hangs and the
- * context stays usable.  on == 0 restores normal operation.  Synchronous (a copy to a
- * device variable on the current device); call it only while no attention work is in
- * flight.  Returns CSA_ERR_CUDA if the copy fails.
+ * context stays usable.  on == 0 restores normal operation.  A process-wide host flag,
+ * passed to every attention launch enqueued after the call (a CUDA graph captured
+ * earlier keeps the value it was captured with).  Always returns CSA_OK.
  */
 csa_status_t csa_debug_withhold_attention_loads(int32_t on);
 

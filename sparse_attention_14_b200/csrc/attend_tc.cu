@@ -37,6 +37,7 @@
 //    pack_k7_kernel fills with the rotated last chunk of just the keys each query uses;
 //    with few queries, each query's key tiles are split over two CTAs that write
 //    unnormalised partials, merged (sink, division, de-rotation) by attend_combine_kernel.
+#include <atomic>
 #include <mutex>
 
 #include "attend.cuh"
@@ -45,10 +46,12 @@
 namespace csa {
 
 __device__ unsigned int g_attend_tc_status;
-// Test hook (csa_debug_withhold_attention_loads): when nonzero the loader publishes
-// nothing, so every bounded wait on it runs out after a short bound and the kernel takes
-// its error path (status bit, skipped work) without any fault or hang.
-__device__ unsigned int g_attend_tc_withhold;
+// Test hook (csa_debug_withhold_attention_loads): while set, the attention kernel is
+// launched with withhold = 1, its loader publishes nothing, so every bounded wait on it
+// runs out after a short bound and the kernel takes its error path (status bit, skipped
+// work) without any fault or hang.  A host flag passed as a kernel argument: a device
+// variable read at kernel entry would put a memory round trip before the first load.
+static std::atomic<int> g_attend_tc_withhold{0};
 
 namespace {
 
@@ -185,13 +188,15 @@ __global__ void __launch_bounds__(kRopeQThreads) rope_q_chunk_kernel(const __nv_
 // the attention's key tiles: rows qi*kmax7 + kt*128 + r hold window row kt*128 + r for the
 // n_wt window tiles, then entry (kt - n_wt)*128 + r (the valid idx values in slot order for
 // CSA, every visible entry for HCA); rows past the last key are zero.  Block (qi, kt) fills
-// tile kt of query qi; block (qi, 0) also writes the query's rotated chunk to q7.
+// tile kt of query qi; block (qi, 0) also writes the query's rotated chunk to q7.  For CSA
+// the blocks also write the compacted entry list (ent_g, row stride kmax7) and the entry
+// count (n_ent_g), which the attention's loaders read instead of compacting idx again.
 constexpr int kK7Threads = 256;
 __global__ void __launch_bounds__(kK7Threads) pack_k7_kernel(
     const __nv_bfloat16 *__restrict__ kv, int64_t S_kv, int64_t kv_pos0, const __nv_bfloat16 *__restrict__ pool,
     int64_t P, const int32_t *__restrict__ idx, int topk, int mode, int64_t S_q, int64_t q_pos0, int window,
     int ratio, RopeTable rope, int kmax7, __nv_bfloat16 *__restrict__ k7, const __nv_bfloat16 *__restrict__ q,
-    __nv_bfloat16 *__restrict__ q7) {
+    __nv_bfloat16 *__restrict__ q7, int32_t *__restrict__ ent_g, int32_t *__restrict__ n_ent_g) {
     __shared__ float cs_s[32], sn_s[32];
     __shared__ const __nv_bfloat16 *row_src[kTile];
     __shared__ int64_t row_pos[kTile];
@@ -242,6 +247,12 @@ __global__ void __launch_bounds__(kK7Threads) pack_k7_kernel(
             __syncthreads();
             int rank = incl - cnt;
             for (int k = 0; k < wp; ++k) rank += warp_cnt[k];
+            if (e0 == 0 && tid == 0) {
+                // the query's entry count, for the attention (the first entry tile's block)
+                int total = 0;
+                for (int k = 0; k < kK7Threads / 32; ++k) total += warp_cnt[k];
+                n_ent_g[qi] = total;
+            }
             for (int u = 0; u < per; ++u) {
                 const int c = tid * per + u;
                 if (c < topk) {
@@ -250,6 +261,7 @@ __global__ void __launch_bounds__(kK7Threads) pack_k7_kernel(
                         if (rank >= e0 && rank < e0 + kTile) {
                             row_src[rank - e0] = pool + (b * P + j) * kD;
                             row_pos[rank - e0] = (int64_t)j * ratio;
+                            ent_g[qi * (int64_t)kmax7 + rank] = j;   // the compacted list
                         }
                         ++rank;
                     }
@@ -364,8 +376,9 @@ struct QueryGeom {
 __device__ __forceinline__ QueryGeom query_geom(int64_t qi, int64_t S_q, int64_t q_pos0, int64_t kv_pos0,
                                                 int64_t S_kv, int window) {
     QueryGeom g;
-    g.b = qi / S_q;
-    g.i = qi % S_q;
+    // qi < B*S_q < 2^31 (checked on the host): 32-bit division
+    g.b = (int64_t)((uint32_t)qi / (uint32_t)S_q);
+    g.i = (int64_t)((uint32_t)qi % (uint32_t)S_q);
     g.t = q_pos0 + g.i;
     int64_t lo = g.t - window + 1;
     if (lo < kv_pos0) lo = kv_pos0;
@@ -386,7 +399,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     int64_t kv_pos0, int64_t P,
     const int32_t *__restrict__ idx, int topk, int mode, const float *__restrict__ sink,
     __nv_bfloat16 *__restrict__ out, int64_t B, int64_t S_q, int64_t q_pos0, int window, int ratio,
-    float scale, RopeTable rope, int kmax7, int n_split,
+    float scale, RopeTable rope, int kmax7, const int32_t *__restrict__ ent_g,
+    const int32_t *__restrict__ n_ent_g, int withhold, int n_split,
     float *__restrict__ part) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
@@ -397,12 +411,20 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     Small &sm = *reinterpret_cast<Small *>(smem + kOffEnt + kLoaders * ent_bytes);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const bool withhold = *reinterpret_cast<volatile unsigned int *>(&g_attend_tc_withhold) != 0u;
     const uint32_t kWaitIter = withhold ? (1u << 12) : kWaitIterMax;
     // work item w = query w / n_split, key-tile range w % n_split of it (n_split > 1 only for
     // decode-sized calls, whose partial results the combine kernel merges)
     const int64_t nw = B * S_q * n_split;
 
+    if (kK7 && tid == 32) {
+        // decode-sized calls (one work item per CTA): fetch the tensor-map descriptors while
+        // the barriers and tensor memory are set up
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_q)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_q7)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_kv)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_k7)) : "memory");
+        if (mode == 1) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_pool)) : "memory");
+    }
     if (tid == 0) {
         for (int c = 0; c < 8; ++c) mbar_init(&sm.full[c], 1);
         for (int c = 0; c < 4; ++c) mbar_init(&sm.free_[c], 1);
@@ -466,7 +488,29 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 }
             }
             int n_ent;
-            if (mode == 0) {
+            if (kK7 && mode == 0) {
+                // the count and the compacted list from pack_k7_kernel: the count first (the MMA
+                // issuer and softmax wait for it), then the list into this loader's copy
+                n_ent = ent_g ? n_ent_g[qi] : 0;
+                if (li == 0 && lane == 0) {
+                    sm.meta[qc & 1].n_ent = n_ent;
+                    mbar_arrive(&sm.meta_full[qc & 1]);
+                }
+                const int32_t *eg = ent_g + qi * (int64_t)kmax7;
+                for (int e0 = 0; e0 < n_ent; e0 += 8 * 32) {
+                    int32_t v[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int e = e0 + k * 32 + lane;
+                        v[k] = e < n_ent ? eg[e] : 0;
+                    }
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int e = e0 + k * 32 + lane;
+                        if (e < n_ent) ent[e] = v[k];
+                    }
+                }
+            } else if (mode == 0) {
                 // compact the valid idx values in slot order; eight loads per lane in flight
                 int cnt = 0;
                 const int32_t *ip = idx + qi * topk;
@@ -496,7 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 n_ent = (int)nv;
             }
             __syncwarp();
-            if (li == 0 && lane == 0) {
+            if (li == 0 && lane == 0 && !(kK7 && mode == 0)) {
                 sm.meta[qc & 1].n_ent = n_ent;
                 mbar_arrive(&sm.meta_full[qc & 1]);
             }
@@ -1023,12 +1067,25 @@ static size_t split_part_bytes(const AttendArgs &a, int n_split) {
 
 static size_t round256(size_t v) { return (v + 255) & ~(size_t)255; }
 
-// Workspace: the keys part (decode-sized calls: the rotated rope chunks k7 [B*S_q*kmax7, 64]
-// and the split partials; prefill: the rotated window rows and entries), then the rotated
-// last 64-column chunk of every query row [B*S_q*H, 64].
+// Workspace: the keys part, then the rotated last 64-column chunk of every query row
+// [B*S_q*H, 64].  Decode-sized calls: the rotated rope chunks k7 [B*S_q*kmax7, 64], the
+// compacted entry lists [B*S_q*kmax7] and counts [B*S_q] (CSA), the split partials.
+// Prefill: the rotated window rows and entries.
+struct DecodeWs {
+    size_t k7, ent, cnt, part, total;
+};
+static DecodeWs decode_ws(const AttendArgs &a) {
+    DecodeWs d;
+    const size_t nq = (size_t)a.B * a.S_q, kmax7 = (size_t)attend_tc_kmax7(a);
+    d.k7 = 0;
+    d.ent = round256(nq * kmax7 * 64 * 2);
+    d.cnt = d.ent + round256(nq * kmax7 * 4);
+    d.part = d.cnt + round256(nq * 4);
+    d.total = d.part + split_part_bytes(a, attend_tc_split(a));
+    return d;
+}
 static size_t keys_ws_bytes(const AttendArgs &a) {
-    if (attend_tc_decode(a))
-        return round256((size_t)a.B * a.S_q * attend_tc_kmax7(a) * 64 * 2) + split_part_bytes(a, attend_tc_split(a));
+    if (attend_tc_decode(a)) return decode_ws(a).total;
     return round256((size_t)a.B * a.S_kv * a.D * 2) + round256((size_t)a.B * a.P * a.D * 2);
 }
 
@@ -1045,15 +1102,24 @@ csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st) {
     __nv_bfloat16 *q7 = reinterpret_cast<__nv_bfloat16 *>(ws + keys_ws_bytes(a));
     const __nv_bfloat16 *kv_src, *pool_src;   // key rows the tiles read
     __nv_bfloat16 *k7 = nullptr;
+    int32_t *ent_g = nullptr, *n_ent_g = nullptr;
+    float *part = nullptr;
     const int pieces = a.D / 8;
     if (decode) {
+        const DecodeWs d = decode_ws(a);
         kv_src = (const __nv_bfloat16 *)a.kv;
         pool_src = (const __nv_bfloat16 *)a.pool;
-        k7 = reinterpret_cast<__nv_bfloat16 *>(ws);
+        k7 = reinterpret_cast<__nv_bfloat16 *>(ws + d.k7);
+        // CSA with entries to list: the compacted lists and counts (written by pack_k7)
+        if (a.mode == 0 && a.topk > 0 && a.P > 0) {
+            ent_g = reinterpret_cast<int32_t *>(ws + d.ent);
+            n_ent_g = reinterpret_cast<int32_t *>(ws + d.cnt);
+        }
+        if (attend_tc_split(a) > 1) part = reinterpret_cast<float *>(ws + d.part);
         if (nq > 0) {
             pack_k7_kernel<<<dim3((unsigned)nq, (unsigned)(kmax7 / kTile)), kK7Threads, 0, st>>>(
                 kv_src, a.S_kv, a.kv_pos0, pool_src, a.P, a.idx, a.mode == 0 ? a.topk : 0, a.mode, a.S_q, a.q_pos0,
-                a.window, a.ratio, a.rope, kmax7, k7, (const __nv_bfloat16 *)a.q, q7);
+                a.window, a.ratio, a.rope, kmax7, k7, (const __nv_bfloat16 *)a.q, q7, ent_g, n_ent_g);
             CSA_CHECK_LAUNCH("attend: rotate the keys' rope chunks");
         }
     } else {
@@ -1103,13 +1169,12 @@ csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st) {
     ensure_smem((const void *)kern, smem);
     const int sms = device_sm_count();
     const int n_split = attend_tc_split(a);
-    float *part = n_split > 1 ? reinterpret_cast<float *>(ws + round256((size_t)nq * kmax7 * 64 * 2)) : nullptr;
     const int64_t nw = nq * n_split;
     const int grid = (int)(nw < sms ? nw : sms);
     kern<<<grid, kThreads, smem, st>>>(
         map_q, map_q7, map_kv, map_pool, map_k7, pool_src, a.S_kv, a.kv_pos0, a.P, a.idx, a.mode == 0 ? a.topk : 0,
         a.mode, a.sink, (__nv_bfloat16 *)a.out, a.B, a.S_q, a.q_pos0, a.window, a.ratio, a.scale, a.rope, kmax7,
-        n_split, part);
+        ent_g, n_ent_g, g_attend_tc_withhold.load(), n_split, part);
     CSA_CHECK_LAUNCH(a.mode == 0 ? "csa_attend" : "hca_attend");
     if (n_split > 1) {
         attend_combine_kernel<<<dim3((unsigned)nq, kH / kCombHeads), kD / 2, 0, st>>>(
@@ -1166,9 +1231,7 @@ csa_status_t attend_tc_noalloc(AttendArgs &a, cudaStream_t st) {
 }
 
 csa_status_t set_attend_tc_withhold(int on) {
-    const unsigned int v = on ? 1u : 0u;
-    cudaError_t e = cudaMemcpyToSymbol(g_attend_tc_withhold, &v, sizeof(v));
-    CSA_REQUIRE(e == cudaSuccess, CSA_ERR_CUDA, "csa_debug_withhold_attention_loads: %s", cudaGetErrorString(e));
+    g_attend_tc_withhold.store(on ? 1 : 0);
     return CSA_OK;
 }
 

@@ -49,7 +49,7 @@ struct Misc {
     unsigned long long sel_prefix[4];
     unsigned sel_remaining[4];
     int sel_done[4];
-    unsigned warp_part[4][8];
+    unsigned warp_part[4][16];   // per group, per warp (groups of up to 512 threads)
     int abort_;
 };
 
@@ -100,6 +100,7 @@ __device__ __forceinline__ float key_to_float(uint32_t key) {
 template <int GS>
 __device__ unsigned long long group_kth(const unsigned long long *a, int n, int k, int gt, int bar,
                                         unsigned *hist, Misc &ms, int g) {
+    static_assert(GS <= 512, "warp_part holds 16 warps per group");
     constexpr int BPT = 256 / GS > 0 ? 256 / GS : 1;
     const int lane = gt & 31, wid = gt >> 5;
     if (gt == 0) {
@@ -322,7 +323,7 @@ __global__ void __launch_bounds__(Cfg<QB>::kThreads, Cfg<QB>::kMinBlocks) index_
     const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
     const __nv_bfloat16 *__restrict__ w, int64_t B, int64_t S_q, int64_t q_pos0, int64_t P, int ratio,
     int topk, int n_split, int32_t *__restrict__ idx, float *__restrict__ scores_opt,
-    unsigned long long *__restrict__ partial) {
+    unsigned long long *__restrict__ partial, unsigned long long *__restrict__ keys_out) {
     using C = Cfg<QB>;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -364,10 +365,6 @@ __global__ void __launch_bounds__(Cfg<QB>::kThreads, Cfg<QB>::kMinBlocks) index_
             ms.thr[q] = 0ull;
         }
         ms.abort_ = 0;
-    }
-    for (int e = tid; e < QB * 64; e += blockDim.x) {
-        const int q = e >> 6, h = e & 63;
-        w_s[e] = q < nq_valid ? __bfloat162float(w[((b * S_q) + i0 + q) * kHI + h]) : 0.f;
     }
     if (warp == 1) tmem_alloc(&ms.tmem_base, C::kTmemCols);
     tc_fence_before();
@@ -423,6 +420,13 @@ __global__ void __launch_bounds__(Cfg<QB>::kThreads, Cfg<QB>::kMinBlocks) index_
         }
     } else {
         // ---------------- epilogue: scores, streaming top-k
+        // the head weights, loaded here so that the producer's first loads do not wait
+        // for them
+        for (int v = tid - 64; v < QB * 64; v += C::NE * 32) {
+            const int q = v >> 6, h = v & 63;
+            w_s[v] = q < nq_valid ? __bfloat162float(w[((b * S_q) + i0 + q) * kHI + h]) : 0.f;
+        }
+        named_sync(1, C::NE * 32);
         const int e = warp - 2;                      // 0 .. NE-1
         const int g4 = warp & 3;                     // TMEM lane group of this warp
         const int row = g4 * 32 + lane;              // entry row inside the tile
@@ -467,6 +471,16 @@ __global__ void __launch_bounds__(Cfg<QB>::kThreads, Cfg<QB>::kMinBlocks) index_
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&ms.tempty[acc]);
+            if (QB == 1 && keys_out) {
+                // keys only: every visible entry's key goes to the row's slot j; the
+                // selection runs in index_select_kernel.  No barrier inside the loop here, so
+                // a thread whose wait ran out leaves on its own.
+                if (j < nvq[0])
+                    keys_out[(b * S_q + i0) * P + j] = ((unsigned long long)order_key(sc[0]) << 32) |
+                                                       (unsigned long long)(0xFFFFFFFFu - (uint32_t)j);
+                if (!ok) break;
+                continue;
+            }
             if (QB == 1 && C::NE == 8) {
                 // warps e and e+4 hold the two halves of the head sum of the same rows
                 float *part = reinterpret_cast<float *>(hist_all);   // 128 floats, free here
@@ -502,7 +516,7 @@ __global__ void __launch_bounds__(Cfg<QB>::kThreads, Cfg<QB>::kMinBlocks) index_
             if (named_sync_any(1, C::NE * 32, !ok)) break;
         }
         // final: this group's query
-        if (grp < nq_valid) {
+        if (grp < nq_valid && !keys_out) {
             const int q = grp;
             unsigned long long *cand = cand_all + q * kCap;
             group_cut<C::GS>(cand, topk, gt, 2 + q, hist_all + q * 256, ms, q, q);
@@ -546,6 +560,181 @@ __global__ void __launch_bounds__(kMergeThreads) index_merge_kernel(
                                 scores_opt ? scores_opt + row * topk : nullptr);
 }
 
+// Top-k of one query row from the keys of all its visible entries (decode calls whose
+// indexer wrote keys instead of candidates).  1024 threads hold the row's keys in
+// registers, 16 each (entry e = u*1024 + tid).  The scores are binned by value between
+// the row's min and max, bin = floor((score - min) * 2048 / (max - min)) -- a monotone map,
+// so equal scores share a bin and bins are ordered like the keys.  (Binning the score's
+// order-preserving bits instead is logarithmic in the score: with scores near zero in
+// the row, the top of the range falls into a handful of crowded bins.)  The bin holding the k-th largest key is found from
+// the bin counts, and only that bin's keys are ranked: by counting (each of at most 1024
+// keys against the others) or, for a crowded bin, by the radix select group_kth run by
+// 512 of the threads, tightened to the k-th key itself.  The entries with key >= T -- exactly k, the keys
+// being unique -- are written in ascending entry order through a bitmap built with warp
+// ballots.
+constexpr int kSelThreads = 1024, kSelPer = 16, kSelMax = kSelThreads * kSelPer, kSelBins = 2048;
+__global__ void __launch_bounds__(kSelThreads) index_select_kernel(
+    const unsigned long long *__restrict__ keys, int64_t P, int topk, int32_t *__restrict__ idx,
+    float *__restrict__ scores_opt, int64_t S_q, int64_t q_pos0, int ratio) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    unsigned long long *sub = reinterpret_cast<unsigned long long *>(smem_raw);   // [kSelMax] chosen bin
+    unsigned *bitmap = reinterpret_cast<unsigned *>(sub + kSelMax);              // [kSelMax / 32]
+    unsigned *bins = bitmap + kSelMax / 32;                                       // [kSelBins]
+    unsigned *hist = bins + kSelBins;                                             // [256]
+    unsigned *wpart = hist + 256;                                                 // [32]
+    float *red = reinterpret_cast<float *>(wpart + 32);                           // [64]
+    Misc &ms = *reinterpret_cast<Misc *>(red + 64);
+    __shared__ int sel_bin, sel_above, sel_n;
+    __shared__ unsigned long long sel_T;
+    const int64_t row = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int n = (int)n_visible(q_pos0 + row % S_q, ratio, P);   // <= kSelMax (host check)
+    const unsigned long long *kr = keys + row * P;
+    int32_t *idx_row = idx + row * (int64_t)topk;
+    float *score_row = scores_opt ? scores_opt + row * (int64_t)topk : nullptr;
+
+    unsigned long long key[kSelPer];
+#pragma unroll
+    for (int u = 0; u < kSelPer; ++u) {
+        const int e = u * kSelThreads + tid;
+        key[u] = e < n ? __ldcg(kr + e) : 0ull;
+    }
+    float lo = INFINITY, hi = -INFINITY;   // range of the scores
+#pragma unroll
+    for (int u = 0; u < kSelPer; ++u) {
+        if (u * kSelThreads + tid < n) {
+            const float f = key_to_float((uint32_t)(key[u] >> 32));
+            lo = fminf(lo, f);
+            hi = fmaxf(hi, f);
+        }
+    }
+    for (int b = tid; b < kSelBins; b += kSelThreads) bins[b] = 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        lo = fminf(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, o));
+        hi = fmaxf(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, o));
+    }
+    if (lane == 0) {
+        red[wid] = lo;
+        red[32 + wid] = hi;
+    }
+    if (tid == 0) {
+        sel_n = 0;
+        sel_T = 0ull;   // every key is > 0: all entries selected when n <= topk
+    }
+    __syncthreads();
+    if (n > topk) {
+        lo = red[0];
+        hi = red[32];
+        for (int w = 1; w < kSelThreads / 32; ++w) {
+            lo = fminf(lo, red[w]);
+            hi = fmaxf(hi, red[32 + w]);
+        }
+        const float scale = hi > lo ? (float)kSelBins / (hi - lo) : 0.f;
+        auto bin_of = [&](unsigned long long c) {
+            const float f = key_to_float((uint32_t)(c >> 32));
+            const int b = (int)((f - lo) * scale);
+            return b < 0 ? 0 : (b >= kSelBins ? kSelBins - 1 : b);
+        };
+#pragma unroll
+        for (int u = 0; u < kSelPer; ++u)
+            if (u * kSelThreads + tid < n) atomicAdd(&bins[bin_of(key[u])], 1u);
+        __syncthreads();
+        // the bin holding the topk-th largest key: suffix counts over bins, 2 per thread
+        constexpr int BPT = kSelBins / kSelThreads;
+        const int b_hi = kSelBins - tid * BPT;   // my bins: [b_hi - BPT, b_hi), from the top
+        unsigned local = 0;
+#pragma unroll
+        for (int k = 1; k <= BPT; ++k) local += bins[b_hi - k];
+        unsigned incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (lane == 31) wpart[wid] = incl;
+        __syncthreads();
+        unsigned cum = incl - local;   // keys in bins above mine
+        for (int w = 0; w < wid; ++w) cum += wpart[w];
+#pragma unroll
+        for (int k = 1; k <= BPT; ++k) {
+            const unsigned h = bins[b_hi - k];
+            if (cum < (unsigned)topk && (unsigned)topk <= cum + h) {
+                sel_bin = b_hi - k;
+                sel_above = (int)cum;
+            }
+            cum += h;
+        }
+        __syncthreads();
+        const int bstar = sel_bin;
+#pragma unroll
+        for (int u = 0; u < kSelPer; ++u)
+            if (u * kSelThreads + tid < n && bin_of(key[u]) == bstar) sub[atomicAdd(&sel_n, 1)] = key[u];
+        __syncthreads();
+        const int nb = sel_n, kb = topk - sel_above;   // the kb-th largest of the bin's nb keys
+        if (nb <= kSelThreads) {
+            if (tid < nb) {
+                const unsigned long long mine = sub[tid];
+                int rank = 0;
+                for (int i = 0; i < nb; ++i) rank += sub[i] > mine ? 1 : 0;
+                if (rank == kb - 1) sel_T = mine;
+            }
+        } else if (tid < 512) {
+            // crowded bin (many equal or near-equal scores): radix select by warps 0-15,
+            // then the smallest of the bin's keys >= its prefix threshold
+            const unsigned long long t = group_kth<512>(sub, nb, kb, tid, 2, hist, ms, 0);
+            if (tid == 0) sel_T = ~0ull;
+            named_sync(2, 512);
+            for (int e = tid; e < nb; e += 512)
+                if (sub[e] >= t) atomicMin(&sel_T, sub[e]);
+        }
+        __syncthreads();
+    }
+    const unsigned long long T = sel_T;
+    // bitmap of the selected entries: word u*32 + wid holds entries (u*1024 + wid*32 + lane)
+    const int nwords = (n + 31) >> 5;
+#pragma unroll
+    for (int u = 0; u < kSelPer; ++u) {
+        const int e = u * kSelThreads + tid;
+        const unsigned m = __ballot_sync(0xFFFFFFFFu, e < n && key[u] >= T);
+        if (lane == 0 && (e >> 5) < nwords) bitmap[e >> 5] = m;
+    }
+    __syncthreads();
+    // output slots: thread tid owns words [tid*wpt, (tid+1)*wpt); exclusive scan of counts
+    const int wpt = (nwords + kSelThreads - 1) / kSelThreads;
+    unsigned local = 0;
+    for (int w = tid * wpt; w < (tid + 1) * wpt && w < nwords; ++w) local += __popc(bitmap[w]);
+    unsigned incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) wpart[wid] = incl;
+    __syncthreads();
+    unsigned pos = incl - local;
+    for (int w = 0; w < wid; ++w) pos += wpart[w];
+    for (int w = tid * wpt; w < (tid + 1) * wpt && w < nwords; ++w) {
+        unsigned m = bitmap[w];
+        while (m) {
+            const int j = 32 * w + __ffs(m) - 1;
+            m &= m - 1u;
+            idx_row[pos] = j;
+            if (score_row) score_row[pos] = key_to_float((uint32_t)(__ldcg(kr + j) >> 32));
+            ++pos;
+        }
+    }
+    const int n_sel = n < topk ? n : topk;
+    for (int r = n_sel + tid; r < topk; r += kSelThreads) {
+        idx_row[r] = -1;
+        if (score_row) score_row[r] = __int_as_float(0x7fc00000);
+    }
+}
+
+// the chosen bin's keys, bitmap, bins, radix histogram, scan and min/max partials, Misc
+constexpr size_t kSelSmem =
+    (size_t)kSelMax * 8 + kSelMax / 32 * 4 + kSelBins * 4 + 256 * 4 + 32 * 4 + 64 * 4 + sizeof(Misc);
+
 // ------------------------------------------------------------------ host side
 bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint32_t box_rows) {
     return encode_map_bf16_2d(m, ptr, kDI, rows, 64u, box_rows);
@@ -558,6 +747,8 @@ int sm_count() {
 struct Plan {
     int qb;
     int n_split;
+    bool keys;   // split decode rows: the indexer writes every visible entry's key, then
+                 // index_select_kernel selects (rows with at most kSelMax visible entries)
 };
 
 Plan plan(int64_t B, int64_t S_q, int64_t q_pos0, int64_t P, int ratio, int topk) {
@@ -574,13 +765,15 @@ Plan plan(int64_t B, int64_t S_q, int64_t q_pos0, int64_t P, int ratio, int topk
     if (ns > 16) ns = 16;
     while (ns > 1 && (int64_t)pow2_ceil((int)(ns * topk)) > 8192) --ns;
     p.n_split = (int)(ns < 1 ? 1 : ns);
+    p.keys = p.n_split > 1 && p.qb == 1 && n_visible(q_pos0 + S_q - 1, ratio, P) <= kSelMax;
     return p;
 }
 
 template <int QB>
 csa_status_t launch(const CUtensorMap &mk, const CUtensorMap &mq, const __nv_bfloat16 *w, int64_t B,
                     int64_t S_q, int64_t q_pos0, int64_t P, int ratio, int topk, int n_split, int32_t *idx,
-                    float *scores_opt, unsigned long long *partial, cudaStream_t st) {
+                    float *scores_opt, unsigned long long *partial, unsigned long long *keys_out,
+                    cudaStream_t st) {
     using C = Cfg<QB>;
     const int64_t n_qb = B * ((S_q + QB - 1) / QB);
     const int64_t grid = n_qb * n_split;
@@ -588,7 +781,7 @@ csa_status_t launch(const CUtensorMap &mk, const CUtensorMap &mq, const __nv_bfl
     auto kern = index_tc_kernel<QB>;
     ensure_smem((const void *)kern, C::kSmem);
     kern<<<(unsigned)grid, C::kThreads, C::kSmem, st>>>(mk, mq, w, B, S_q, q_pos0, P, ratio, topk, n_split,
-                                                        idx, scores_opt, partial);
+                                                        idx, scores_opt, partial, keys_out);
     CSA_CHECK_LAUNCH("csa_index_topk");
     return CSA_OK;
 }
@@ -606,10 +799,15 @@ static size_t partial_bytes(const Plan &p, int64_t B, int64_t S_q, int topk) {
     return ((size_t)B * S_q * p.n_split * topk * sizeof(unsigned long long) + 255) & ~(size_t)255;
 }
 
+static size_t keys_bytes(int64_t B, int64_t S_q, int64_t P) {
+    return ((size_t)B * S_q * P * sizeof(unsigned long long) + 255) & ~(size_t)255;
+}
+
 size_t index_tc_workspace(int64_t B, int64_t S_q, int64_t q_pos0, int64_t P, int ratio, int topk) {
     Plan p = plan(B, S_q, q_pos0, P, ratio, topk);
     if (p.n_split <= 1) return 0;
-    return partial_bytes(p, B, S_q, topk);   // candidates per (row, range)
+    if (p.keys) return keys_bytes(B, S_q, P);   // every visible entry's key per row
+    return partial_bytes(p, B, S_q, topk);      // candidates per (row, range)
 }
 
 csa_status_t index_tc(const void *qI, const void *w, const void *kI, int64_t B, int64_t S_q, int64_t q_pos0,
@@ -621,20 +819,27 @@ csa_status_t index_tc(const void *qI, const void *w, const void *kI, int64_t B, 
     Plan p = plan(B, S_q, q_pos0, P, ratio, topk);
     CSA_REQUIRE(make_map(&mq, qI, (uint64_t)B * S_q * kHI, (uint32_t)(p.qb * 64)), CSA_ERR_CUDA,
                 "csa_index_topk: cannot encode the q_I tensor map");
-    unsigned long long *partial = nullptr;
+    unsigned long long *partial = nullptr, *keys = nullptr;
     if (p.n_split > 1) {
-        const size_t need = partial_bytes(p, B, S_q, topk);
+        const size_t need = p.keys ? keys_bytes(B, S_q, P) : partial_bytes(p, B, S_q, topk);
         CSA_REQUIRE(workspace && workspace_bytes >= need, CSA_ERR_WORKSPACE,
                     "csa_index_topk: workspace of %zu B given, %zu B needed", workspace_bytes, need);
-        partial = reinterpret_cast<unsigned long long *>(workspace);
+        (p.keys ? keys : partial) = reinterpret_cast<unsigned long long *>(workspace);
     }
     csa_status_t r;
     const __nv_bfloat16 *wb = reinterpret_cast<const __nv_bfloat16 *>(w);
     if (p.qb == 4)
-        r = launch<4>(mk, mq, wb, B, S_q, q_pos0, P, ratio, topk, p.n_split, idx, scores_opt, partial, st);
+        r = launch<4>(mk, mq, wb, B, S_q, q_pos0, P, ratio, topk, p.n_split, idx, scores_opt, partial, nullptr, st);
     else
-        r = launch<1>(mk, mq, wb, B, S_q, q_pos0, P, ratio, topk, p.n_split, idx, scores_opt, partial, st);
+        r = launch<1>(mk, mq, wb, B, S_q, q_pos0, P, ratio, topk, p.n_split, idx, scores_opt, partial, keys, st);
     if (r != CSA_OK || p.n_split <= 1) return r;
+    if (p.keys) {
+        ensure_smem((const void *)index_select_kernel, kSelSmem);
+        index_select_kernel<<<(unsigned)(B * S_q), kSelThreads, kSelSmem, st>>>(keys, P, topk, idx, scores_opt,
+                                                                               S_q, q_pos0, ratio);
+        CSA_CHECK_LAUNCH("csa_index_topk select");
+        return CSA_OK;
+    }
     const int total = p.n_split * topk;
     const size_t smem = (size_t)(pow2_ceil(total) + pow2_ceil(topk)) * 8 + 256 * 4 + sizeof(Misc) +
                         (size_t)((P + 31) / 32) * 4;
