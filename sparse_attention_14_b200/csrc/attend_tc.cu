@@ -35,8 +35,10 @@
 //    0-6 of window rows by TMA from the raw rows, of entries by 16-byte copies from the
 //    pool, and chunk 7 (the rope channels) by TMA from a small buffer that
 //    pack_k7_kernel fills with the rotated last chunk of just the keys each query uses;
-//    with few queries, each query's key tiles are split over two CTAs that write
-//    unnormalised partials, merged (sink, division, de-rotation) by attend_combine_kernel.
+//    with few queries, each query's key tiles are split over the two CTAs of a cluster:
+//    the second (never more tiles) writes its unnormalised O^T, maxima and row sums to the
+//    workspace and releases them with a cluster-scope arrive on the first's barrier; the
+//    first merges them (sink, division, de-rotation) and stores the output.
 #include <atomic>
 #include <mutex>
 
@@ -78,6 +80,7 @@ struct Meta {
 
 struct Small {
     uint64_t full[8], free_[4], s_full, p_full, o_full, q_tma, q_free, meta_full[2], drain;
+    uint64_t peer_data;   // split decode pair: the rank-1 CTA's partial is in the workspace
     uint32_t tmem_base;
     int abort_;
     int last_tma[8];   // per key slot: tile counter of its last TMA load, -1 if its last load was not one
@@ -400,8 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     const int32_t *__restrict__ idx, int topk, int mode, const float *__restrict__ sink,
     __nv_bfloat16 *__restrict__ out, int64_t B, int64_t S_q, int64_t q_pos0, int window, int ratio,
     float scale, RopeTable rope, int kmax7, const int32_t *__restrict__ ent_g,
-    const int32_t *__restrict__ n_ent_g, int withhold, int n_split,
-    float *__restrict__ part) {
+    const int32_t *__restrict__ n_ent_g, int withhold, int n_split, float *__restrict__ part) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     unsigned char *smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -436,6 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         mbar_init(&sm.meta_full[0], 1);
         mbar_init(&sm.meta_full[1], 1);
         mbar_init(&sm.drain, 1);
+        mbar_init(&sm.peer_data, kSoftThreads);
         fence_mbar_init();
         sm.abort_ = 0;
         for (int c = 0; c < 8; ++c) sm.last_tma[c] = -1;
@@ -444,6 +447,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // split decode queries run as 2-CTA clusters: both CTAs' barriers are initialised before
+    // either arrives on the other's
+    const bool pair = kK7 && n_split == 2;
+    if (pair) cluster_sync_all();
     const uint32_t tmem = sm.tmem_base;
 
     if (warp == 0 || warp == 10) {
@@ -848,20 +855,69 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             warp_reduce32<false>(l_part);
             sm.red[lg][hb + lane] = l_part[0];
             named_sync(1, kSoftThreads);
-            if (part) {
-                // a key range of a split query: unnormalised O^T, the running maxima (log2
-                // units) and the row sums without the sink, for the combine kernel
-                float *pml = part + nw * (int64_t)(kH * kD) + w * (2 * kH);
-                if (st < kH) {
-                    pml[st] = sm.m_used[st];
-                    pml[kH + st] = sm.red[0][st] + sm.red[1][st] + sm.red[2][st] + sm.red[3][st];
-                }
+            if (pair) {
+                // a split query's CTA pair (cluster ranks 0 and 1 = key ranges 0 and 1; rank 0
+                // never has fewer tiles): rank 1 writes its unnormalised O^T [64 heads, 512],
+                // running maxima and row sums (log2 units, no sink) to the workspace as soon as
+                // its MMAs are done and releases them with a cluster-scope arrive on rank 0's
+                // barrier; rank 0 finishes its own tiles, acquires, merges and stores
                 ok = !named_sync_any(1, kSoftThreads, !mbar_wait(&sm.o_full, qc & 1u, kWaitIter));
                 if (!ok) break;
                 tc_fence_after();
-                float *po = part + w * (int64_t)(kH * kD);
+                float *pm = part + qi * (int64_t)(2 * kH);                 // m[64], l[64]
+                float *po = part + B * S_q * (2 * kH) + qi * (int64_t)(kH * kD);
+                if ((w % 2) == 1) {
+                    if (st < kH) {
+                        pm[st] = sm.m_used[st];
+                        pm[kH + st] = sm.red[0][st] + sm.red[1][st] + sm.red[2][st] + sm.red[3][st];
+                    }
+#pragma unroll 1
+                    for (int mt = 0; mt < 4; ++mt) {
+                        float o[32];
+                        if (kt1 > kt0) {
+                            tmem_ld32(trow + kColO + mt * 64 + hb, o);
+                            tmem_ld_wait();
+                        } else {
+#pragma unroll
+                            for (int h = 0; h < 32; ++h) o[h] = 0.f;
+                        }
+#pragma unroll
+                        for (int h = 0; h < 32; ++h) po[(int64_t)(hb + h) * kD + mt * 128 + x] = o[h];
+                    }
+                    tc_fence_before();
+                    // every thread releases its own writes with its arrival (count kSoftThreads)
+                    mbar_arrive_remote(cluster_map(smem_u32(&sm.peer_data), 0));
+                    continue;
+                }
+                ok = !named_sync_any(1, kSoftThreads, !mbar_wait_cluster(&sm.peer_data, 0u, kWaitIter));
+                if (!ok) break;
+                if (st < kH) {
+                    // M over both ranges and the sink; weights 2^(m_s - M) / l
+                    const float m0 = sm.m_used[st], m1 = __ldcg(pm + st);
+                    const float l0 = sm.red[0][st] + sm.red[1][st] + sm.red[2][st] + sm.red[3][st];
+                    const float l1 = __ldcg(pm + kH + st);
+                    const float sk = sink[st];
+                    float M = sk == -INFINITY ? -INFINITY : sk * kLog2e;
+                    M = fmaxf(M, fmaxf(m0, m1));
+                    const float w0 = M == -INFINITY ? 0.f : exp2f(m0 - M);
+                    const float w1 = M == -INFINITY ? 0.f : exp2f(m1 - M);
+                    float l = w0 * l0 + w1 * l1;
+                    if (sk != -INFINITY && M != -INFINITY) l += exp2f(sk * kLog2e - M);
+                    const float il = l > 0.f ? 1.f / l : 0.f;
+                    sm.alpha[st] = w0 * il;
+                    sm.inv_l[st] = w1 * il;
+                }
+                named_sync(1, kSoftThreads);
+                __nv_bfloat16 *orow = out + qi * (int64_t)kH * kD;
 #pragma unroll 1
                 for (int mt = 0; mt < 4; ++mt) {
+                    const int d = mt * 128 + x;
+                    float o1[32];
+#pragma unroll
+                    for (int h = 0; h < 32; ++h) o1[h] = __ldcg(po + (int64_t)(hb + h) * kD + d);
+                    float cs = 1.f, sn = 0.f;
+                    const bool rot = d >= rope.first;
+                    if (rot) rope_cs(-qg.t, rope.turn[(d - rope.first) >> 1], &cs, &sn);
                     float o[32];
                     if (kt1 > kt0) {
                         tmem_ld32(trow + kColO + mt * 64 + hb, o);
@@ -871,7 +927,20 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                         for (int h = 0; h < 32; ++h) o[h] = 0.f;
                     }
 #pragma unroll
-                    for (int h = 0; h < 32; ++h) po[(int64_t)(hb + h) * kD + mt * 128 + x] = o[h];
+                    for (int h = 0; h < 32; ++h) o[h] = o[h] * sm.alpha[hb + h] + o1[h] * sm.inv_l[hb + h];
+                    float pr[32];
+#pragma unroll
+                    for (int h = 0; h < 32; ++h) pr[h] = __shfl_xor_sync(0xFFFFFFFFu, o[h], 1);
+                    if ((lane & 1) == 0) {
+#pragma unroll
+                        for (int h = 0; h < 32; ++h) {
+                            const float a = o[h], bb = pr[h];
+                            const float ra = rot ? a * cs - bb * sn : a;
+                            const float rb = rot ? a * sn + bb * cs : bb;
+                            *reinterpret_cast<__nv_bfloat162 *>(orow + (int64_t)(hb + h) * kD + d) =
+                                __floats2bfloat162_rn(ra, rb);
+                        }
+                    }
                 }
                 tc_fence_before();
                 continue;
@@ -933,88 +1002,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // neither CTA of a pair leaves while the other may still write to its shared memory
+    if (pair) cluster_sync_all();
     if (warp == 1) tmem_dealloc(tmem, 512);
-}
-
-// Merges the key-range partials of split queries: per head, M = max over the ranges (and
-// the sink), weights 2^(m_s - M), l = sum of weighted row sums plus the sink term, then
-// O = sum of weighted O_s / l, the -t de-rotation of the rope channels and the bf16 store.
-// Block (query, group of 8 heads); every thread loads its 8 channel pairs of every range
-// before combining them, so the reads of a block are all in flight together.
-constexpr int kMaxSplit = 4;
-constexpr int kCombHeads = 8;
-__global__ void __launch_bounds__(256) attend_combine_kernel(const float *__restrict__ part, int n_split,
-                                                             int64_t nq, const float *__restrict__ sink,
-                                                             __nv_bfloat16 *__restrict__ out, int64_t S_q,
-                                                             int64_t q_pos0, RopeTable rope) {
-    __shared__ float wgt[kCombHeads][kMaxSplit];
-    __shared__ float inv_l[kCombHeads];
-    __shared__ float rcs[2][32];
-    const int64_t qi = blockIdx.x;
-    const int h0 = blockIdx.y * kCombHeads;
-    const int tid = threadIdx.x;
-    const float *pml = part + nq * n_split * (int64_t)(kH * kD);
-    if (tid < kCombHeads) {
-        const int h = h0 + tid;
-        const float sk = sink[h];
-        float M = sk == -INFINITY ? -INFINITY : sk * kLog2e;
-        for (int sp = 0; sp < n_split; ++sp) M = fmaxf(M, pml[(qi * n_split + sp) * (2 * kH) + h]);
-        float l = 0.f;
-        for (int sp = 0; sp < n_split; ++sp) {
-            const float *ml = pml + (qi * n_split + sp) * (2 * kH);
-            const float wv = M == -INFINITY ? 0.f : exp2f(ml[h] - M);
-            wgt[tid][sp] = wv;
-            l += wv * ml[kH + h];
-        }
-        if (sk != -INFINITY && M != -INFINITY) l += exp2f(sk * kLog2e - M);
-        inv_l[tid] = l > 0.f ? 1.f / l : 0.f;
-    }
-    if (tid >= 32 && tid < 64) {
-        // warp 1, lane p: pair p (n_pairs <= 32 on this path), table read warp-uniformly
-        const int p = tid - 32;
-        uint64_t tv = 0;
-        for (int k = 0; k < rope.n_pairs; ++k) {
-            const uint64_t v = rope.turn[k];
-            if (p == k) tv = v;
-        }
-        if (p < rope.n_pairs) {
-            float cs, sn;
-            rope_cs(-(q_pos0 + qi % S_q), tv, &cs, &sn);
-            rcs[0][p] = cs;
-            rcs[1][p] = sn;
-        }
-    }
-    // thread: channel pair d = 2 * tid of the 8 heads
-    const int d = 2 * tid;
-    float2 v[kMaxSplit][kCombHeads];
-#pragma unroll
-    for (int sp = 0; sp < kMaxSplit; ++sp)
-        if (sp < n_split)
-#pragma unroll
-            for (int hh = 0; hh < kCombHeads; ++hh)
-                v[sp][hh] = *reinterpret_cast<const float2 *>(part + (qi * n_split + sp) * (int64_t)(kH * kD) +
-                                                            (int64_t)(h0 + hh) * kD + d);
-    __syncthreads();
-    float cs = 1.f, sn = 0.f;
-    const bool rot = d >= rope.first;
-    if (rot) {
-        cs = rcs[0][(d - rope.first) >> 1];
-        sn = rcs[1][(d - rope.first) >> 1];
-    }
-#pragma unroll
-    for (int hh = 0; hh < kCombHeads; ++hh) {
-        float a = 0.f, b = 0.f;
-#pragma unroll
-        for (int sp = 0; sp < kMaxSplit; ++sp)
-            if (sp < n_split) {
-                a += wgt[hh][sp] * v[sp][hh].x;
-                b += wgt[hh][sp] * v[sp][hh].y;
-            }
-        a *= inv_l[hh];
-        b *= inv_l[hh];
-        const float ra = rot ? a * cs - b * sn : a, rb = rot ? a * sn + b * cs : b;
-        *reinterpret_cast<__nv_bfloat162 *>(out + (qi * kH + h0 + hh) * (int64_t)kD + d) = __floats2bfloat162_rn(ra, rb);
-    }
 }
 
 }  // namespace
@@ -1052,18 +1042,16 @@ int attend_tc_kmax7(const AttendArgs &a) {
     return (int)(tiles > 0 ? tiles * kTile : kTile);
 }
 
-// Decode-sized calls with few queries split each query's key tiles over two CTAs (the
-// device has 148 SMs) and merge the partials in a second kernel.
+// Decode-sized calls with at most half as many queries as the device has SMs split each
+// query's key tiles over two CTAs, launched as a 2-CTA cluster that merges the two partial
+// results through shared memory.  Every CTA then has exactly one work item, which the
+// pair's handshake relies on.
 static int attend_tc_split(const AttendArgs &a) {
     if (!attend_tc_decode(a)) return 1;
     const int64_t nq = a.B * a.S_q;
-    return (nq * 2 <= 148 && attend_tc_kmax7(a) > kTile) ? 2 : 1;
+    return (nq * 2 <= device_sm_count() && attend_tc_kmax7(a) > kTile) ? 2 : 1;
 }
 
-static size_t split_part_bytes(const AttendArgs &a, int n_split) {
-    if (n_split <= 1) return 0;
-    return (size_t)a.B * a.S_q * n_split * (size_t)(kH * kD + 2 * kH) * sizeof(float);
-}
 
 static size_t round256(size_t v) { return (v + 255) & ~(size_t)255; }
 
@@ -1081,7 +1069,10 @@ static DecodeWs decode_ws(const AttendArgs &a) {
     d.ent = round256(nq * kmax7 * 64 * 2);
     d.cnt = d.ent + round256(nq * kmax7 * 4);
     d.part = d.cnt + round256(nq * 4);
-    d.total = d.part + split_part_bytes(a, attend_tc_split(a));
+    // the second key range's partial of split queries: m, l [nq, 2*64], O^T [nq, 64, 512]
+    // (sized for the split whether or not this device splits: the workspace query has no
+    // device to ask)
+    d.total = d.part + round256(nq * (2 * kH + (size_t)kH * kD) * 4);
     return d;
 }
 static size_t keys_ws_bytes(const AttendArgs &a) {
@@ -1110,12 +1101,12 @@ csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st) {
         kv_src = (const __nv_bfloat16 *)a.kv;
         pool_src = (const __nv_bfloat16 *)a.pool;
         k7 = reinterpret_cast<__nv_bfloat16 *>(ws + d.k7);
+        part = reinterpret_cast<float *>(ws + d.part);
         // CSA with entries to list: the compacted lists and counts (written by pack_k7)
         if (a.mode == 0 && a.topk > 0 && a.P > 0) {
             ent_g = reinterpret_cast<int32_t *>(ws + d.ent);
             n_ent_g = reinterpret_cast<int32_t *>(ws + d.cnt);
         }
-        if (attend_tc_split(a) > 1) part = reinterpret_cast<float *>(ws + d.part);
         if (nq > 0) {
             pack_k7_kernel<<<dim3((unsigned)nq, (unsigned)(kmax7 / kTile)), kK7Threads, 0, st>>>(
                 kv_src, a.S_kv, a.kv_pos0, pool_src, a.P, a.idx, a.mode == 0 ? a.topk : 0, a.mode, a.S_q, a.q_pos0,
@@ -1171,16 +1162,30 @@ csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st) {
     const int n_split = attend_tc_split(a);
     const int64_t nw = nq * n_split;
     const int grid = (int)(nw < sms ? nw : sms);
-    kern<<<grid, kThreads, smem, st>>>(
-        map_q, map_q7, map_kv, map_pool, map_k7, pool_src, a.S_kv, a.kv_pos0, a.P, a.idx, a.mode == 0 ? a.topk : 0,
-        a.mode, a.sink, (__nv_bfloat16 *)a.out, a.B, a.S_q, a.q_pos0, a.window, a.ratio, a.scale, a.rope, kmax7,
-        ent_g, n_ent_g, g_attend_tc_withhold.load(), n_split, part);
-    CSA_CHECK_LAUNCH(a.mode == 0 ? "csa_attend" : "hca_attend");
-    if (n_split > 1) {
-        attend_combine_kernel<<<dim3((unsigned)nq, kH / kCombHeads), kD / 2, 0, st>>>(
-            part, n_split, nq, a.sink, (__nv_bfloat16 *)a.out, a.S_q, a.q_pos0, a.rope);
-        CSA_CHECK_LAUNCH("attend: combine key ranges");
+    // split queries: each pair of CTAs (key ranges 0 and 1 of one query) is a 2-CTA cluster
+    // that merges through shared memory
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    if (n_split == 2) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
     }
+    const cudaError_t le = cudaLaunchKernelEx(
+        &cfg, kern, map_q, map_q7, map_kv, map_pool, map_k7, pool_src, (int64_t)a.S_kv, (int64_t)a.kv_pos0,
+        (int64_t)a.P, a.idx, a.mode == 0 ? a.topk : 0, a.mode, a.sink, (__nv_bfloat16 *)a.out, (int64_t)a.B,
+        (int64_t)a.S_q, (int64_t)a.q_pos0, a.window, a.ratio, a.scale, a.rope, kmax7, (const int32_t *)ent_g,
+        (const int32_t *)n_ent_g, g_attend_tc_withhold.load(), n_split, part);
+    CSA_REQUIRE(le == cudaSuccess, CSA_ERR_CUDA, "%s: launch failed: %s", a.mode == 0 ? "csa_attend" : "hca_attend",
+                cudaGetErrorString(le));
+    CSA_CHECK_LAUNCH(a.mode == 0 ? "csa_attend" : "hca_attend");
     return CSA_OK;
 }
 
