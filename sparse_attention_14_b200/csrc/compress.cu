@@ -11,10 +11,11 @@
 // (8 bf16 or 4+4 fp32 as two vectors), a warp covers 256 contiguous channels of one row,
 // and each thread keeps a running (max, sum of weights, weighted sum) per channel --
 // an online softmax -- so the window is read exactly once, in one pass.
-//  * short windows (up to 8 tokens, e.g. CSA: 2m = 8): one thread per (entry, 8
-//    channels); fp32 loads four tokens at a time into an online softmax, bf16 keeps the
-//    whole window's raw vectors in registers and takes the maximum first (one
-//    exponential per token and channel);
+//  * bf16 with m <= 8 (CSA: m = 4, windows of two blocks of m rows): a thread owns a run
+//    of consecutive entries of one 8-channel group, reduces each block of m rows once to
+//    a partial state and merges neighbouring blocks (compress_run_bf16_kernel);
+//  * other short windows (up to 8 tokens, fp32): one thread per (entry, 8 channels),
+//    loading four tokens at a time into an online softmax;
 //  * longer windows (HCA: 128 tokens): the window is split over `split` thread rows of
 //    one CTA, each row reads every split-th token (so a warp-row reads consecutive rows
 //    of HBM), and the partial softmax states are merged through shared memory.
@@ -95,10 +96,7 @@ __global__ void __launch_bounds__(256) compress_rows_kernel(const T *__restrict_
     store8(pool + (b * P + j) * D + g8 * 8, o);
 }
 
-// bf16, windows of up to 8 tokens (CSA): one thread per (b, j, 8-channel group) with the
-// whole window's raw 16-byte vectors in registers (all 16 loads in flight at once), then
-// two passes: the per-channel maximum, then one exponential per token and channel (the
-// online form above needs two).
+// Eight bf16 of a 16-byte vector as floats.
 __device__ __forceinline__ void unpack8(const uint4 &u, float *v) {
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -108,53 +106,54 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float *v) {
     }
 }
 
-__global__ void __launch_bounds__(256) compress_rows8_bf16_kernel(const __nv_bfloat16 *__restrict__ kv,
-                                                                   const __nv_bfloat16 *__restrict__ gate,
-                                                                   __nv_bfloat16 *__restrict__ pool, int64_t B,
-                                                                   int64_t S, int D, int ratio, int overlap,
-                                                                   int64_t P) {
-    const int groups = D / 8;
-    int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    int64_t total = B * P * groups;
-    if (gid >= total) return;
-    int g8 = (int)(gid % groups);
-    int64_t j = (gid / groups) % P;
-    int64_t b = gid / ((int64_t)groups * P);
-    int64_t lo = overlap ? (j - 1) * ratio : j * ratio;
-    if (lo < 0) lo = 0;
-    const int n = (int)((j + 1) * ratio - lo);   // <= 8
-    const uint4 *kv_p = reinterpret_cast<const uint4 *>(kv + (b * S + lo) * D + g8 * 8);
-    const uint4 *g_p = reinterpret_cast<const uint4 *>(gate + (b * S + lo) * D + g8 * 8);
-    const int stride = D / 8;   // uint4 per row
-    uint4 gr[8], vr[8];
+// bf16, windows of whole blocks of at most 8 rows: entry j pools the blocks j-1 and j
+// (overlap) or block j alone, block i being rows [i*m, (i+1)*m).  A thread owns one
+// 8-channel group and a run of R consecutive entries: it reads each block's rows once,
+// reduces the block to a partial softmax state (max, sum of weights, weighted sum; the
+// maximum taken first, one exponential per row and channel), merges neighbouring blocks
+// into entries.  Every raw row is read once, where a thread per entry reads the
+// overlapping half twice; the loads of a block are issued together, and occupancy (about
+// three 256-thread blocks per SM) covers the latency.
+template <int M>
+struct Block8 {
+    uint4 g[M], v[M];
+};
+template <int M>
+__device__ __forceinline__ void load_block(Block8<M> &blk, const __nv_bfloat16 *kv, const __nv_bfloat16 *gate,
+                                           int64_t row0, int n, int stride) {
+    const uint4 *kp = reinterpret_cast<const uint4 *>(kv) + row0 * stride;
+    const uint4 *gp = reinterpret_cast<const uint4 *>(gate) + row0 * stride;
 #pragma unroll
-    for (int s = 0; s < 8; ++s) {
+    for (int s = 0; s < M; ++s) {
         if (s < n) {
-            gr[s] = __ldg(g_p + (int64_t)s * stride);
-            vr[s] = __ldg(kv_p + (int64_t)s * stride);
+            blk.g[s] = __ldg(gp + (int64_t)s * stride);
+            blk.v[s] = __ldg(kp + (int64_t)s * stride);
         }
     }
-    float mx[8];
+}
+template <int M>
+__device__ __forceinline__ void reduce_block(const Block8<M> &blk, int n, float *mx, float *den, float *num) {
 #pragma unroll
-    for (int c = 0; c < 8; ++c) mx[c] = -INFINITY;
+    for (int c = 0; c < 8; ++c) {
+        mx[c] = -INFINITY;
+        den[c] = 0.f;
+        num[c] = 0.f;
+    }
 #pragma unroll
-    for (int s = 0; s < 8; ++s) {
+    for (int s = 0; s < M; ++s) {
         if (s < n) {
             float gv[8];
-            unpack8(gr[s], gv);
+            unpack8(blk.g[s], gv);
 #pragma unroll
             for (int c = 0; c < 8; ++c) mx[c] = fmaxf(mx[c], gv[c]);
         }
     }
-    float den[8], num[8];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) den[c] = num[c] = 0.f;
-#pragma unroll
-    for (int s = 0; s < 8; ++s) {
+    for (int s = 0; s < M; ++s) {
         if (s < n) {
             float gv[8], vv[8];
-            unpack8(gr[s], gv);
-            unpack8(vr[s], vv);
+            unpack8(blk.g[s], gv);
+            unpack8(blk.v[s], vv);
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 const float e = __expf(gv[c] - mx[c]);
@@ -163,10 +162,62 @@ __global__ void __launch_bounds__(256) compress_rows8_bf16_kernel(const __nv_bfl
             }
         }
     }
-    float o[8];
+}
+
+template <int M>
+__global__ void __launch_bounds__(256) compress_run_bf16_kernel(const __nv_bfloat16 *__restrict__ kv,
+                                                                 const __nv_bfloat16 *__restrict__ gate,
+                                                                 __nv_bfloat16 *__restrict__ pool, int64_t B,
+                                                                 int64_t S, int D, int ratio, int overlap,
+                                                                 int64_t P, int R) {
+    const int groups = D / 8;
+    const int64_t runs = (P + R - 1) / R;
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= B * runs * groups) return;
+    const int g8 = (int)(gid % groups);
+    const int64_t run = (gid / groups) % runs;
+    const int64_t b = gid / ((int64_t)groups * runs);
+    const int64_t j0 = run * R;
+    const int64_t j1 = j0 + R < P ? j0 + R : P;
+    const __nv_bfloat16 *kvb = kv + b * S * D + g8 * 8, *gb = gate + b * S * D + g8 * 8;
+    const int stride = D / 8;
+    // block i: rows [i*ratio, i*ratio + ratio); only whole blocks below S are pooled
+    float pmx[8], pden[8], pnum[8];   // state of the previous block (overlap)
 #pragma unroll
-    for (int c = 0; c < 8; ++c) o[c] = num[c] / den[c];
-    store8(pool + (b * P + j) * D + g8 * 8, o);
+    for (int c = 0; c < 8; ++c) {
+        pmx[c] = -INFINITY;
+        pden[c] = 0.f;
+        pnum[c] = 0.f;
+    }
+    int64_t i = overlap ? j0 - 1 : j0;   // first block to read
+    if (i < 0) i = 0;
+    for (; i < j1; ++i) {
+        Block8<M> cur;
+        load_block<M>(cur, kvb, gb, i * ratio, ratio, stride);
+        float mx[8], den[8], num[8];
+        reduce_block<M>(cur, ratio, mx, den, num);
+        if (i >= j0) {
+            float o[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                float m = mx[c], d = den[c], nu = num[c];
+                if (overlap && pmx[c] != -INFINITY) {
+                    const float mm = fmaxf(m, pmx[c]);
+                    const float a = __expf(m - mm), bb = __expf(pmx[c] - mm);
+                    d = d * a + pden[c] * bb;
+                    nu = nu * a + pnum[c] * bb;
+                }
+                o[c] = nu / d;
+            }
+            store8(pool + (b * P + i) * D + g8 * 8, o);
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            pmx[c] = mx[c];
+            pden[c] = den[c];
+            pnum[c] = num[c];
+        }
+    }
 }
 
 // CTA per (entry j, batch b, channel block); threadIdx.x = 8-channel group within the
@@ -225,15 +276,28 @@ template <typename T>
 csa_status_t launch_compress(const T *kv, const T *gate, T *pool, int64_t B, int64_t S, int D,
                              int ratio, int overlap, int64_t P, cudaStream_t st) {
     const int64_t win = overlap ? 2 * (int64_t)ratio : ratio;
-    if (win <= 8) {
+    if (sizeof(T) == 2 && ratio <= 8) {
+        // runs of R entries per thread, R chosen so that the grid still fills the device
+        // (about 512 threads per SM)
+        const int64_t per = B * (int64_t)(D / 8);
+        int64_t R = per * P / ((int64_t)device_sm_count() * 512);
+        R = R < 1 ? 1 : (R > 16 ? 16 : R);
+        const int64_t total = per * ((P + R - 1) / R);
+        const int64_t blocks = ceil_div(total, 256);
+        CSA_REQUIRE(blocks < (1ll << 31), CSA_ERR_UNSUPPORTED, "csa_compress: too many entries");
+        if (ratio <= 4)
+            compress_run_bf16_kernel<4><<<(unsigned)blocks, 256, 0, st>>>(
+                (const __nv_bfloat16 *)kv, (const __nv_bfloat16 *)gate, (__nv_bfloat16 *)pool, B, S, D, ratio,
+                overlap, P, (int)R);
+        else
+            compress_run_bf16_kernel<8><<<(unsigned)blocks, 256, 0, st>>>(
+                (const __nv_bfloat16 *)kv, (const __nv_bfloat16 *)gate, (__nv_bfloat16 *)pool, B, S, D, ratio,
+                overlap, P, (int)R);
+    } else if (win <= 8) {
         int64_t total = B * P * (D / 8);
         int64_t blocks = ceil_div(total, 256);
         CSA_REQUIRE(blocks < (1ll << 31), CSA_ERR_UNSUPPORTED, "csa_compress: too many entries");
-        if constexpr (sizeof(T) == 2)
-            compress_rows8_bf16_kernel<<<(unsigned)blocks, 256, 0, st>>>(kv, gate, pool, B, S, D, ratio, overlap, P);
-        else
-            compress_rows_kernel<T, 8><<<(unsigned)blocks, 256, 0, st>>>(kv, gate, pool, B, S, D, ratio,
-                                                                         overlap, P);
+        compress_rows_kernel<T, 8><<<(unsigned)blocks, 256, 0, st>>>(kv, gate, pool, B, S, D, ratio, overlap, P);
     } else {
         int split = 8;
         while (split > 1 && win / split < 4) split /= 2;

@@ -11,44 +11,122 @@
 // indexer queries q_I [B,S_q,H_I,d_I] (group H_I, period S_q, step 1, pos0 = q_pos0) and
 // the pooled index keys k_I [B,P,d_I] (group 1, period P, step ratio, pos0 0).
 //
-// The pass is HBM-bound: every row is read and written once.  A thread owns one 16-byte
-// vector (8 bf16, or 8 fp32 as two vectors); since D - R is even and a multiple-of-8
-// vector never splits a pair, each thread rotates its own pairs.
+// The pass is HBM-bound: every row is read and written once (in place, only the vectors
+// holding rope channels).  A thread works on 16-byte-aligned vectors of 8 elements (8
+// bf16, or 8 fp32 as two loads); since D - R is even and a vector never splits a pair,
+// each thread rotates its own pairs.
 #include "common.cuh"
 
 namespace csa {
 namespace {
 
+constexpr int kRopeThreads = 256, kRopeUnroll = 4;
+
+// Persistent grid: the table's turns are staged in shared memory once per block, and
+// every thread keeps kRopeUnroll 16-byte loads in flight.  In place (out == x), only the
+// vectors holding rope channels are touched (the others already hold their output).
+// For bf16, when the touched vectors per row (np) divide the block, a thread keeps one
+// vector column and steps over rows, so that the index and position arithmetic is per
+// row and in 32 bits (64-bit divisions per element made this pass instruction-bound).
 template <typename T>
-__global__ void __launch_bounds__(256) rope_any_kernel(const T *x, T *out, int64_t rows, int D,
-                                                       int64_t pos0, int64_t group,
-                                                       int64_t period, int64_t step,
-                                                       RopeTable rope) {
+__global__ void __launch_bounds__(kRopeThreads, 4) rope_any_kernel(const T *x, T *out, int64_t rows, int D,
+                                                                int64_t pos0, int64_t group, int64_t period,
+                                                                int64_t step, RopeTable rope, int inplace) {
     __shared__ uint64_t turn_s[kMaxRopePairs];
-    stage_turns(rope, turn_s, threadIdx.x, blockDim.x);
+    stage_turns(rope, turn_s, threadIdx.x, kRopeThreads);
     __syncthreads();
     const int pieces = D / 8;
-    const int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (v >= rows * pieces) return;
-    const int64_t r = v / pieces;
-    const int d0 = (int)(v % pieces) * 8;
-    float a[8];
-    load8(x + r * D + d0, a);
-    if (d0 + 8 > rope.first) {
-        const int64_t pos = pos0 + ((r / group) % period) * step;
+    const int p0 = inplace ? rope.first / 8 : 0;   // first vector of a row this pass touches
+    const int np = pieces - p0;                    // vectors per row it touches
+    auto rotate = [&](float *a, int64_t r, int d0) {
+        if (d0 + 8 > rope.first) {
+            const int64_t pos = pos0 + ((r / group) % period) * step;
 #pragma unroll
-        for (int c = 0; c < 8; c += 2) {
-            const int d = d0 + c;
-            if (d >= rope.first) {
-                float cs, sn;
-                rope_cs(pos, turn_s[(d - rope.first) >> 1], &cs, &sn);
-                const float u = a[c], w = a[c + 1];
-                a[c] = u * cs - w * sn;
-                a[c + 1] = u * sn + w * cs;
+            for (int c = 0; c < 8; c += 2) {
+                const int d = d0 + c;
+                if (d >= rope.first) {
+                    float cs, sn;
+                    rope_cs(pos, turn_s[(d - rope.first) >> 1], &cs, &sn);
+                    const float w0 = a[c], w1 = a[c + 1];
+                    a[c] = w0 * cs - w1 * sn;
+                    a[c + 1] = w0 * sn + w1 * cs;
+                }
             }
         }
+    };
+    if (sizeof(T) == 2 && kRopeThreads % np == 0 && rows < ((int64_t)1 << 31) && group < ((int64_t)1 << 31)) {
+        // bf16: thread = vector column p0 + tid % np, rows tid / np + k * (rows per grid
+        // step); the vectors stay raw 16-byte words (4 registers each) so that twice as
+        // many loads fit in flight, and only rope vectors are widened to float
+        constexpr int U = 2 * kRopeUnroll;
+        const int d0 = (p0 + (int)(threadIdx.x % (unsigned)np)) * 8;
+        const bool rot = d0 + 8 > rope.first;
+        const uint32_t rpb = kRopeThreads / np;                       // rows per block step
+        const uint32_t rstep = rpb * gridDim.x;                       // rows per grid step
+        const uint32_t g32 = (uint32_t)group, per32 = (uint32_t)period;
+        const uint4 *xv = reinterpret_cast<const uint4 *>(x);
+        uint4 *ov = reinterpret_cast<uint4 *>(out);
+        const int64_t vrow = D / 8;                                   // 16-byte vectors per row
+        for (uint32_t r0 = blockIdx.x * rpb + threadIdx.x / (unsigned)np; r0 < (uint64_t)rows; r0 += rstep * U) {
+            uint4 w[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const uint64_t r = (uint64_t)r0 + (uint64_t)u * rstep;
+                if (r < (uint64_t)rows) w[u] = xv[(int64_t)r * vrow + d0 / 8];
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const uint64_t r = (uint64_t)r0 + (uint64_t)u * rstep;
+                if (r >= (uint64_t)rows) continue;
+                if (rot) {
+                    float a[8];
+                    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&w[u]);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const float2 f = __bfloat1622float2(h[c]);
+                        a[2 * c] = f.x;
+                        a[2 * c + 1] = f.y;
+                    }
+                    const int64_t pos = pos0 + (int64_t)(((uint32_t)r / g32) % per32) * step;
+#pragma unroll
+                    for (int c = 0; c < 8; c += 2) {
+                        const int d = d0 + c;
+                        if (d >= rope.first) {
+                            float cs, sn;
+                            rope_cs(pos, turn_s[(d - rope.first) >> 1], &cs, &sn);
+                            const float w0 = a[c], w1 = a[c + 1];
+                            a[c] = w0 * cs - w1 * sn;
+                            a[c + 1] = w0 * sn + w1 * cs;
+                        }
+                    }
+                    __nv_bfloat162 *o2 = reinterpret_cast<__nv_bfloat162 *>(&w[u]);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) o2[c] = __floats2bfloat162_rn(a[2 * c], a[2 * c + 1]);
+                }
+                ov[(int64_t)r * vrow + d0 / 8] = w[u];
+            }
+        }
+        return;
     }
-    store8(out + r * D + d0, a);
+    const int64_t total = rows * np;
+    const int64_t stride = (int64_t)gridDim.x * kRopeThreads;
+    for (int64_t v0 = (int64_t)blockIdx.x * kRopeThreads + threadIdx.x; v0 < total; v0 += stride * kRopeUnroll) {
+        float a[kRopeUnroll][8];
+#pragma unroll
+        for (int u = 0; u < kRopeUnroll; ++u) {
+            const int64_t v = v0 + u * stride;
+            if (v < total) load8(x + (v / np) * D + (p0 + (int)(v % np)) * 8, a[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < kRopeUnroll; ++u) {
+            const int64_t v = v0 + u * stride;
+            if (v >= total) continue;
+            const int64_t r = v / np;
+            const int d0 = (p0 + (int)(v % np)) * 8;
+            rotate(a[u], r, d0);
+            store8(out + r * D + d0, a[u]);
+        }
+    }
 }
 
 }  // namespace
@@ -82,17 +160,21 @@ extern "C" csa_status_t csa_rope_rows(const void *x, void *out, int64_t rows, in
     const uintptr_t xa = (uintptr_t)x, oa = (uintptr_t)out, n = (uintptr_t)(rows * D * e);
     CSA_REQUIRE(xa == oa || xa + n <= oa || oa + n <= xa, CSA_ERR_INVALID_ARG,
                 "csa_rope_rows: out must be x itself or not overlap it");
-    const int64_t blocks = ceil_div(rows * (D / 8), 256);
-    CSA_REQUIRE(blocks < ((int64_t)1 << 31), CSA_ERR_UNSUPPORTED, "csa_rope_rows: too many rows");
+    const int inplace = xa == oa ? 1 : 0;
     RopeTable rope;
     make_rope_table(&rope, D, rope_dim, rope_base);
+    if (inplace && rope_dim == 0) return CSA_OK;   // nothing to rotate, nothing to copy
+    const int64_t np = D / 8 - (inplace ? rope.first / 8 : 0);
+    const int64_t want = ceil_div(rows * np, (int64_t)kRopeThreads * kRopeUnroll);
+    const int64_t cap = (int64_t)device_sm_count() * 8;
+    const int64_t blocks = want < cap ? want : cap;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (dtype == CSA_F32)
-        rope_any_kernel<float><<<(unsigned)blocks, 256, 0, st>>>((const float *)x, (float *)out, rows,
-                                                                 D, pos0, group, period, step, rope);
+        rope_any_kernel<float><<<(unsigned)blocks, kRopeThreads, 0, st>>>(
+            (const float *)x, (float *)out, rows, D, pos0, group, period, step, rope, inplace);
     else
-        rope_any_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(
-            (const __nv_bfloat16 *)x, (__nv_bfloat16 *)out, rows, D, pos0, group, period, step, rope);
+        rope_any_kernel<__nv_bfloat16><<<(unsigned)blocks, kRopeThreads, 0, st>>>(
+            (const __nv_bfloat16 *)x, (__nv_bfloat16 *)out, rows, D, pos0, group, period, step, rope, inplace);
     CSA_CHECK_LAUNCH("csa_rope_rows");
     return CSA_OK;
 }
