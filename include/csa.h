@@ -155,8 +155,10 @@ csa_status_t csa_rope_rows(const void *x, void *out, int64_t rows, int32_t D, in
                            double rope_base, int64_t pos0, int64_t group, int64_t period,
                            int64_t step, csa_dtype_t dtype, void *stream);
 
-/* Scratch bytes csa_index_topk needs for these sizes (0 when the call needs none; a
- * decode-sized call is split over entry ranges and merges through the workspace). */
+/* Scratch bytes csa_index_topk needs for these sizes (0 when the call needs none).  A
+ * decode-sized call is split over entry ranges: rows with at most 16384 visible entries
+ * pass every entry's 64-bit key through the workspace to a selection kernel, longer rows
+ * pass each range's candidates to a merge kernel. */
 size_t csa_index_topk_workspace_bytes(int64_t B, int64_t S_q, int64_t q_pos0, int64_t P,
                                       int32_t H_I, int32_t d_I, int32_t ratio, int32_t topk,
                                       csa_dtype_t dtype);
@@ -186,6 +188,9 @@ size_t csa_index_topk_workspace_bytes(int64_t B, int64_t S_q, int64_t q_pos0, in
  *   out : [B, S_q, H, D] output
  *   workspace : device scratch of at least csa_attend_workspace_bytes(...) bytes.
  *   Requires q_pos0 >= 0 when S_q > 0 and window >= 1.
+ * The tensor-core path (bf16, H = 64, D = 512, rope_dim <= 64) reads kv and pool in place
+ * for decode-sized calls (S_q * 64 < S_kv + P); these take it when both pointers are
+ * 16-byte aligned, and the general path otherwise.
  */
 csa_status_t csa_attend(const void *q, const void *kv, int64_t S_kv, int64_t kv_pos0,
                         const void *pool, int64_t P, const int32_t *idx, int32_t topk,
