@@ -210,6 +210,8 @@ __global__ void __launch_bounds__(kK7Threads) pack_k7_kernel(
     const int64_t qi = blockIdx.x;
     const int kt = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
+    grid_wait();   // idx from the indexer
+    grid_launch_dependents();
     if (kt == 0 && tid < kRopeQThreads) rotate_q_chunk_part(q, q7, qi, S_q, q_pos0, rope, tid, cs_s, sn_s);
     const int64_t b = qi / S_q, t = q_pos0 + qi % S_q;
     const int64_t nv = n_visible(t, ratio, P);
@@ -452,6 +454,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     const bool pair = kK7 && n_split == 2;
     if (pair) cluster_sync_all();
     const uint32_t tmem = sm.tmem_base;
+    // set-up done: wait for the preceding kernel's results, then let the next one start
+    grid_wait();
+    grid_launch_dependents();
 
     if (warp == 0 || warp == 10) {
         // ===================================================== loaders
@@ -1108,9 +1113,13 @@ csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st) {
             n_ent_g = reinterpret_cast<int32_t *>(ws + d.cnt);
         }
         if (nq > 0) {
-            pack_k7_kernel<<<dim3((unsigned)nq, (unsigned)(kmax7 / kTile)), kK7Threads, 0, st>>>(
-                kv_src, a.S_kv, a.kv_pos0, pool_src, a.P, a.idx, a.mode == 0 ? a.topk : 0, a.mode, a.S_q, a.q_pos0,
-                a.window, a.ratio, a.rope, kmax7, k7, (const __nv_bfloat16 *)a.q, q7, ent_g, n_ent_g);
+            const cudaError_t le = launch_dependent(
+                pack_k7_kernel, dim3((unsigned)nq, (unsigned)(kmax7 / kTile)), dim3(kK7Threads), 0, st, 1, kv_src,
+                (int64_t)a.S_kv, (int64_t)a.kv_pos0, pool_src, (int64_t)a.P, a.idx, a.mode == 0 ? a.topk : 0, a.mode,
+                (int64_t)a.S_q, (int64_t)a.q_pos0, a.window, a.ratio, a.rope, kmax7, k7, (const __nv_bfloat16 *)a.q,
+                q7, ent_g, n_ent_g);
+            CSA_REQUIRE(le == cudaSuccess, CSA_ERR_CUDA, "attend: rope-chunk packing launch failed: %s",
+                        cudaGetErrorString(le));
             CSA_CHECK_LAUNCH("attend: rotate the keys' rope chunks");
         }
     } else {
@@ -1163,24 +1172,10 @@ csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st) {
     const int64_t nw = nq * n_split;
     const int grid = (int)(nw < sms ? nw : sms);
     // split queries: each pair of CTAs (key ranges 0 and 1 of one query) is a 2-CTA cluster
-    // that merges through shared memory
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    if (n_split == 2) {
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-    }
-    const cudaError_t le = cudaLaunchKernelEx(
-        &cfg, kern, map_q, map_q7, map_kv, map_pool, map_k7, pool_src, (int64_t)a.S_kv, (int64_t)a.kv_pos0,
-        (int64_t)a.P, a.idx, a.mode == 0 ? a.topk : 0, a.mode, a.sink, (__nv_bfloat16 *)a.out, (int64_t)a.B,
+    // that merges in-kernel
+    const cudaError_t le = launch_dependent(
+        kern, dim3((unsigned)grid), dim3(kThreads), smem, st, n_split == 2 ? 2 : 1, map_q, map_q7, map_kv, map_pool,
+        map_k7, pool_src, (int64_t)a.S_kv, (int64_t)a.kv_pos0, (int64_t)a.P, a.idx, a.mode == 0 ? a.topk : 0, a.mode, a.sink, (__nv_bfloat16 *)a.out, (int64_t)a.B,
         (int64_t)a.S_q, (int64_t)a.q_pos0, a.window, a.ratio, a.scale, a.rope, kmax7, (const int32_t *)ent_g,
         (const int32_t *)n_ent_g, g_attend_tc_withhold.load(), n_split, part);
     CSA_REQUIRE(le == cudaSuccess, CSA_ERR_CUDA, "%s: launch failed: %s", a.mode == 0 ? "csa_attend" : "hca_attend",

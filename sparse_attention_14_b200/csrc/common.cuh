@@ -5,6 +5,8 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+
+#include <utility>
 #include <math.h>
 #include <stdint.h>
 #include <stdio.h>
@@ -37,6 +39,43 @@ void count_launches(int n);  // kernels enqueued by this library (csa_launch_cou
     } while (0)
 
 inline bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// ---------------------------------------------------------------- dependent launch
+// Kernels of a chain (the decode step: indexer, selection, key packing, attention) are
+// launched with programmatic stream serialization: a kernel may start while its
+// predecessor finishes, runs its set-up (barriers, tensor memory, descriptor prefetch)
+// that touches no global memory, then waits for the predecessor's completion and memory
+// (grid_wait) before its first global access.  Once every CTA of a kernel has called
+// grid_launch_dependents (after its own set-up and wait), its successor may be scheduled.
+// Without the launch attribute both are no-ops.
+__device__ __forceinline__ void grid_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Launch with programmatic stream serialization (and optionally a 1-D cluster).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             int cluster_x, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (cluster_x > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = (unsigned)cluster_x;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // ---------------------------------------------------------------- element access
 template <typename T> struct Elem;

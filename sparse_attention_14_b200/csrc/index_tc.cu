@@ -371,6 +371,9 @@ __global__ void __launch_bounds__(Cfg<QB>::kThreads, Cfg<QB>::kMinBlocks) index_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ms.tmem_base;
+    // set-up done: wait for the preceding kernel's results, then let the next one start
+    grid_wait();
+    grid_launch_dependents();
     const uint32_t sB = base + C::kOffB, sA = base + C::kOffA;
 
     if (warp == 0) {
@@ -588,6 +591,8 @@ __global__ void __launch_bounds__(kSelThreads) index_select_kernel(
     __shared__ unsigned long long sel_T;
     const int64_t row = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    grid_wait();   // the indexer's keys
+    grid_launch_dependents();
     const int n = (int)n_visible(q_pos0 + row % S_q, ratio, P);   // <= kSelMax (host check)
     const unsigned long long *kr = keys + row * P;
     int32_t *idx_row = idx + row * (int64_t)topk;
@@ -780,8 +785,10 @@ csa_status_t launch(const CUtensorMap &mk, const CUtensorMap &mq, const __nv_bfl
     CSA_REQUIRE(grid < (1ll << 31), CSA_ERR_UNSUPPORTED, "csa_index_topk: grid too large");
     auto kern = index_tc_kernel<QB>;
     ensure_smem((const void *)kern, C::kSmem);
-    kern<<<(unsigned)grid, C::kThreads, C::kSmem, st>>>(mk, mq, w, B, S_q, q_pos0, P, ratio, topk, n_split,
-                                                        idx, scores_opt, partial, keys_out);
+    const cudaError_t le = launch_dependent(kern, dim3((unsigned)grid), dim3(C::kThreads), C::kSmem, st, 1, mk, mq, w,
+                                            B, S_q, q_pos0, P, ratio, topk, n_split, idx, scores_opt, partial,
+                                            keys_out);
+    CSA_REQUIRE(le == cudaSuccess, CSA_ERR_CUDA, "csa_index_topk: launch failed: %s", cudaGetErrorString(le));
     CSA_CHECK_LAUNCH("csa_index_topk");
     return CSA_OK;
 }
@@ -835,8 +842,11 @@ csa_status_t index_tc(const void *qI, const void *w, const void *kI, int64_t B, 
     if (r != CSA_OK || p.n_split <= 1) return r;
     if (p.keys) {
         ensure_smem((const void *)index_select_kernel, kSelSmem);
-        index_select_kernel<<<(unsigned)(B * S_q), kSelThreads, kSelSmem, st>>>(keys, P, topk, idx, scores_opt,
-                                                                               S_q, q_pos0, ratio);
+        const cudaError_t le = launch_dependent(index_select_kernel, dim3((unsigned)(B * S_q)), dim3(kSelThreads),
+                                                kSelSmem, st, 1, (const unsigned long long *)keys, P, topk, idx,
+                                                scores_opt, S_q, q_pos0, ratio);
+        CSA_REQUIRE(le == cudaSuccess, CSA_ERR_CUDA, "csa_index_topk select: launch failed: %s",
+                    cudaGetErrorString(le));
         CSA_CHECK_LAUNCH("csa_index_topk select");
         return CSA_OK;
     }
