@@ -522,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                         if (e < n_ent) ent[e] = v[k];
                     }
                 }
-            } else if (mode == 0) {
+            } else if (!kK7 && mode == 0) {
                 // compact the valid idx values in slot order; eight loads per lane in flight
                 int cnt = 0;
                 const int32_t *ip = idx + qi * topk;
@@ -870,7 +870,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 if (!ok) break;
                 tc_fence_after();
                 float *pm = part + qi * (int64_t)(2 * kH);                 // m[64], l[64]
-                float *po = part + B * S_q * (2 * kH) + qi * (int64_t)(kH * kD);
+                // O^T of the second range as float4 [mt][h4][st] (heads 4*h4 .. 4*h4+3 of
+                // thread st): each side moves its 32 values per slice with 8 vector accesses,
+                // and each warp access covers 512 contiguous bytes
+                float4 *po = reinterpret_cast<float4 *>(part + B * S_q * (2 * kH) + qi * (int64_t)(kH * kD));
                 if ((w % 2) == 1) {
                     if (st < kH) {
                         pm[st] = sm.m_used[st];
@@ -887,7 +890,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                             for (int h = 0; h < 32; ++h) o[h] = 0.f;
                         }
 #pragma unroll
-                        for (int h = 0; h < 32; ++h) po[(int64_t)(hb + h) * kD + mt * 128 + x] = o[h];
+                        for (int h4 = 0; h4 < 8; ++h4)
+                            po[(mt * 8 + h4) * kSoftThreads + st] =
+                                make_float4(o[4 * h4], o[4 * h4 + 1], o[4 * h4 + 2], o[4 * h4 + 3]);
                     }
                     tc_fence_before();
                     // every thread releases its own writes with its arrival (count kSoftThreads)
@@ -914,12 +919,25 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 }
                 named_sync(1, kSoftThreads);
                 __nv_bfloat16 *orow = out + qi * (int64_t)kH * kD;
+                float4 o1v[2][8];   // the peer's values of two slices in flight together
 #pragma unroll 1
                 for (int mt = 0; mt < 4; ++mt) {
                     const int d = mt * 128 + x;
+                    if ((mt & 1) == 0) {
+#pragma unroll
+                        for (int u = 0; u < 2; ++u)
+#pragma unroll
+                            for (int h4 = 0; h4 < 8; ++h4) o1v[u][h4] = __ldcg(po + ((mt + u) * 8 + h4) * kSoftThreads + st);
+                    }
                     float o1[32];
 #pragma unroll
-                    for (int h = 0; h < 32; ++h) o1[h] = __ldcg(po + (int64_t)(hb + h) * kD + d);
+                    for (int h4 = 0; h4 < 8; ++h4) {
+                        const float4 v = (mt & 1) ? o1v[1][h4] : o1v[0][h4];
+                        o1[4 * h4] = v.x;
+                        o1[4 * h4 + 1] = v.y;
+                        o1[4 * h4 + 2] = v.z;
+                        o1[4 * h4 + 3] = v.w;
+                    }
                     float cs = 1.f, sn = 0.f;
                     const bool rot = d >= rope.first;
                     if (rot) rope_cs(-qg.t, rope.turn[(d - rope.first) >> 1], &cs, &sn);

@@ -94,6 +94,15 @@ MID = [
     LayerSpec(name="p0_csa_window_bf16", dtype="bf16", B=1, S_q=300, S_kv=300, q_pos0=0,
               kv_pos0=0, H=64, D=512, R=64, base=160000.0, W=300, m=4, P=0, kind="csa", H_I=64,
               d_I=128, topk=32, decode=True, workload=78),
+    # decode-sized calls at an early position: no entry is visible yet, so the query has a
+    # single (window) key tile and the second CTA of its split pair has none (an empty
+    # partial merged by the first); CSA and HCA
+    LayerSpec(name="early_decode_csa_bf16", dtype="bf16", B=3, S_q=1, S_kv=3, q_pos0=2,
+              kv_pos0=0, H=64, D=512, R=64, base=160000.0, W=128, m=4, P=100, kind="csa",
+              H_I=64, d_I=128, topk=64, decode=True, workload=77),
+    LayerSpec(name="early_decode_hca_bf16", dtype="bf16", B=2, S_q=1, S_kv=100, q_pos0=99,
+              kv_pos0=0, H=64, D=512, R=64, base=160000.0, W=128, m=128, P=4, kind="hca",
+              decode=True, workload=76),
     # odd shapes: general path
     LayerSpec(name="odd_csa_bf16", dtype="bf16", B=1, S_q=77, S_kv=77, q_pos0=0, kv_pos0=0, H=5,
               D=40, R=8, base=10000.0, W=9, m=3, P=25, kind="csa", H_I=3, d_I=24, topk=7,
