@@ -41,6 +41,7 @@
 //    first merges them (sink, division, de-rotation) and stores the output.
 #include <atomic>
 #include <mutex>
+#include <vector>
 
 #include "attend.cuh"
 #include "umma.cuh"
@@ -90,6 +91,15 @@ struct Small {
     float alpha[kH];
     float red[4][kH];
     float inv_l[kH];
+};
+
+// Prefill: CTA c takes the contiguous work items [start[c], start[c+1]), split so that each
+// CTA gets about the same number of key tiles.  Consecutive queries then run on one CTA
+// (their windows overlap in all but one row and their selected entries largely coincide,
+// which L2 serves).  start[0] < 0: work items strided over the grid (decode-sized calls).
+constexpr int kMaxCtas = 160;
+struct CtaRanges {
+    int32_t start[kMaxCtas + 1];
 };
 
 __host__ __device__ __forceinline__ size_t tc_ent_bytes(int topk) {
@@ -405,7 +415,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     const int32_t *__restrict__ idx, int topk, int mode, const float *__restrict__ sink,
     __nv_bfloat16 *__restrict__ out, int64_t B, int64_t S_q, int64_t q_pos0, int window, int ratio,
     float scale, RopeTable rope, int kmax7, const int32_t *__restrict__ ent_g,
-    const int32_t *__restrict__ n_ent_g, int withhold, int n_split, float *__restrict__ part) {
+    const int32_t *__restrict__ n_ent_g, int withhold, int n_split, float *__restrict__ part,
+    const __grid_constant__ CtaRanges ranges) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     unsigned char *smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -419,6 +430,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     // work item w = query w / n_split, key-tile range w % n_split of it (n_split > 1 only for
     // decode-sized calls, whose partial results the combine kernel merges)
     const int64_t nw = B * S_q * n_split;
+    // this CTA's work items: w_lo, w_lo + w_step, ... < w_hi
+    const bool ranged = !kK7 && ranges.start[0] >= 0;
+    const int64_t w_lo = ranged ? ranges.start[blockIdx.x] : blockIdx.x;
+    const int64_t w_hi = ranged ? ranges.start[blockIdx.x + 1] : nw;
+    const int w_step = ranged ? 1 : (int)gridDim.x;
 
     if (kK7 && tid == 32) {
         // decode-sized calls (one work item per CTA): fetch the tensor-map descriptors while
@@ -467,9 +483,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         int32_t *ent = reinterpret_cast<int32_t *>(smem + kOffEnt + li * ent_bytes);
         uint32_t g = 0, qc = 0;
         int q_pending = -1;   // work item of the last Q TMA issued (its phase completes when it lands)
-        for (int64_t w = blockIdx.x; w < nw && !sm.abort_ && !withhold; w += gridDim.x, ++qc) {
+        for (int64_t w = w_lo; w < w_hi && !sm.abort_ && !withhold; w += w_step, ++qc) {
             const int64_t qi = w / n_split;
-            const int64_t qn = (w + gridDim.x) / n_split;   // query of the next work item
+            const int64_t qn = (w + w_step) / n_split;   // query of the next work item
             const QueryGeom qg = query_geom(qi, S_q, q_pos0, kv_pos0, S_kv, window);
             const int64_t nv = n_visible(qg.t, ratio, P);
             // Q of this query (its rope channels already rotated by rope_q_chunk_kernel): start
@@ -487,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                     tma_load_2d(s_q + (uint32_t)c * 8192u, &map_q, 64 * c, (int)(qi * kH), &sm.q_tma);
                 tma_load_2d(s_q + 7u * 8192u, &map_q7, 0, (int)(qi * kH), &sm.q_tma);
                 // bring the next query's Q into L2 while this query runs
-                if (w + gridDim.x < nw) {
+                if (w + w_step < w_hi) {
                     for (int c = 0; c < 7; ++c)
                         asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
                                          reinterpret_cast<uint64_t>(&map_q)),
@@ -543,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 }
                 n_ent = cnt;
                 // warm L2 with the next query's idx row
-                if (w + gridDim.x < nw) {
+                if (w + w_step < w_hi) {
                     const char *np = reinterpret_cast<const char *>(idx + qn * topk);
                     for (int off = lane * 128; off < topk * 4; off += 32 * 128)
                         asm volatile("prefetch.global.L2 [%0];" ::"l"(np + off));
@@ -697,7 +713,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             const uint32_t hi = (uint32_t)(d_kv >> 32);   // SBO 1024, version, swizzle: shared
             uint32_t g = 0, qc = 0;
             bool ok = true;
-            for (int64_t w = blockIdx.x; ok && w < nw; w += gridDim.x, ++qc) {
+            for (int64_t w = w_lo; ok && w < w_hi; w += w_step, ++qc) {
                 const QueryGeom qg = query_geom(w / n_split, S_q, q_pos0, kv_pos0, S_kv, window);
                 ok = mbar_wait(&sm.meta_full[qc & 1], (qc >> 1) & 1u, kWaitIter);
                 if (!ok) break;
@@ -759,7 +775,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         const float c2 = scale * kLog2e;
         uint32_t g = 0, qc = 0;
         bool ok = true;
-        for (int64_t w = blockIdx.x; ok && w < nw; w += gridDim.x, ++qc) {
+        for (int64_t w = w_lo; ok && w < w_hi; w += w_step, ++qc) {
             const int64_t qi = w / n_split;
             const QueryGeom qg = query_geom(qi, S_q, q_pos0, kv_pos0, S_kv, window);
             // every exit after a wait that ran out is decided together (vote at the named
@@ -1188,14 +1204,40 @@ csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st) {
     const int sms = device_sm_count();
     const int n_split = attend_tc_split(a);
     const int64_t nw = nq * n_split;
-    const int grid = (int)(nw < sms ? nw : sms);
+    int grid = (int)(nw < sms ? nw : sms);
+    if (grid > kMaxCtas) grid = kMaxCtas;
+    CtaRanges ranges;
+    ranges.start[0] = -1;
+    if (!decode && nw > grid) {
+        // key tiles per query with the kernel's geometry (every idx value assumed valid)
+        std::vector<int64_t> pre((size_t)a.S_q + 1, 0);
+        for (int64_t i = 0; i < a.S_q; ++i) {
+            const int64_t t = a.q_pos0 + i;
+            int64_t lo = t - a.window + 1;
+            if (lo < a.kv_pos0) lo = a.kv_pos0;
+            const int64_t hi = t < a.kv_pos0 + a.S_kv - 1 ? t : a.kv_pos0 + a.S_kv - 1;
+            const int64_t n_win = hi >= lo ? hi - lo + 1 : 0;
+            const int64_t nv = n_visible(t, a.ratio, a.P);
+            const int64_t n_e = a.mode == 0 ? (a.topk < nv ? a.topk : nv) : nv;
+            pre[(size_t)i + 1] = pre[(size_t)i] + (n_win + kTile - 1) / kTile + (n_e + kTile - 1) / kTile + 1;
+        }
+        // work item w = b * S_q + i: its cumulative cost is b * pre[S_q] + pre[i]
+        const int64_t per_b = pre[(size_t)a.S_q], total = per_b * a.B;
+        int64_t w = 0;
+        for (int c = 0; c <= grid; ++c) {
+            const int64_t target = total * c / grid;
+            while (w < nw && (w / a.S_q) * per_b + pre[(size_t)(w % a.S_q)] < target) ++w;
+            ranges.start[c] = (int32_t)w;
+        }
+        ranges.start[grid] = (int32_t)nw;
+    }
     // split queries: each pair of CTAs (key ranges 0 and 1 of one query) is a 2-CTA cluster
     // that merges in-kernel
     const cudaError_t le = launch_dependent(
         kern, dim3((unsigned)grid), dim3(kThreads), smem, st, n_split == 2 ? 2 : 1, map_q, map_q7, map_kv, map_pool,
         map_k7, pool_src, (int64_t)a.S_kv, (int64_t)a.kv_pos0, (int64_t)a.P, a.idx, a.mode == 0 ? a.topk : 0, a.mode, a.sink, (__nv_bfloat16 *)a.out, (int64_t)a.B,
         (int64_t)a.S_q, (int64_t)a.q_pos0, a.window, a.ratio, a.scale, a.rope, kmax7, (const int32_t *)ent_g,
-        (const int32_t *)n_ent_g, g_attend_tc_withhold.load(), n_split, part);
+        (const int32_t *)n_ent_g, g_attend_tc_withhold.load(), n_split, part, ranges);
     CSA_REQUIRE(le == cudaSuccess, CSA_ERR_CUDA, "%s: launch failed: %s", a.mode == 0 ? "csa_attend" : "hca_attend",
                 cudaGetErrorString(le));
     CSA_CHECK_LAUNCH(a.mode == 0 ? "csa_attend" : "hca_attend");
