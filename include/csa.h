@@ -155,10 +155,13 @@ csa_status_t csa_rope_rows(const void *x, void *out, int64_t rows, int32_t D, in
                            double rope_base, int64_t pos0, int64_t group, int64_t period,
                            int64_t step, csa_dtype_t dtype, void *stream);
 
-/* Scratch bytes csa_index_topk needs for these sizes (0 when the call needs none).  A
- * decode-sized call is split over entry ranges: rows with at most 16384 visible entries
- * pass every entry's 64-bit key through the workspace to a selection kernel, longer rows
- * pass each range's candidates to a merge kernel. */
+/* Scratch bytes csa_index_topk needs for these sizes (0 when the call needs none).  When
+ * every row has at most 16384 visible entries, the indexer writes every visible entry's
+ * 32-bit score key to the workspace (one row of round_up(P, 4) keys per query) and a
+ * selection kernel picks the top-k: decode-sized calls, and prefill calls whose key rows
+ * take at most 2 GiB.  Otherwise a decode-sized call split over entry ranges passes each
+ * range's candidates to a merge kernel, and a prefill call keeps its candidates in shared
+ * memory (no workspace). */
 size_t csa_index_topk_workspace_bytes(int64_t B, int64_t S_q, int64_t q_pos0, int64_t P,
                                       int32_t H_I, int32_t d_I, int32_t ratio, int32_t topk,
                                       csa_dtype_t dtype);

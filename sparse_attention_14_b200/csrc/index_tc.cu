@@ -12,15 +12,18 @@
 //  * warp roles: warp 0 issues TMA loads into a ring of entry tiles, warp 1 issues the
 //    MMAs (one thread), the epilogue warps read D from TMEM (thread = entry row) and
 //    form sum_h w[q,h] ReLU(D) for their queries, while the next tile's MMA runs;
-//  * top-k without writing scores to HBM: each query keeps a candidate buffer of
-//    kCap = 2048 64-bit keys (order-preserving score bits, then the complemented entry index,
-//    so that equal scores rank the lower index first) and a threshold; a tile inserts
-//    only keys above the threshold, and whenever the buffer could overflow it is cut
-//    back to exactly k by an exact radix select over the 64-bit keys (which then becomes
-//    the threshold);
-//  * output: the k survivors in ascending entry order (deterministic), or, for a
-//    decode-sized problem split over entry ranges, each range's candidates go to the
-//    workspace and a merge kernel selects the final k.
+//  * keys: a key is the order-preserving score bits, then the complemented entry index,
+//    so that keys are unique and equal scores rank the lower index first;
+//  * rows of at most 16384 visible entries (the usual case): the indexer writes every
+//    visible entry's 32-bit score key to a workspace row and a selection kernel picks the
+//    top-k (value bins, then an exact rank inside the k-th key's bin).  Prefill runs a
+//    persistent key stream (index_keys_kernel): its MMAs never wait for a selection;
+//  * longer rows: each query keeps a candidate buffer of kCap = 2048 keys in shared memory
+//    and a threshold; a tile inserts only keys above the threshold, and whenever the
+//    buffer could overflow it is cut back to exactly k by an exact radix select (which
+//    then becomes the threshold); a decode-sized problem split over entry ranges passes
+//    each range's candidates through the workspace to a merge kernel;
+//  * output: the k selected entries in ascending entry order (deterministic).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -85,6 +88,9 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         : "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
         : "memory");
 }
+
+// the key workspace holds one row of 32-bit score keys per query, rows 16-byte aligned
+__host__ __device__ __forceinline__ int64_t key_pitch(int64_t P) { return (P + 3) & ~(int64_t)3; }
 
 __device__ __forceinline__ float key_to_float(uint32_t key) {
     uint32_t u = (key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key;
@@ -323,7 +329,7 @@ __global__ void __launch_bounds__(Cfg<QB>::kThreads, Cfg<QB>::kMinBlocks) index_
     const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
     const __nv_bfloat16 *__restrict__ w, int64_t B, int64_t S_q, int64_t q_pos0, int64_t P, int ratio,
     int topk, int n_split, int32_t *__restrict__ idx, float *__restrict__ scores_opt,
-    unsigned long long *__restrict__ partial, unsigned long long *__restrict__ keys_out) {
+    unsigned long long *__restrict__ partial, uint32_t *__restrict__ keys_out) {
     using C = Cfg<QB>;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -475,12 +481,10 @@ __global__ void __launch_bounds__(Cfg<QB>::kThreads, Cfg<QB>::kMinBlocks) index_
             __syncwarp();
             if (lane == 0) mbar_arrive(&ms.tempty[acc]);
             if (QB == 1 && keys_out) {
-                // keys only: every visible entry's key goes to the row's slot j; the
+                // keys only: every visible entry's score key goes to the row's slot j; the
                 // selection runs in index_select_kernel.  No barrier inside the loop here, so
                 // a thread whose wait ran out leaves on its own.
-                if (j < nvq[0])
-                    keys_out[(b * S_q + i0) * P + j] = ((unsigned long long)order_key(sc[0]) << 32) |
-                                                       (unsigned long long)(0xFFFFFFFFu - (uint32_t)j);
+                if (j < nvq[0]) keys_out[(b * S_q + i0) * key_pitch(P) + j] = order_key(sc[0]);
                 if (!ok) break;
                 continue;
             }
@@ -545,6 +549,261 @@ __global__ void __launch_bounds__(Cfg<QB>::kThreads, Cfg<QB>::kMinBlocks) index_
     if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
 }
 
+// Prefill key stream: persistent CTAs walk the blocks of 4 consecutive queries, longest
+// first and in snake order over the grid (CTA c takes blocks c, 2G-1-c, 2G+c, ...), so that
+// every CTA gets about the same number of entry tiles.  A block's q_I rows (64 KB) go to
+// one of two B stages, so the next block's load overlaps this block's tiles; entry tiles
+// of k_I stream through three A stages; D = k_I . q_I^T [128 entries, 4 queries x 64 heads]
+// is double-buffered in TMEM across blocks.  The epilogue forms each (query, entry) score
+// and writes its order-preserving key to the row's slot; index_select_kernel selects.
+constexpr int kKsNST = 3;
+struct KsCfg {
+    static constexpr int N = 256;                                 // 4 queries x 64 heads
+    static constexpr int NE = 8;                                  // epilogue warps
+    static constexpr int kThreads = (2 + NE) * 32;
+    static constexpr uint32_t kBChunk = 256 * 64 * 2;             // one 64-column chunk of q_I rows
+    static constexpr uint32_t kBBytes = 2 * kBChunk;              // 64 KB
+    static constexpr uint32_t kABytes = kTileE * kDI * 2;         // 32 KB
+    static constexpr uint32_t kOffB = 0;
+    static constexpr uint32_t kOffA = 2 * kBBytes;
+    static constexpr uint32_t kOffW = kOffA + kKsNST * kABytes;
+    static constexpr uint32_t kOffMisc = kOffW + 256 * 4;
+};
+struct KsMisc {
+    uint64_t afull[kKsNST], aempty[kKsNST], bfull[2], bempty[2], tfull[2], tempty[2];
+    uint32_t tmem_base;
+};
+constexpr size_t kKsSmem = KsCfg::kOffMisc + sizeof(KsMisc) + 1024;
+
+// query block of round r for CTA c (-1: none); blocks are numbered longest first
+__device__ __forceinline__ int64_t ks_block(int64_t r, int c, int G, int64_t n_qb) {
+    const int64_t k = r * G + ((r & 1) ? (G - 1 - c) : c);
+    return k < n_qb ? k : -1;
+}
+
+__global__ void __launch_bounds__(KsCfg::kThreads, 1) index_keys_kernel(
+    const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
+    const __nv_bfloat16 *__restrict__ w, int64_t B, int64_t S_q, int64_t q_pos0, int64_t P, int ratio,
+    uint32_t *__restrict__ keys_out) {
+    using C = KsCfg;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t base = smem_u32(smem);
+    float *w_s = reinterpret_cast<float *>(smem + C::kOffW);
+    KsMisc &ms = *reinterpret_cast<KsMisc *>(smem + C::kOffMisc);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int G = (int)gridDim.x, c = (int)blockIdx.x;
+    const int64_t qb_per_seq = (S_q + 3) / 4;
+    const int64_t n_qb = B * qb_per_seq;
+    // block k (longest first): query block qb_per_seq - 1 - k / B of sequence k % B
+    auto geom = [&](int64_t k, int64_t *b, int64_t *i0, int *nq, int *n_tiles) {
+        *b = k % B;
+        *i0 = (qb_per_seq - 1 - k / B) * 4;
+        *nq = (int)((S_q - *i0) < 4 ? (S_q - *i0) : 4);
+        const int64_t nv_max = n_visible(q_pos0 + *i0 + *nq - 1, ratio, P);
+        *n_tiles = (int)((nv_max + kTileE - 1) / kTileE);
+    };
+
+    if (tid == 0) {
+        for (int s = 0; s < kKsNST; ++s) {
+            mbar_init(&ms.afull[s], 1);
+            mbar_init(&ms.aempty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&ms.bfull[a], 1);
+            mbar_init(&ms.bempty[a], 1);
+            mbar_init(&ms.tfull[a], 1);
+            mbar_init(&ms.tempty[a], C::NE);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(&ms.tmem_base, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ms.tmem_base;
+    grid_wait();
+    grid_launch_dependents();
+    const uint32_t sB = base + C::kOffB, sA = base + C::kOffA;
+
+    if (warp == 0) {
+        // ---------------- producer
+        if (lane == 0) {
+            // the next block with entry tiles at or after round r0
+            auto find = [&](int64_t r0, int64_t *rr, int64_t *b, int64_t *i0, int *nt) {
+                for (int64_t r1 = r0; r1 * G < n_qb; ++r1) {
+                    const int64_t k = ks_block(r1, c, G, n_qb);
+                    if (k < 0) continue;
+                    int nq;
+                    geom(k, b, i0, &nq, nt);
+                    if (*nt == 0) continue;
+                    *rr = r1;
+                    return true;
+                }
+                return false;
+            };
+            auto issue_b = [&](uint32_t bi, int64_t b, int64_t i0) {
+                const uint32_t bs = bi & 1u;
+                mbar_expect_tx(&ms.bfull[bs], C::kBBytes);
+                const int yq = (int)((b * S_q + i0) * kHI);
+                tma_load_2d(sB + bs * C::kBBytes, &map_q, 0, yq, &ms.bfull[bs]);
+                tma_load_2d(sB + bs * C::kBBytes + C::kBChunk, &map_q, 64, yq, &ms.bfull[bs]);
+            };
+            int64_t rc = 0, bc = 0, ic = 0;
+            int ntc = 0;
+            bool have = find(0, &rc, &bc, &ic, &ntc);
+            if (have) issue_b(0u, bc, ic);
+            uint32_t it = 0, bi = 0;
+            bool ok = true;
+            while (have && ok) {
+                int64_t rn = 0, bn = 0, in = 0;
+                int ntn = 0;
+                const bool has_next = find(rc + 1, &rn, &bn, &in, &ntn);
+                // the next block's q_I rows go to the other B stage as soon as the MMAs of the
+                // block before this one have released it, so they land while this block runs
+                const uint32_t bx = bi + 1;
+                bool next_issued = !has_next;
+                for (int t = 0; t < ntc; ++t, ++it) {
+                    if (!next_issued && (bx < 2 || mbar_test_wait(&ms.bempty[bx & 1u], ((bx >> 1) - 1) & 1u))) {
+                        issue_b(bx, bn, in);
+                        next_issued = true;
+                    }
+                    const uint32_t s = it % kKsNST;
+                    if (it >= kKsNST) ok = mbar_wait(&ms.aempty[s], ((it / kKsNST) - 1) & 1u);
+                    if (!ok) break;
+                    mbar_expect_tx(&ms.afull[s], C::kABytes);
+                    const int ye = (int)(bc * P + (int64_t)t * kTileE);
+                    const uint32_t dst = sA + s * C::kABytes;
+                    tma_load_2d(dst, &map_k, 0, ye, &ms.afull[s]);
+                    tma_load_2d(dst + 16384u, &map_k, 64, ye, &ms.afull[s]);
+                }
+                if (ok && !next_issued) {
+                    ok = mbar_wait(&ms.bempty[bx & 1u], ((bx >> 1) - 1) & 1u);
+                    if (ok) issue_b(bx, bn, in);
+                }
+                ++bi;
+                rc = rn;
+                bc = bn;
+                ic = in;
+                ntc = ntn;
+                have = has_next;
+            }
+            if (!ok) atomicOr(&g_index_tc_status, 1u);
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(128, C::N, 0, 0);
+            const uint64_t d_a = sdesc_sw128(sA, 16, 1024), d_b = sdesc_sw128(sB, 16, 1024);
+            const uint32_t a_lo0 = (uint32_t)d_a, b_lo0 = (uint32_t)d_b, hi = (uint32_t)(d_a >> 32);
+            uint32_t it = 0, bi = 0;
+            bool ok = true;
+            for (int64_t r = 0; ok && r * G < n_qb; ++r) {
+                const int64_t k = ks_block(r, c, G, n_qb);
+                if (k < 0) continue;
+                int64_t b, i0;
+                int nq, n_tiles;
+                geom(k, &b, &i0, &nq, &n_tiles);
+                if (n_tiles == 0) continue;
+                const uint32_t bs = bi & 1u;
+                ok = mbar_wait(&ms.bfull[bs], (bi >> 1) & 1u);
+                if (!ok) break;
+                const uint32_t b_lo = b_lo0 + ((bs * C::kBBytes) >> 4);
+                for (int t = 0; t < n_tiles; ++t, ++it) {
+                    const uint32_t s = it % kKsNST, acc = it & 1u;
+                    ok = mbar_wait(&ms.afull[s], (it / kKsNST) & 1u);
+                    if (ok && it >= 2) ok = mbar_wait(&ms.tempty[acc], ((it >> 1) - 1) & 1u);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t a_lo = a_lo0 + ((s * C::kABytes) >> 4);
+#pragma unroll
+                    for (int ks = 0; ks < kDI / 16; ++ks)
+                        mma_bf16_w(tmem + acc * (uint32_t)C::N,
+                                   a_lo + (uint32_t)(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4), hi,
+                                   b_lo + (uint32_t)(((ks >> 2) * C::kBChunk + (ks & 3) * 32) >> 4), hi, idesc,
+                                   ks > 0 ? 1u : 0u);
+                    mma_commit(&ms.aempty[s]);
+                    mma_commit(&ms.tfull[acc]);
+                }
+                if (!ok) break;
+                mma_commit(&ms.bempty[bs]);
+                ++bi;
+            }
+            if (!ok) atomicOr(&g_index_tc_status, 1u);
+        }
+    } else {
+        // ---------------- epilogue: thread = entry row of the tile, 2 queries x 64 heads
+        const int e = warp - 2;                  // 0 .. NE-1
+        const int g4 = warp & 3;                 // TMEM lane group of this warp
+        const int row = g4 * 32 + lane;
+        const int qa = 2 * (e >> 2);
+        const int et = e * 32 + lane;            // 0 .. 255
+        uint32_t it = 0;
+        bool ok = true;
+        for (int64_t r = 0; r * G < n_qb; ++r) {
+            const int64_t k = ks_block(r, c, G, n_qb);
+            if (k < 0) continue;
+            int64_t b, i0;
+            int nq, n_tiles;
+            geom(k, &b, &i0, &nq, &n_tiles);
+            if (n_tiles == 0) continue;
+            // the previous block's weights are no longer read; stage this block's
+            if (named_sync_any(1, C::NE * 32, !ok)) break;
+            {
+                const int q = et >> 6, h = et & 63;
+                w_s[et] = q < nq ? __bfloat162float(w[(b * S_q + i0 + q) * kHI + h]) : 0.f;
+            }
+            named_sync(1, C::NE * 32);
+            int64_t nvq[2];
+#pragma unroll
+            for (int qq = 0; qq < 2; ++qq)
+                nvq[qq] = qa + qq < nq ? n_visible(q_pos0 + i0 + qa + qq, ratio, P) : 0;
+            uint32_t *krow = keys_out + (b * S_q + i0 + qa) * key_pitch(P);
+            for (int t = 0; t < n_tiles; ++t, ++it) {
+                const uint32_t acc = it & 1u;
+                if (!mbar_wait(&ms.tfull[acc], (it >> 1) & 1u)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const int64_t j = (int64_t)t * kTileE + row;
+                const uint32_t trow = tmem + ((uint32_t)(g4 * 32) << 16) + acc * (uint32_t)C::N;
+                float sc[2];
+#pragma unroll
+                for (int qq = 0; qq < 2; ++qq) {
+                    const int q = qa + qq;
+                    float v[64];
+                    tmem_ld32(trow + (uint32_t)(q * 64), v);
+                    tmem_ld32(trow + (uint32_t)(q * 64 + 32), v + 32);
+                    tmem_ld_wait();
+                    float s4[4] = {0.f, 0.f, 0.f, 0.f};
+                    const float4 *wq = reinterpret_cast<const float4 *>(w_s + q * 64);
+#pragma unroll
+                    for (int h4 = 0; h4 < 16; ++h4) {
+                        const float4 ww = wq[h4];
+                        s4[0] = fmaf(ww.x, fmaxf(v[4 * h4 + 0], 0.f), s4[0]);
+                        s4[1] = fmaf(ww.y, fmaxf(v[4 * h4 + 1], 0.f), s4[1]);
+                        s4[2] = fmaf(ww.z, fmaxf(v[4 * h4 + 2], 0.f), s4[2]);
+                        s4[3] = fmaf(ww.w, fmaxf(v[4 * h4 + 3], 0.f), s4[3]);
+                    }
+                    sc[qq] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ms.tempty[acc]);
+#pragma unroll
+                for (int qq = 0; qq < 2; ++qq)
+                    if (j < nvq[qq]) krow[qq * key_pitch(P) + j] = order_key(sc[qq]);
+            }
+        }
+        if (!ok) atomicOr(&g_index_tc_status, 1u);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
 // Merge the per-range candidates of one query row (decode split).
 constexpr int kMergeThreads = 256;
 __global__ void __launch_bounds__(kMergeThreads) index_merge_kernel(
@@ -563,26 +822,40 @@ __global__ void __launch_bounds__(kMergeThreads) index_merge_kernel(
                                 scores_opt ? scores_opt + row * topk : nullptr);
 }
 
-// Top-k of one query row from the keys of all its visible entries (decode calls whose
-// indexer wrote keys instead of candidates).  1024 threads hold the row's keys in
-// registers, 16 each (entry e = u*1024 + tid).  The scores are binned by value between
-// the row's min and max, bin = floor((score - min) * 2048 / (max - min)) -- a monotone map,
+// Top-k of one query row from the score keys of all its visible entries (calls whose
+// indexer wrote keys instead of candidates).  The block holds the row's keys in
+// registers, PER per thread (entry e = u*T + tid), each widened to the 64-bit key
+// (order-preserving score bits, then the complemented entry index, so keys are unique and
+// equal scores rank the lower index first).  The scores are binned by value between the
+// row's min and max, bin = floor((score - min) * 2048 / (max - min)) -- a monotone map,
 // so equal scores share a bin and bins are ordered like the keys.  (Binning the score's
 // order-preserving bits instead is logarithmic in the score: with scores near zero in
-// the row, the top of the range falls into a handful of crowded bins.)  The bin holding the k-th largest key is found from
-// the bin counts, and only that bin's keys are ranked: by counting (each of at most 1024
-// keys against the others) or, for a crowded bin, by the radix select group_kth run by
-// 512 of the threads, tightened to the k-th key itself.  The entries with key >= T -- exactly k, the keys
-// being unique -- are written in ascending entry order through a bitmap built with warp
-// ballots.
-constexpr int kSelThreads = 1024, kSelPer = 16, kSelMax = kSelThreads * kSelPer, kSelBins = 2048;
-__global__ void __launch_bounds__(kSelThreads) index_select_kernel(
-    const unsigned long long *__restrict__ keys, int64_t P, int topk, int32_t *__restrict__ idx,
+// the row, the top of the range falls into a handful of crowded bins.)  The bin holding
+// the k-th largest key is found from the bin counts, and only that bin's keys are ranked:
+// by counting (each of at most T keys against the others) or, for a crowded bin, by the
+// radix select group_kth, tightened to the k-th key itself.  The entries with key >= the
+// k-th -- exactly k -- are written in ascending entry order through a bitmap built with
+// warp ballots.
+constexpr int kSelBins = 2048;
+constexpr int kSelMax = 1024 * 16;   // visible entries per row, largest block
+template <int T, int PER>
+struct SelCfg {
+    static constexpr int kMax = T * PER;
+    static constexpr int kRadix = T > 512 ? 512 : T;   // threads of the crowded-bin select
+    // the chosen bin's keys, bitmap, bins, radix histogram, scan and min/max partials, Misc
+    static constexpr size_t kSmem =
+        (size_t)kMax * 8 + kMax / 32 * 4 + kSelBins * 4 + 256 * 4 + 32 * 4 + 64 * 4 + sizeof(Misc);
+};
+
+template <int T, int PER>
+__global__ void __launch_bounds__(T) index_select_kernel(
+    const uint32_t *__restrict__ keys, int64_t P, int topk, int32_t *__restrict__ idx,
     float *__restrict__ scores_opt, int64_t S_q, int64_t q_pos0, int ratio) {
+    using SC = SelCfg<T, PER>;
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    unsigned long long *sub = reinterpret_cast<unsigned long long *>(smem_raw);   // [kSelMax] chosen bin
-    unsigned *bitmap = reinterpret_cast<unsigned *>(sub + kSelMax);              // [kSelMax / 32]
-    unsigned *bins = bitmap + kSelMax / 32;                                       // [kSelBins]
+    unsigned long long *sub = reinterpret_cast<unsigned long long *>(smem_raw);   // [kMax] chosen bin
+    unsigned *bitmap = reinterpret_cast<unsigned *>(sub + SC::kMax);             // [kMax / 32]
+    unsigned *bins = bitmap + SC::kMax / 32;                                      // [kSelBins]
     unsigned *hist = bins + kSelBins;                                             // [256]
     unsigned *wpart = hist + 256;                                                 // [32]
     float *red = reinterpret_cast<float *>(wpart + 32);                           // [64]
@@ -593,27 +866,28 @@ __global__ void __launch_bounds__(kSelThreads) index_select_kernel(
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     grid_wait();   // the indexer's keys
     grid_launch_dependents();
-    const int n = (int)n_visible(q_pos0 + row % S_q, ratio, P);   // <= kSelMax (host check)
-    const unsigned long long *kr = keys + row * P;
+    const int n = (int)n_visible(q_pos0 + row % S_q, ratio, P);   // <= kMax (host check)
+    const uint32_t *kr = keys + row * key_pitch(P);
     int32_t *idx_row = idx + row * (int64_t)topk;
     float *score_row = scores_opt ? scores_opt + row * (int64_t)topk : nullptr;
 
-    unsigned long long key[kSelPer];
+    unsigned long long key[PER];
 #pragma unroll
-    for (int u = 0; u < kSelPer; ++u) {
-        const int e = u * kSelThreads + tid;
-        key[u] = e < n ? __ldcg(kr + e) : 0ull;
+    for (int u = 0; u < PER; ++u) {
+        const int e = u * T + tid;
+        key[u] = e < n ? ((unsigned long long)__ldcg(kr + e) << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)e)
+                       : 0ull;
     }
     float lo = INFINITY, hi = -INFINITY;   // range of the scores
 #pragma unroll
-    for (int u = 0; u < kSelPer; ++u) {
-        if (u * kSelThreads + tid < n) {
+    for (int u = 0; u < PER; ++u) {
+        if (u * T + tid < n) {
             const float f = key_to_float((uint32_t)(key[u] >> 32));
             lo = fminf(lo, f);
             hi = fmaxf(hi, f);
         }
     }
-    for (int b = tid; b < kSelBins; b += kSelThreads) bins[b] = 0u;
+    for (int b = tid; b < kSelBins; b += T) bins[b] = 0u;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         lo = fminf(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, o));
@@ -631,7 +905,7 @@ __global__ void __launch_bounds__(kSelThreads) index_select_kernel(
     if (n > topk) {
         lo = red[0];
         hi = red[32];
-        for (int w = 1; w < kSelThreads / 32; ++w) {
+        for (int w = 1; w < T / 32; ++w) {
             lo = fminf(lo, red[w]);
             hi = fmaxf(hi, red[32 + w]);
         }
@@ -642,11 +916,11 @@ __global__ void __launch_bounds__(kSelThreads) index_select_kernel(
             return b < 0 ? 0 : (b >= kSelBins ? kSelBins - 1 : b);
         };
 #pragma unroll
-        for (int u = 0; u < kSelPer; ++u)
-            if (u * kSelThreads + tid < n) atomicAdd(&bins[bin_of(key[u])], 1u);
+        for (int u = 0; u < PER; ++u)
+            if (u * T + tid < n) atomicAdd(&bins[bin_of(key[u])], 1u);
         __syncthreads();
-        // the bin holding the topk-th largest key: suffix counts over bins, 2 per thread
-        constexpr int BPT = kSelBins / kSelThreads;
+        // the bin holding the topk-th largest key: suffix counts over bins, BPT per thread
+        constexpr int BPT = kSelBins / T;
         const int b_hi = kSelBins - tid * BPT;   // my bins: [b_hi - BPT, b_hi), from the top
         unsigned local = 0;
 #pragma unroll
@@ -673,40 +947,40 @@ __global__ void __launch_bounds__(kSelThreads) index_select_kernel(
         __syncthreads();
         const int bstar = sel_bin;
 #pragma unroll
-        for (int u = 0; u < kSelPer; ++u)
-            if (u * kSelThreads + tid < n && bin_of(key[u]) == bstar) sub[atomicAdd(&sel_n, 1)] = key[u];
+        for (int u = 0; u < PER; ++u)
+            if (u * T + tid < n && bin_of(key[u]) == bstar) sub[atomicAdd(&sel_n, 1)] = key[u];
         __syncthreads();
         const int nb = sel_n, kb = topk - sel_above;   // the kb-th largest of the bin's nb keys
-        if (nb <= kSelThreads) {
+        if (nb <= T) {
             if (tid < nb) {
                 const unsigned long long mine = sub[tid];
                 int rank = 0;
                 for (int i = 0; i < nb; ++i) rank += sub[i] > mine ? 1 : 0;
                 if (rank == kb - 1) sel_T = mine;
             }
-        } else if (tid < 512) {
-            // crowded bin (many equal or near-equal scores): radix select by warps 0-15,
-            // then the smallest of the bin's keys >= its prefix threshold
-            const unsigned long long t = group_kth<512>(sub, nb, kb, tid, 2, hist, ms, 0);
+        } else if (tid < SC::kRadix) {
+            // crowded bin (many equal or near-equal scores): radix select by the first
+            // kRadix threads, then the smallest of the bin's keys >= its prefix threshold
+            const unsigned long long t = group_kth<SC::kRadix>(sub, nb, kb, tid, 2, hist, ms, 0);
             if (tid == 0) sel_T = ~0ull;
-            named_sync(2, 512);
-            for (int e = tid; e < nb; e += 512)
+            named_sync(2, SC::kRadix);
+            for (int e = tid; e < nb; e += SC::kRadix)
                 if (sub[e] >= t) atomicMin(&sel_T, sub[e]);
         }
         __syncthreads();
     }
-    const unsigned long long T = sel_T;
-    // bitmap of the selected entries: word u*32 + wid holds entries (u*1024 + wid*32 + lane)
+    const unsigned long long thr = sel_T;
+    // bitmap of the selected entries: word u*(T/32) + wid holds entries (u*T + wid*32 + lane)
     const int nwords = (n + 31) >> 5;
 #pragma unroll
-    for (int u = 0; u < kSelPer; ++u) {
-        const int e = u * kSelThreads + tid;
-        const unsigned m = __ballot_sync(0xFFFFFFFFu, e < n && key[u] >= T);
+    for (int u = 0; u < PER; ++u) {
+        const int e = u * T + tid;
+        const unsigned m = __ballot_sync(0xFFFFFFFFu, e < n && key[u] >= thr);
         if (lane == 0 && (e >> 5) < nwords) bitmap[e >> 5] = m;
     }
     __syncthreads();
     // output slots: thread tid owns words [tid*wpt, (tid+1)*wpt); exclusive scan of counts
-    const int wpt = (nwords + kSelThreads - 1) / kSelThreads;
+    const int wpt = (nwords + T - 1) / T;
     unsigned local = 0;
     for (int w = tid * wpt; w < (tid + 1) * wpt && w < nwords; ++w) local += __popc(bitmap[w]);
     unsigned incl = local;
@@ -725,20 +999,286 @@ __global__ void __launch_bounds__(kSelThreads) index_select_kernel(
             const int j = 32 * w + __ffs(m) - 1;
             m &= m - 1u;
             idx_row[pos] = j;
-            if (score_row) score_row[pos] = key_to_float((uint32_t)(__ldcg(kr + j) >> 32));
+            if (score_row) score_row[pos] = key_to_float(__ldcg(kr + j));
             ++pos;
         }
     }
     const int n_sel = n < topk ? n : topk;
-    for (int r = n_sel + tid; r < topk; r += kSelThreads) {
+    for (int r = n_sel + tid; r < topk; r += T) {
         idx_row[r] = -1;
         if (score_row) score_row[r] = __int_as_float(0x7fc00000);
     }
 }
 
-// the chosen bin's keys, bitmap, bins, radix histogram, scan and min/max partials, Misc
-constexpr size_t kSelSmem =
-    (size_t)kSelMax * 8 + kSelMax / 32 * 4 + kSelBins * 4 + 256 * 4 + 32 * 4 + 64 * 4 + sizeof(Misc);
+// Rows of at most 2048 visible entries: one warp per row, no block-wide barrier.  The
+// row's 32-bit score keys are copied into the warp's shared memory (16-byte async copies);
+// every pass reads four consecutive keys per lane and step (entries e = 4*(i*32 + lane) + c).
+// The scores are binned by value between the row's min and max into 1024 bins (a monotone
+// map); the bin holding the k-th largest key is found from the bin counts.  A bin of at
+// most 64 keys is ranked by counting on the 64-bit keys (score key, complemented entry
+// index).  A crowded bin falls back to an MSB-first radix select on its 32-bit keys (four
+// 8-bit passes, exact), and the equal keys at the threshold are taken in ascending entry
+// order.  Either way the threshold T is one row key, and exactly k keys are >= T; they are
+// written in ascending entry order.
+constexpr int kWsWarps = 4, kWsBins = 1024, kWsSub = 64;
+constexpr int kWsMax = 2048;   // entries per row
+struct WsWarp {
+    uint4 k4[kWsMax / 4];                // the row's keys
+    unsigned bins[kWsBins];
+    unsigned long long sub[kWsSub];
+    unsigned long long thr;
+    unsigned cnt;
+};
+constexpr size_t kWsSmem = (size_t)kWsWarps * sizeof(WsWarp);
+
+__global__ void __launch_bounds__(kWsWarps * 32) index_select_warp_kernel(
+    const uint32_t *__restrict__ keys, int64_t P, int topk, int32_t *__restrict__ idx,
+    float *__restrict__ scores_opt, int64_t rows, int64_t S_q, int64_t q_pos0, int ratio) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    grid_wait();   // the indexer's keys
+    grid_launch_dependents();
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int64_t row = (int64_t)blockIdx.x * kWsWarps + wid;
+    if (row >= rows) return;   // warps are independent: no block barrier follows
+    WsWarp &ws = reinterpret_cast<WsWarp *>(smem_raw)[wid];
+    const int n = (int)n_visible(q_pos0 + row % S_q, ratio, P);   // <= kWsMax (host check)
+    const uint32_t *kr = keys + row * key_pitch(P);
+    int32_t *idx_row = idx + row * (int64_t)topk;
+    float *score_row = scores_opt ? scores_opt + row * (int64_t)topk : nullptr;
+    const int nsteps = (n + 127) >> 7;   // steps of 32 lanes x 4 keys
+
+    // the row's keys (the tail of the last 16-byte piece is never read as a key)
+    for (int v = lane; v < (n + 3) >> 2; v += 32) cp_async16(smem_u32(&ws.k4[v]), kr + 4 * v, 16u);
+    cp_async_commit();
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncwarp();
+    auto load4 = [&](int i, uint32_t k[4]) {
+        const uint4 v = ws.k4[i * 32 + lane];
+        k[0] = v.x;
+        k[1] = v.y;
+        k[2] = v.z;
+        k[3] = v.w;
+    };
+    unsigned long long T = 0ull;   // every key is > 0: all entries selected when n <= topk
+    if (n > topk) {
+        // ---- value bins between the row's min and max
+        float lo = INFINITY, hi = -INFINITY;
+        for (int i = 0; i < nsteps; ++i) {
+            uint32_t k[4];
+            load4(i, k);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                if (4 * (i * 32 + lane) + c < n) {
+                    const float f = key_to_float(k[c]);
+                    lo = fminf(lo, f);
+                    hi = fmaxf(hi, f);
+                }
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            lo = fminf(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, o));
+            hi = fmaxf(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, o));
+        }
+        const float scale = hi > lo ? (float)kWsBins / (hi - lo) : 0.f;
+        auto bin_of = [&](uint32_t k) {
+            // NaN (0 * inf) goes to bin 0 and +inf to the top bin: still monotone in the score
+            const float x = fminf(fmaxf((key_to_float(k) - lo) * scale, 0.f), (float)(kWsBins - 1));
+            return (int)x;
+        };
+        uint4 *b4 = reinterpret_cast<uint4 *>(ws.bins);
+        for (int i = lane; i < kWsBins / 4; i += 32) b4[i] = make_uint4(0u, 0u, 0u, 0u);
+        __syncwarp();
+        for (int i = 0; i < nsteps; ++i) {
+            uint32_t k[4];
+            load4(i, k);
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                if (4 * (i * 32 + lane) + c < n) atomicAdd(&ws.bins[bin_of(k[c])], 1u);
+        }
+        __syncwarp();
+        // lane l owns bins [kWsBins - 32(l+1), kWsBins - 32l), counted from the top
+        constexpr int BPL = kWsBins / 32;
+        const int b_hi = kWsBins - lane * BPL;
+        unsigned local = 0;
+#pragma unroll
+        for (int k = 0; k < BPL / 4; ++k) {
+            const uint4 v = b4[(b_hi - BPL) / 4 + k];
+            local += v.x + v.y + v.z + v.w;
+        }
+        unsigned incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        // the lane whose range holds the topk-th largest key finds the bin
+        int my_bin = -1;
+        unsigned my_above = 0, my_cnt = 0;
+        {
+            unsigned cum = incl - local;
+            if (cum < (unsigned)topk && (unsigned)topk <= incl) {
+                for (int k = 1; k <= BPL; ++k) {
+                    const unsigned h = ws.bins[b_hi - k];
+                    if (cum < (unsigned)topk && (unsigned)topk <= cum + h) {
+                        my_bin = b_hi - k;
+                        my_above = cum;
+                        my_cnt = h;
+                        break;
+                    }
+                    cum += h;
+                }
+            }
+        }
+        const unsigned who = __ballot_sync(0xFFFFFFFFu, my_bin >= 0);
+        const int src = __ffs(who) - 1;
+        const int bstar = __shfl_sync(0xFFFFFFFFu, my_bin, src);
+        const int need = topk - (int)__shfl_sync(0xFFFFFFFFu, my_above, src);   // >= 1
+        const int nb = (int)__shfl_sync(0xFFFFFFFFu, my_cnt, src);
+        if (nb <= kWsSub) {
+            // ---- rank the bin's keys by counting
+            if (lane == 0) ws.cnt = 0u;
+            __syncwarp();
+            for (int i = 0; i < nsteps; ++i) {
+                uint32_t k[4];
+                load4(i, k);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int e = 4 * (i * 32 + lane) + c;
+                    if (e < n && bin_of(k[c]) == bstar)
+                        ws.sub[atomicAdd(&ws.cnt, 1u)] =
+                            ((unsigned long long)k[c] << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)e);
+                }
+            }
+            __syncwarp();
+            for (int i = lane; i < nb; i += 32) {
+                const unsigned long long mine = ws.sub[i];
+                int rank = 0;
+                for (int j = 0; j < nb; ++j) rank += ws.sub[j] > mine ? 1 : 0;
+                if (rank == need - 1) ws.thr = mine;
+            }
+            __syncwarp();
+            T = ws.thr;
+        } else {
+            // ---- crowded bin: exact radix select on its 32-bit keys, then ties by index
+            uint32_t prefix = 0;
+            int rem = need;
+            for (int shift = 24; shift >= 0; shift -= 8) {
+                const uint32_t mask = shift == 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
+                for (int i = lane; i < 64; i += 32) b4[i] = make_uint4(0u, 0u, 0u, 0u);
+                __syncwarp();
+                for (int i = 0; i < nsteps; ++i) {
+                    uint32_t k[4];
+                    load4(i, k);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        if (4 * (i * 32 + lane) + c < n && (k[c] & mask) == prefix && bin_of(k[c]) == bstar)
+                            atomicAdd(&ws.bins[(k[c] >> shift) & 255u], 1u);
+                }
+                __syncwarp();
+                // lane l owns digits [256 - 8(l+1), 256 - 8l), from the top
+                const int d_hi = 256 - lane * 8;
+                unsigned loc = 0;
+#pragma unroll
+                for (int k = 1; k <= 8; ++k) loc += ws.bins[d_hi - k];
+                unsigned inc = loc;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const unsigned v = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+                    if (lane >= o) inc += v;
+                }
+                int my_d = -1;
+                unsigned my_ab = 0;
+                unsigned cum = inc - loc;
+                if (cum < (unsigned)rem && (unsigned)rem <= inc) {
+#pragma unroll
+                    for (int k = 1; k <= 8; ++k) {
+                        const unsigned h = ws.bins[d_hi - k];
+                        if (my_d < 0 && cum < (unsigned)rem && (unsigned)rem <= cum + h) {
+                            my_d = d_hi - k;
+                            my_ab = cum;
+                        }
+                        cum += h;
+                    }
+                }
+                const unsigned w2 = __ballot_sync(0xFFFFFFFFu, my_d >= 0);
+                const int s2 = __ffs(w2) - 1;
+                prefix |= (uint32_t)__shfl_sync(0xFFFFFFFFu, my_d, s2) << shift;
+                rem -= (int)__shfl_sync(0xFFFFFFFFu, my_ab, s2);
+                __syncwarp();
+            }
+            // prefix is the threshold key; take its first rem equal keys in entry order
+            // (order within a step: lane, then c)
+            int cnt = 0;
+            bool found = false;
+            for (int i = 0; i < nsteps && !found; ++i) {
+                uint32_t k[4];
+                load4(i, k);
+                int mine = 0;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) mine += (4 * (i * 32 + lane) + c < n && k[c] == prefix) ? 1 : 0;
+                int inc = mine;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int v = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+                    if (lane >= o) inc += v;
+                }
+                const int tot = __shfl_sync(0xFFFFFFFFu, inc, 31);
+                if (cnt + tot >= rem) {
+                    // the lane holding the rem-th equal key of this step
+                    int r = cnt + inc - mine;   // equal keys before this lane's
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int e = 4 * (i * 32 + lane) + c;
+                        if (e < n && k[c] == prefix) {
+                            ++r;
+                            if (r == rem) ws.thr = (unsigned long long)e;
+                        }
+                    }
+                    found = true;
+                }
+                cnt += tot;
+            }
+            __syncwarp();
+            const uint32_t es = (uint32_t)ws.thr;
+            T = ((unsigned long long)prefix << 32) | (unsigned long long)(0xFFFFFFFFu - es);
+        }
+    }
+    // ---- emit the selected entries in ascending order
+    int base = 0;
+    for (int i = 0; i < nsteps; ++i) {
+        uint32_t k[4];
+        load4(i, k);
+        bool sel[4];
+        int mine = 0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int e = 4 * (i * 32 + lane) + c;
+            sel[c] = e < n && (((unsigned long long)k[c] << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)e)) >= T;
+            mine += sel[c] ? 1 : 0;
+        }
+        int inc = mine;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+            if (lane >= o) inc += v;
+        }
+        int pos = base + inc - mine;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            if (sel[c]) {
+                idx_row[pos] = 4 * (i * 32 + lane) + c;
+                if (score_row) score_row[pos] = key_to_float(k[c]);
+                ++pos;
+            }
+        }
+        base += __shfl_sync(0xFFFFFFFFu, inc, 31);
+    }
+    for (int r = base + lane; r < topk; r += 32) {
+        idx_row[r] = -1;
+        if (score_row) score_row[r] = __int_as_float(0x7fc00000);
+    }
+}
 
 // ------------------------------------------------------------------ host side
 bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint32_t box_rows) {
@@ -752,9 +1292,15 @@ int sm_count() {
 struct Plan {
     int qb;
     int n_split;
-    bool keys;   // split decode rows: the indexer writes every visible entry's key, then
-                 // index_select_kernel selects (rows with at most kSelMax visible entries)
+    bool keys;   // the indexer writes every visible entry's score key, then index_select_kernel
+                 // selects (rows with at most kSelMax visible entries): split decode rows, and
+                 // prefill calls through the persistent key stream when the keys fit kKeysCap
+    int sel;     // selection kernel: rows of <= 2048 (0: one warp per row), 4096 (1), 16384 (2) entries
 };
+
+// the largest key workspace a prefill call takes (4 bytes per query row and entry); larger
+// calls keep the per-block candidate buffers
+constexpr size_t kKeysCap = (size_t)2 << 30;
 
 Plan plan(int64_t B, int64_t S_q, int64_t q_pos0, int64_t P, int ratio, int topk) {
     Plan p;
@@ -770,14 +1316,18 @@ Plan plan(int64_t B, int64_t S_q, int64_t q_pos0, int64_t P, int ratio, int topk
     if (ns > 16) ns = 16;
     while (ns > 1 && (int64_t)pow2_ceil((int)(ns * topk)) > 8192) --ns;
     p.n_split = (int)(ns < 1 ? 1 : ns);
-    p.keys = p.n_split > 1 && p.qb == 1 && n_visible(q_pos0 + S_q - 1, ratio, P) <= kSelMax;
+    const int64_t nv_max = n_visible(q_pos0 + S_q - 1, ratio, P);
+    const bool decode_keys = p.n_split > 1 && p.qb == 1;
+    const bool prefill_keys = p.n_split == 1 && p.qb == 4 && (size_t)B * S_q * key_pitch(P) * 4 <= kKeysCap;
+    p.keys = (decode_keys || prefill_keys) && nv_max <= kSelMax;
+    p.sel = nv_max <= kWsMax ? 0 : (nv_max <= 4096 ? 1 : 2);
     return p;
 }
 
 template <int QB>
 csa_status_t launch(const CUtensorMap &mk, const CUtensorMap &mq, const __nv_bfloat16 *w, int64_t B,
                     int64_t S_q, int64_t q_pos0, int64_t P, int ratio, int topk, int n_split, int32_t *idx,
-                    float *scores_opt, unsigned long long *partial, unsigned long long *keys_out,
+                    float *scores_opt, unsigned long long *partial, uint32_t *keys_out,
                     cudaStream_t st) {
     using C = Cfg<QB>;
     const int64_t n_qb = B * ((S_q + QB - 1) / QB);
@@ -807,13 +1357,26 @@ static size_t partial_bytes(const Plan &p, int64_t B, int64_t S_q, int topk) {
 }
 
 static size_t keys_bytes(int64_t B, int64_t S_q, int64_t P) {
-    return ((size_t)B * S_q * P * sizeof(unsigned long long) + 255) & ~(size_t)255;
+    return ((size_t)B * S_q * key_pitch(P) * sizeof(uint32_t) + 255) & ~(size_t)255;
+}
+
+template <int T, int PER>
+csa_status_t launch_select(const uint32_t *keys, int64_t rows, int64_t P, int topk, int32_t *idx,
+                           float *scores_opt, int64_t S_q, int64_t q_pos0, int ratio, cudaStream_t st) {
+    using SC = SelCfg<T, PER>;
+    auto kern = index_select_kernel<T, PER>;
+    ensure_smem((const void *)kern, SC::kSmem);
+    const cudaError_t le = launch_dependent(kern, dim3((unsigned)rows), dim3(T), SC::kSmem, st, 1, keys, P, topk,
+                                            idx, scores_opt, S_q, q_pos0, ratio);
+    CSA_REQUIRE(le == cudaSuccess, CSA_ERR_CUDA, "csa_index_topk select: launch failed: %s", cudaGetErrorString(le));
+    CSA_CHECK_LAUNCH("csa_index_topk select");
+    return CSA_OK;
 }
 
 size_t index_tc_workspace(int64_t B, int64_t S_q, int64_t q_pos0, int64_t P, int ratio, int topk) {
     Plan p = plan(B, S_q, q_pos0, P, ratio, topk);
+    if (p.keys) return keys_bytes(B, S_q, P);   // every visible entry's score key per row
     if (p.n_split <= 1) return 0;
-    if (p.keys) return keys_bytes(B, S_q, P);   // every visible entry's key per row
     return partial_bytes(p, B, S_q, topk);      // candidates per (row, range)
 }
 
@@ -826,30 +1389,52 @@ csa_status_t index_tc(const void *qI, const void *w, const void *kI, int64_t B, 
     Plan p = plan(B, S_q, q_pos0, P, ratio, topk);
     CSA_REQUIRE(make_map(&mq, qI, (uint64_t)B * S_q * kHI, (uint32_t)(p.qb * 64)), CSA_ERR_CUDA,
                 "csa_index_topk: cannot encode the q_I tensor map");
-    unsigned long long *partial = nullptr, *keys = nullptr;
-    if (p.n_split > 1) {
+    unsigned long long *partial = nullptr;
+    uint32_t *keys = nullptr;
+    if (p.keys || p.n_split > 1) {
         const size_t need = p.keys ? keys_bytes(B, S_q, P) : partial_bytes(p, B, S_q, topk);
         CSA_REQUIRE(workspace && workspace_bytes >= need, CSA_ERR_WORKSPACE,
                     "csa_index_topk: workspace of %zu B given, %zu B needed", workspace_bytes, need);
-        (p.keys ? keys : partial) = reinterpret_cast<unsigned long long *>(workspace);
+        if (p.keys)
+            keys = reinterpret_cast<uint32_t *>(workspace);
+        else
+            partial = reinterpret_cast<unsigned long long *>(workspace);
     }
     csa_status_t r;
     const __nv_bfloat16 *wb = reinterpret_cast<const __nv_bfloat16 *>(w);
-    if (p.qb == 4)
+    if (p.keys && p.qb == 4) {
+        // prefill key stream: one persistent CTA per SM at most
+        const int64_t n_qb = B * ((S_q + 3) / 4);
+        const int grid = (int)(n_qb < sm_count() ? n_qb : sm_count());
+        ensure_smem((const void *)index_keys_kernel, kKsSmem);
+        const cudaError_t le = launch_dependent(index_keys_kernel, dim3((unsigned)grid), dim3(KsCfg::kThreads),
+                                                kKsSmem, st, 1, mk, mq, wb, B, S_q, q_pos0, P, ratio, keys);
+        CSA_REQUIRE(le == cudaSuccess, CSA_ERR_CUDA, "csa_index_topk: launch failed: %s", cudaGetErrorString(le));
+        CSA_CHECK_LAUNCH("csa_index_topk keys");
+        r = CSA_OK;
+    } else if (p.qb == 4) {
         r = launch<4>(mk, mq, wb, B, S_q, q_pos0, P, ratio, topk, p.n_split, idx, scores_opt, partial, nullptr, st);
-    else
+    } else {
         r = launch<1>(mk, mq, wb, B, S_q, q_pos0, P, ratio, topk, p.n_split, idx, scores_opt, partial, keys, st);
-    if (r != CSA_OK || p.n_split <= 1) return r;
-    if (p.keys) {
-        ensure_smem((const void *)index_select_kernel, kSelSmem);
-        const cudaError_t le = launch_dependent(index_select_kernel, dim3((unsigned)(B * S_q)), dim3(kSelThreads),
-                                                kSelSmem, st, 1, (const unsigned long long *)keys, P, topk, idx,
-                                                scores_opt, S_q, q_pos0, ratio);
-        CSA_REQUIRE(le == cudaSuccess, CSA_ERR_CUDA, "csa_index_topk select: launch failed: %s",
-                    cudaGetErrorString(le));
-        CSA_CHECK_LAUNCH("csa_index_topk select");
-        return CSA_OK;
     }
+    if (r != CSA_OK) return r;
+    if (p.keys) {
+        if (p.sel == 0) {
+            const int64_t rows = B * S_q;
+            ensure_smem((const void *)index_select_warp_kernel, kWsSmem);
+            const cudaError_t le = launch_dependent(index_select_warp_kernel,
+                                                    dim3((unsigned)((rows + kWsWarps - 1) / kWsWarps)),
+                                                    dim3(kWsWarps * 32), kWsSmem, st, 1, (const uint32_t *)keys, P,
+                                                    topk, idx, scores_opt, rows, S_q, q_pos0, ratio);
+            CSA_REQUIRE(le == cudaSuccess, CSA_ERR_CUDA, "csa_index_topk select: launch failed: %s",
+                        cudaGetErrorString(le));
+            CSA_CHECK_LAUNCH("csa_index_topk select");
+            return CSA_OK;
+        }
+        if (p.sel == 1) return launch_select<512, 8>(keys, B * S_q, P, topk, idx, scores_opt, S_q, q_pos0, ratio, st);
+        return launch_select<1024, 16>(keys, B * S_q, P, topk, idx, scores_opt, S_q, q_pos0, ratio, st);
+    }
+    if (p.n_split <= 1) return r;
     const int total = p.n_split * topk;
     const size_t smem = (size_t)(pow2_ceil(total) + pow2_ceil(topk)) * 8 + 256 * 4 + sizeof(Misc) +
                         (size_t)((P + 31) / 32) * 4;

@@ -262,6 +262,36 @@ def test_index_all_ties_take_lowest_entries(S_q, q_pos0, P, topk):
         assert idx[0, i].tolist() == want and idx[1, i].tolist() == want, i
 
 
+@pytest.mark.parametrize("B,S_q,q_pos0,P,topk", [(1, 1200, 12000, 3001, 512), (2, 600, 40000, 9003, 1024),
+                                                 (1, 1201, 4947, 1537, 512)])
+def test_index_prefill_key_stream_parity(B, S_q, q_pos0, P, topk):
+    """Prefill-sized calls go through the persistent key stream and a selection kernel
+    sized by the longest row: rows of up to 4096 and 16384 visible entries (block
+    selects), and a row-length ramp up to 1537 entries (one warp per row) with an odd P,
+    so the key rows are padded.  Sampled rows against the oracle."""
+    g = torch.Generator().manual_seed(S_q * 7 + P)
+    q_I = (torch.randn((B, S_q, 64, 128), generator=g) * 0.5).to(torch.bfloat16)
+    w = torch.randn((B, S_q, 64), generator=g).to(torch.bfloat16)
+    k_I = torch.randn((B, P, 128), generator=g).to(torch.bfloat16)
+    idx, scores = csa.csa_index_topk(q_I.to(DEV), w.to(DEV), k_I.to(DEV), q_pos0, 4, topk, want_scores=True)
+    assert csa.csa_index_topk_workspace_bytes(B, S_q, q_pos0, P, 64, 128, 4, topk) > 0
+    torch.cuda.synchronize()
+    rows = sorted(random.Random(P).sample(range(S_q), 12) + [0, S_q - 1])
+    tpos = np.asarray(rows, dtype=np.int64) + q_pos0
+    sc = oracle.index_scores(to_np(q_I[:, rows]), to_np(w[:, rows]), to_np(k_I), tpos, 4)
+    o_idx, _ = oracle.topk(sc, tpos, 4, topk)
+    g_idx = idx.cpu().numpy()[:, rows]
+    g_sc = scores.cpu().numpy()[:, rows].astype(np.float64)
+    kk = [min(topk, oracle.n_visible(int(t), 4, P)) for t in tpos]
+    for b in range(B):
+        check_topk(g_idx[b], o_idx[b], sc[b], kk)
+        for r in range(len(rows)):
+            assert (np.diff(g_idx[b, r, :kk[r]]) > 0).all(), "row %d not in ascending order" % rows[r]
+        valid = g_idx[b] >= 0
+        ref = np.where(valid, np.take_along_axis(sc[b], np.maximum(g_idx[b], 0), axis=1), 0.0)
+        assert rel_err(np.where(valid, g_sc[b], 0.0), ref) <= TOL["bf16"] * 0.05
+
+
 def test_no_kernel_gave_up():
     import sparse_attention_14_b200 as csa
     spec = MID[1]
