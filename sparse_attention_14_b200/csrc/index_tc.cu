@@ -1013,14 +1013,14 @@ __global__ void __launch_bounds__(T) index_select_kernel(
 // Rows of at most 2048 visible entries: one warp per row, no block-wide barrier.  The
 // row's 32-bit score keys are copied into the warp's shared memory (16-byte async copies);
 // every pass reads four consecutive keys per lane and step (entries e = 4*(i*32 + lane) + c).
-// The scores are binned by value between the row's min and max into 1024 bins (a monotone
+// The scores are binned by value between the row's min and max into 512 bins (a monotone
 // map); the bin holding the k-th largest key is found from the bin counts.  A bin of at
 // most 64 keys is ranked by counting on the 64-bit keys (score key, complemented entry
 // index).  A crowded bin falls back to an MSB-first radix select on its 32-bit keys (four
 // 8-bit passes, exact), and the equal keys at the threshold are taken in ascending entry
 // order.  Either way the threshold T is one row key, and exactly k keys are >= T; they are
 // written in ascending entry order.
-constexpr int kWsWarps = 4, kWsBins = 1024, kWsSub = 64;
+constexpr int kWsWarps = 4, kWsBins = 512, kWsSub = 64;
 constexpr int kWsMax = 2048;   // entries per row
 struct WsWarp {
     uint4 k4[kWsMax / 4];                // the row's keys
@@ -1047,10 +1047,14 @@ __global__ void __launch_bounds__(kWsWarps * 32) index_select_warp_kernel(
     float *score_row = scores_opt ? scores_opt + row * (int64_t)topk : nullptr;
     const int nsteps = (n + 127) >> 7;   // steps of 32 lanes x 4 keys
 
-    // the row's keys (the tail of the last 16-byte piece is never read as a key)
+    // the row's keys, then 0 up to the end of the last step: a 0 key (a NaN score) leaves
+    // the min and max alone, falls into bin 0 (its count is taken back) and is never
+    // selected when n > topk (a real key is never 0: scores are not NaN)
     for (int v = lane; v < (n + 3) >> 2; v += 32) cp_async16(smem_u32(&ws.k4[v]), kr + 4 * v, 16u);
     cp_async_commit();
     asm volatile("cp.async.wait_group 0;" ::: "memory");
+    uint32_t *ks = reinterpret_cast<uint32_t *>(ws.k4);
+    for (int e = n + lane; e < nsteps * 128; e += 32) ks[e] = 0u;
     __syncwarp();
     auto load4 = [&](int i, uint32_t k[4]) {
         const uint4 v = ws.k4[i * 32 + lane];
@@ -1068,11 +1072,9 @@ __global__ void __launch_bounds__(kWsWarps * 32) index_select_warp_kernel(
             load4(i, k);
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                if (4 * (i * 32 + lane) + c < n) {
-                    const float f = key_to_float(k[c]);
-                    lo = fminf(lo, f);
-                    hi = fmaxf(hi, f);
-                }
+                const float f = key_to_float(k[c]);
+                lo = fminf(lo, f);
+                hi = fmaxf(hi, f);
             }
         }
 #pragma unroll
@@ -1093,9 +1095,10 @@ __global__ void __launch_bounds__(kWsWarps * 32) index_select_warp_kernel(
             uint32_t k[4];
             load4(i, k);
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
-                if (4 * (i * 32 + lane) + c < n) atomicAdd(&ws.bins[bin_of(k[c])], 1u);
+            for (int c = 0; c < 4; ++c) atomicAdd(&ws.bins[bin_of(k[c])], 1u);
         }
+        __syncwarp();
+        if (lane == 0) ws.bins[0] -= (unsigned)(nsteps * 128 - n);   // the padding
         __syncwarp();
         // lane l owns bins [kWsBins - 32(l+1), kWsBins - 32l), counted from the top
         constexpr int BPL = kWsBins / 32;
