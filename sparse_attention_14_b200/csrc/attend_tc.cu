@@ -93,10 +93,10 @@ struct Small {
     float inv_l[kH];
 };
 
-// Prefill: CTA c takes the contiguous work items [start[c], start[c+1]), split so that each
-// CTA gets about the same number of key tiles.  Consecutive queries then run on one CTA
-// (their windows overlap in all but one row and their selected entries largely coincide,
-// which L2 serves).  start[0] < 0: work items strided over the grid (decode-sized calls).
+// CSA prefill with few queries per CTA: CTA c takes the contiguous work items
+// [start[c], start[c+1]), split so that each CTA gets about the same number of key tiles;
+// consecutive queries then run on one CTA.  start[0] < 0: work items strided over the grid
+// (longer prefills, HCA, decode-sized calls).
 constexpr int kMaxCtas = 160;
 struct CtaRanges {
     int32_t start[kMaxCtas + 1];
@@ -1208,7 +1208,11 @@ csa_status_t attend_tc(const AttendArgs &a, cudaStream_t st) {
     if (grid > kMaxCtas) grid = kMaxCtas;
     CtaRanges ranges;
     ranges.start[0] = -1;
-    if (!decode && nw > grid) {
+    // measured: contiguous runs sped CSA up at 55 queries per CTA (S = 8192: 1.218 -> 1.184
+    // ms) but slowed it at 885 (S = 131072: 19.1 -> 20.7 ms) and HCA at 443 and 885 (+4 %,
+    // +3 %), where queries strided over the grid keep every CTA inside one band of the
+    // sequence
+    if (!decode && nw > grid && a.mode == 0 && nw <= 64 * (int64_t)grid) {
         // key tiles per query with the kernel's geometry (every idx value assumed valid)
         std::vector<int64_t> pre((size_t)a.S_q + 1, 0);
         for (int64_t i = 0; i < a.S_q; ++i) {
