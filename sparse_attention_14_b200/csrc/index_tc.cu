@@ -761,7 +761,9 @@ __global__ void __launch_bounds__(KsCfg::kThreads, 1) index_keys_kernel(
             uint32_t *krow = keys_out + (b * S_q + i0 + qa) * key_pitch(P);
             for (int t = 0; t < n_tiles; ++t, ++it) {
                 const uint32_t acc = it & 1u;
-                if (!mbar_wait(&ms.tfull[acc], (it >> 1) & 1u)) {
+                // the warp leaves together (its lanes meet again at __syncwarp below); other
+                // warps find out at the next block's vote, after their own bounded waits
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait(&ms.tfull[acc], (it >> 1) & 1u))) {
                     ok = false;
                     break;
                 }
