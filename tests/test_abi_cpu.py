@@ -153,3 +153,33 @@ def test_binding_raises_without_device_tensors(lib):
     x = torch.zeros(1, 8, 64)
     with pytest.raises(ValueError):
         csa.csa_compress(x, x, 4, True)
+
+
+def _ws_index(B, S_q, q_pos0, P, topk, dtype=None):
+    import torch
+    return csa.csa_index_topk_workspace_bytes(B, S_q, q_pos0, P, 64, 128, 4, topk,
+                                              dtype or torch.bfloat16)
+
+
+def test_index_workspace_plan(lib):
+    """The indexer's workspace query, host logic only: one row of 32-bit score keys per
+    query (pitch round_up(P, 4), the total rounded up to 256 bytes) whenever every row has
+    at most 16384 visible entries -- prefill calls whose key rows take at most 2 GiB and
+    split decode calls -- else candidates (decode) or none (prefill)."""
+    import torch
+    up = lambda n: (n + 255) // 256 * 256
+    # S=8192 prefill, P=2048: 8192 rows of 2048 keys
+    assert _ws_index(1, 8192, 0, 2048, 512) == 8192 * 2048 * 4
+    # odd P: rows padded to a multiple of 4 keys
+    assert _ws_index(2, 603, 0, 150, 64) == up(2 * 603 * 152 * 4)
+    # rows longer than 16384 visible entries keep the shared-memory candidates: no workspace
+    assert _ws_index(1, 131072, 0, 32768, 512) == 0
+    # key rows above 2 GiB (65536 rows of 16384 keys = 4 GiB): candidates, no workspace
+    assert _ws_index(1, 65536, 0, 16384, 512) == 0
+    # decode, 64 rows at 65536 cached tokens: split over entry ranges, keys of every entry
+    assert _ws_index(64, 1, 65535, 16384, 512) == 64 * 16384 * 4
+    # decode rows beyond 16384 visible entries: per-range candidates (64-bit keys)
+    ws = _ws_index(64, 1, 4 * 20000 - 1, 20000, 512)
+    assert ws > 0 and ws % (64 * 512 * 8) == 0
+    # the general (fp32) path needs none
+    assert _ws_index(1, 8192, 0, 2048, 512, torch.float32) == 0
