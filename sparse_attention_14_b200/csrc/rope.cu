@@ -129,6 +129,73 @@ __global__ void __launch_bounds__(kRopeThreads, 4) rope_any_kernel(const T *x, T
     }
 }
 
+// bf16 rows in groups that share a position (the indexer queries: the H_I heads of a query):
+// a warp takes one group at a time, its lanes = (row offset, 16-byte vector column), so a
+// lane keeps one column's angles for the whole group and the angles are computed once per
+// group and column instead of once per row.  Each warp access covers 32/np rows x np
+// contiguous vectors.
+template <int NP>
+__global__ void __launch_bounds__(kRopeThreads) rope_group_kernel(const __nv_bfloat16 *x, __nv_bfloat16 *out,
+                                                                  int64_t rows, int D, int64_t pos0, int64_t group,
+                                                                  int64_t period, int64_t step, RopeTable rope,
+                                                                  int p0) {
+    __shared__ uint64_t turn_s[kMaxRopePairs];
+    stage_turns(rope, turn_s, threadIdx.x, kRopeThreads);
+    __syncthreads();
+    constexpr int RPI = 32 / NP;                 // rows per warp access
+    constexpr int U = 8;                          // accesses in flight per lane
+    const int lane = threadIdx.x & 31;
+    const int v = p0 + lane % NP;                 // this lane's vector column
+    const int d0 = v * 8;
+    const int rs = lane / NP;                     // this lane's row offset inside an access
+    const bool rot = d0 + 8 > rope.first;
+    const int64_t n_groups = (rows + group - 1) / group;
+    const int64_t warps = (int64_t)gridDim.x * (kRopeThreads / 32);
+    const uint4 *xv = reinterpret_cast<const uint4 *>(x);
+    uint4 *ov = reinterpret_cast<uint4 *>(out);
+    const int64_t vrow = D / 8;
+    for (int64_t gi = (int64_t)blockIdx.x * (kRopeThreads / 32) + (threadIdx.x >> 5); gi < n_groups; gi += warps) {
+        // the column's angles at this group's position
+        float cs[4], sn[4];
+        if (rot) {
+            const int64_t pos = pos0 + (gi % period) * step;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int d = d0 + 2 * c;
+                cs[c] = 1.f;
+                sn[c] = 0.f;
+                if (d >= rope.first) rope_cs(pos, turn_s[(d - rope.first) >> 1], &cs[c], &sn[c]);
+            }
+        }
+        const int64_t r_begin = gi * group, r_end = r_begin + group < rows ? r_begin + group : rows;
+        for (int64_t r0 = r_begin + rs; r0 < r_end; r0 += (int64_t)RPI * U) {
+            uint4 w[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t r = r0 + (int64_t)u * RPI;
+                if (r < r_end) w[u] = xv[r * vrow + v];
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t r = r0 + (int64_t)u * RPI;
+                if (r >= r_end) continue;
+                if (rot) {
+                    __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&w[u]);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        if (d0 + 2 * c >= rope.first) {
+                            const float2 f = __bfloat1622float2(h[c]);
+                            const float w0 = f.x, w1 = f.y;
+                            h[c] = __floats2bfloat162_rn(w0 * cs[c] - w1 * sn[c], w0 * sn[c] + w1 * cs[c]);
+                        }
+                    }
+                }
+                ov[r * vrow + v] = w[u];
+            }
+        }
+    }
+}
+
 }  // namespace
 }  // namespace csa
 
@@ -169,6 +236,21 @@ extern "C" csa_status_t csa_rope_rows(const void *x, void *out, int64_t rows, in
     const int64_t cap = (int64_t)device_sm_count() * 8;
     const int64_t blocks = want < cap ? want : cap;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (dtype == CSA_BF16 && (np == 8 || np == 16) && group >= 32 / np && group % (32 / np) == 0) {
+        // groups of rows at one position (the indexer queries' heads): angles once per group
+        const int p0 = inplace ? rope.first / 8 : 0;
+        const int64_t n_groups = ceil_div(rows, group);
+        const int64_t gb = ceil_div(n_groups, (int64_t)(kRopeThreads / 32));
+        const unsigned grid = (unsigned)(gb < cap ? gb : cap);
+        if (np == 8)
+            rope_group_kernel<8><<<grid, kRopeThreads, 0, st>>>((const __nv_bfloat16 *)x, (__nv_bfloat16 *)out, rows, D,
+                                                              pos0, group, period, step, rope, p0);
+        else
+            rope_group_kernel<16><<<grid, kRopeThreads, 0, st>>>((const __nv_bfloat16 *)x, (__nv_bfloat16 *)out, rows,
+                                                               D, pos0, group, period, step, rope, p0);
+        CSA_CHECK_LAUNCH("csa_rope_rows");
+        return CSA_OK;
+    }
     if (dtype == CSA_F32)
         rope_any_kernel<float><<<(unsigned)blocks, kRopeThreads, 0, st>>>(
             (const float *)x, (float *)out, rows, D, pos0, group, period, step, rope, inplace);

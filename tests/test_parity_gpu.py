@@ -449,6 +449,10 @@ ROPE_CASES = [  # name, dtype, shape, group, period, step, pos0, rope_dim, base
     ("k_I_bf16", torch.bfloat16, (2, 50, 128), 1, 50, 4, 0, 64, 160000.0),
     ("odd_f32", torch.float32, (3, 11, 40), 1, 33, 3, 7, 8, 10000.0),
     ("full_width_far_f32", torch.float32, (4, 16), 2, 2, 5, 2 ** 30, 16, 10000.0),
+    # groups of rows at one position (64 heads per query; 21 rows in groups of 4, the last
+    # one partial): the kernel that computes the angles once per group and column
+    ("q_I_h64_bf16", torch.bfloat16, (2, 37, 64, 128), 64, 37, 1, 4000, 64, 160000.0),
+    ("ragged_groups_bf16", torch.bfloat16, (3, 7, 128), 4, 5, 3, 11, 64, 10000.0),
 ]
 
 
