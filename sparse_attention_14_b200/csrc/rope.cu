@@ -14,7 +14,9 @@
 // The pass is HBM-bound: every row is read and written once (in place, only the vectors
 // holding rope channels).  A thread works on 16-byte-aligned vectors of 8 elements (8
 // bf16, or 8 fp32 as two loads); since D - R is even and a vector never splits a pair,
-// each thread rotates its own pairs.
+// each thread rotates its own pairs.  Rows in groups at one position (the queries' heads)
+// take rope_group_kernel, which evaluates each column's angles once per group; other rows
+// take rope_any_kernel.
 #include "common.cuh"
 
 namespace csa {
